@@ -1,0 +1,380 @@
+"""CPU oracle of the compressed-sparse-attention hot path (fp64, numpy).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library; it reads the same seeded storage-format inputs.
+
+It is a plain, slow, obviously correct restatement of what the method
+computes.  Every input is first decoded exactly to fp64 (bf16 bit patterns,
+E4M3 codes times their fp32 scale); every step then runs in fp64 with numpy
+reductions and ``@`` as the only library primitives.
+
+Sources (web pages; cited by page title and section):
+
+* "DeepSeek-V4.1-Flash, illustrated" (mxino.github.io/illustrations/
+  deepseek-v41-flash), Equation (1) figure: the compressor turns the projected
+  KV entries C_l and compression weights Z_l into pooled entries; ratio 1 is
+  the unpooled main-KV projection; non-overlapping pairs at ratio 2.
+* "Model architectures" atlas (llm-switchboard.icompaas.com/app/architectures),
+  "compressed KV" entry: CSA squeezes every m KV tokens into one entry with
+  learned compression weights, then runs top-k lightning-indexer selection
+  over the compressed entries plus a sliding window; HCA compresses harder and
+  runs dense attention over the short stream.  "Sliding-window attention"
+  entry: token t attends to the previous W tokens, rolling buffer.  "MLA"
+  entry: attention runs over the latent directly (K = V = latent).
+* Tech-report tour (astryx-dracula tech-report.tsx), chapter "Compressed
+  Sparse Attention 2": section "The indexer selects, SWA covers the rest"
+  (indexer query x indexer key scores main KV entries, top 512 per query, the
+  query attends to those entries together with the sliding-window KV; ratio 1
+  is the uncompressed special case); section "A simpler compressor" (no
+  overlap, no absolute position term, indexer K projected from main KV);
+  chapter "SWA Bounded Replay", section "Replay only the window" (keys in
+  [max(s, i-W+1), i]).
+
+Readings where the pages are silent or garbled (each listed in the design doc):
+
+* Equation (1)'s body is not extracted.  Reading: within each block of m
+  consecutive tokens the pooling weights are a softmax over the block's m
+  gate logits Z, taken separately for every channel, and the entry is the
+  weighted sum of the block's C rows.  A partial trailing block emits nothing.
+* Indexer score: s_j = sum_h w_h * ReLU(q_h . k_j), no softmax, no scale.
+* Top-k order: score descending, index ascending on exact ties (-0 == +0).
+* One online softmax covers the selected (or all, for HCA) compressed entries,
+  the window keys, and a per-head sink logit that only adds exp(sink) to the
+  denominator.  Window and compressed entries are not de-duplicated.
+* A compressed block j is visible to a query at absolute position t iff its
+  last token (j+1)m-1 <= t, i.e. n_visible(t) = floor((t+1)/m).
+
+Parity unpinned: the exact form of Equation (1) is not printed on the pages;
+only the invariants the pages fix (ratio 1 = unpooled copy, non-overlapping
+blocks, no positional term) and closed forms of the per-channel softmax
+reading pin the compressor.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+E4M3_MAX = 448.0
+
+
+# ===========================================================================
+# storage formats
+# ===========================================================================
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit pattern -> value: the upper 16 bits of an IEEE binary32."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _e4m3_table() -> np.ndarray:
+    """Value of every E4M3 (OCP 'fn' variant) code, from the format definition.
+
+    Layout s eeee mmm, exponent bias 7.  e == 0: subnormal m/8 * 2^-6.
+    e == 15 and m == 7: NaN (no infinities).  Otherwise (1 + m/8) * 2^(e-7).
+    """
+    t = np.empty(256, np.float64)
+    for code in range(256):
+        s = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            t[code] = np.nan
+        elif e == 0:
+            t[code] = s * (m / 8.0) * 2.0 ** -6
+        else:
+            t[code] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return t
+
+
+E4M3_VALUES = _e4m3_table()
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    return E4M3_VALUES[np.asarray(codes, dtype=np.uint8)]
+
+
+def decode(data: np.ndarray, dtype: str, scale: np.ndarray | None = None, group: int = 0) -> np.ndarray:
+    """Exact fp64 value of a stored tensor (codes times group scale for FP8)."""
+    if dtype == "f32":
+        return np.asarray(data, dtype=np.float32).astype(np.float64)
+    if dtype == "bf16":
+        return bf16_to_f64(data)
+    if dtype == "fp8":
+        v = e4m3_to_f64(data)
+        sc = np.repeat(np.asarray(scale, np.float64), group, axis=-1)
+        return v * sc
+    raise ValueError(dtype)
+
+
+def decode_stored(t) -> np.ndarray:
+    """Decode a ``workloads.Stored`` (duck-typed: data, dtype, scale, group)."""
+    return decode(t.data, t.dtype, t.scale, t.group)
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest E4M3 value, ties to even code,
+    saturating at +-448 (the largest finite value).  Returns codes (uint8)."""
+    x = np.asarray(x, np.float64)
+    finite = E4M3_VALUES[:127]                  # codes 0x00..0x7E, ascending
+    mag = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.searchsorted(finite, mag, side="left")   # first value >= mag
+    hi = np.minimum(hi, 126)
+    lo = np.maximum(hi - 1, 0)
+    d_hi = finite[hi] - mag
+    d_lo = mag - finite[lo]
+    pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (lo % 2 == 0))
+    code = np.where(pick_lo, lo, hi).astype(np.uint8)
+    code = np.where(mag == finite[hi], hi, code).astype(np.uint8)
+    neg = (x < 0) & (code != 0)
+    return (code | np.where(neg, 0x80, 0)).astype(np.uint8)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (8 significant bits), ties
+    to even.  Normal range only, which covers every value the path stores."""
+    x = np.asarray(x, np.float64)
+    f, e = np.frexp(x)                      # x = f * 2^e, 0.5 <= |f| < 1
+    return np.ldexp(np.rint(f * 256.0), e - 8)
+
+
+def round_to_storage(x: np.ndarray, dtype: str, group: int = 0) -> np.ndarray:
+    """Value that remains after storing fp64 ``x`` in format ``dtype``:
+    fp32 (IEEE round-to-nearest-even cast), bf16 (``bf16_round``) or E4M3
+    with a per-group scale (``quantize_groups``, then decoded)."""
+    if dtype == "f32":
+        return np.asarray(x, np.float64).astype(np.float32).astype(np.float64)
+    if dtype == "bf16":
+        return bf16_round(x)
+    if dtype == "fp8":
+        codes, scale = quantize_groups(x, group)
+        return decode(codes, "fp8", scale, group)
+    raise ValueError(dtype)
+
+
+def quantize_groups(x: np.ndarray, group: int) -> tuple[np.ndarray, np.ndarray]:
+    """E4M3 storage of fp64 values: per ``group`` channels, scale = max|x|/448
+    (1.0 for an all-zero group), codes = RNE-saturating E4M3 of x/scale."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    g = x.reshape(x.shape[:-1] + (d // group, group))
+    amax = np.abs(g).max(axis=-1)
+    scale = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    codes = e4m3_round(g / scale[..., None]).reshape(x.shape)
+    return codes, scale
+
+
+# ===========================================================================
+# a1: the compressor
+# ===========================================================================
+def compress(C: np.ndarray, Z: np.ndarray, m: int) -> np.ndarray:
+    """Pool every m consecutive rows of C into one entry.
+
+    "DeepSeek-V4.1-Flash, illustrated", Equation (1) (C_l, Z_l rule) and the
+    atlas's "compressed KV" entry (every m KV tokens -> one entry with learned
+    compression weights); tech-report tour, "A simpler compressor"
+    (non-overlapping groups, no absolute positional term).
+
+    For block j and channel c:
+        a_i = exp(Z[i,c]) / sum_{i' in block j} exp(Z[i',c])
+        out[j,c] = sum_{i in block j} a_i * C[i,c]
+    computed with the block maximum subtracted before exp.  Rows after the
+    last complete block are ignored.  C, Z: [T][d] -> [T // m][d].
+    """
+    C = np.asarray(C, np.float64)
+    Z = np.asarray(Z, np.float64)
+    T, d = C.shape
+    n = T // m
+    Cb = C[: n * m].reshape(n, m, d)
+    Zb = Z[: n * m].reshape(n, m, d)
+    M = Zb.max(axis=1, keepdims=True)
+    e = np.exp(Zb - M)
+    a = e / e.sum(axis=1, keepdims=True)
+    return (a * Cb).sum(axis=1)
+
+
+def project_index_keys(C_hat: np.ndarray, w_ik: np.ndarray) -> np.ndarray:
+    """Indexer keys projected from main-KV entries: k_I = C_hat @ W_IK.
+
+    Tech-report tour, "A simpler compressor": CSA2 derives indexer K by
+    projecting main KV entries.  [n][d] @ [d][d_idx] -> [n][d_idx].
+    """
+    return np.asarray(C_hat, np.float64) @ np.asarray(w_ik, np.float64)
+
+
+# ===========================================================================
+# a2 / a3: lightning indexer and per-query top-k
+# ===========================================================================
+def n_visible(t: int | np.ndarray, m: int):
+    """Compressed blocks whose last token is at or before position t."""
+    return (np.asarray(t) + 1) // m
+
+
+def index_scores(q_idx: np.ndarray, w: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """Lightning-indexer scores of one query against ``keys``.
+
+    s_j = sum_h w_h * max(0, q_h . k_j).  Atlas, "Trained sparse attention"
+    entry (DSA: lightning indexer + top-k token selection) and "compressed
+    KV" entry; tech-report tour, "The indexer selects, SWA covers the rest".
+    q_idx [h][d_idx], w [h], keys [n][d_idx] -> [n].
+    """
+    dots = np.asarray(keys, np.float64) @ np.asarray(q_idx, np.float64).T   # [n][h]
+    return (np.maximum(dots, 0.0) * np.asarray(w, np.float64)[None, :]).sum(axis=1)
+
+
+def topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest scores: score descending, index ascending on
+    exact ties (-0 equals +0).  Fewer than k candidates: pad with -1.
+    Tech-report tour, "The indexer selects, SWA covers the rest"."""
+    s = np.asarray(scores, np.float64)
+    n = s.shape[0]
+    order = np.lexsort((np.arange(n), -s))
+    take = order[: min(k, n)]
+    out = np.full(k, -1, np.int64)
+    out[: take.shape[0]] = take
+    return out
+
+
+def boundary_gap(scores: np.ndarray, k: int) -> float:
+    """s_(k) - s_(k+1) of the sorted scores (inf when nothing is cut off)."""
+    s = np.sort(np.asarray(scores, np.float64))[::-1]
+    if k <= 0 or k >= s.shape[0]:
+        return math.inf
+    return float(s[k - 1] - s[k])
+
+
+# ===========================================================================
+# a4 / a5: sparse (or dense) attention + sliding window + sink, one softmax
+# ===========================================================================
+def window_positions(t: int, W: int, lo: int = 0) -> np.ndarray:
+    """Absolute key positions of the sliding window of a query at t.
+
+    Atlas, "Sliding-window attention" entry (token t sees the previous W
+    tokens); tech-report tour, "Replay only the window": a replay starting at
+    s restricts the keys to [max(s, i-W+1), i].
+    """
+    start = max(lo, t - W + 1, 0)
+    return np.arange(start, t + 1, dtype=np.int64) if W > 0 else np.zeros(0, np.int64)
+
+
+def attend(q: np.ndarray, entries: np.ndarray, win_k: np.ndarray, win_v: np.ndarray,
+           sink: np.ndarray | None, tau: float) -> tuple[np.ndarray, np.ndarray]:
+    """One softmax over compressed entries (K = V = entry), window keys and a
+    sink logit per head.
+
+    For head h:  l_j = tau q_h . e_j,  l_p = tau q_h . k_p,
+      M = max(sink_h, all l),  L = exp(sink_h - M) + sum exp(l - M),
+      out_h = (sum_j exp(l_j - M) e_j + sum_p exp(l_p - M) v_p) / L,
+      lse_h = M + log L.
+    q [h][d], entries [n][d], win_k / win_v [p][d], sink [h] or None.
+    With nothing to attend to and no sink: out = 0, lse = -inf.
+    """
+    q = np.asarray(q, np.float64)
+    keys = np.concatenate([np.asarray(entries, np.float64).reshape(-1, q.shape[1]),
+                           np.asarray(win_k, np.float64).reshape(-1, q.shape[1])], axis=0)
+    vals = np.concatenate([np.asarray(entries, np.float64).reshape(-1, q.shape[1]),
+                           np.asarray(win_v, np.float64).reshape(-1, q.shape[1])], axis=0)
+    h = q.shape[0]
+    logits = tau * (q @ keys.T)                             # [h][n+p]
+    s = np.full(h, -np.inf) if sink is None else np.asarray(sink, np.float64)
+    M = np.maximum(s, logits.max(axis=1) if logits.shape[1] else np.full(h, -np.inf))
+    out = np.zeros_like(q)
+    lse = np.full(h, -np.inf)
+    ok = np.isfinite(M)
+    if ok.any():
+        e = np.exp(logits[ok] - M[ok, None])
+        L = e.sum(axis=1) + np.exp(s[ok] - M[ok])
+        out[ok] = (e @ vals) / L[:, None]
+        lse[ok] = M[ok] + np.log(L)
+    return out, lse
+
+
+def sparse_swa_attention(q, kv_rows, idx, n_vis, swa_k, swa_v, swa_cap, t, W, sink, tau,
+                         swa_lo: int = 0):
+    """Attention of one query token (all heads) at absolute position t.
+
+    kv_rows: this request's compressed entries [cap][d] (fp64).
+    idx: selected entry indices (-1 = padding); None selects all n_vis
+         visible entries (the HCA branch, atlas "compressed KV" entry).
+    swa_k / swa_v: [swa_cap][d] ring, position p in slot p % swa_cap.
+    """
+    if idx is None:
+        sel = np.arange(n_vis, dtype=np.int64)
+    else:
+        sel = np.asarray(idx, np.int64)
+        sel = sel[sel >= 0]
+    ent = np.asarray(kv_rows, np.float64)[sel]
+    pos = window_positions(t, W, swa_lo)
+    slots = pos % swa_cap
+    return attend(q, ent, np.asarray(swa_k, np.float64)[slots], np.asarray(swa_v, np.float64)[slots],
+                  sink, tau)
+
+
+# ===========================================================================
+# a6: one decode step
+# ===========================================================================
+def decode_step(inp, tau: float = 1.0):
+    """One decode step for every request of a ``workloads.DecodeInputs``.
+
+    Tech-report tour, "Full, Reindex, and Reuse" (Full mode: compute main KV,
+    project indexer K, select a fresh top-k) and "The indexer selects, SWA
+    covers the rest".  Steps per request b with the new token at position t:
+      1. the token's SWA key/value enter ring slot t % swa_cap;
+      2. its C/Z row enters open-block slot t % m; if (t+1) % m == 0 the block
+         is pooled (``compress``) into entry (t+1)/m - 1, and its indexer key
+         is projected from it (``project_index_keys``);
+      3. scores of the n_visible(t) entries, top-k (skipped when dense);
+      4. one softmax over selected entries + window + sink.
+    The new entry and its indexer key are stored in the caches' formats
+    (``round_to_storage``) before they are scored and attended, as the
+    caches hold them in storage format.
+    Returns dict with out [B][h_q][d], lse [B][h_q], idx [B][k] (or None),
+    scores [B][n] and the new cache rows (fp64, before storage rounding).
+    """
+    wl = inp.wl
+    B, m, d = wl.batch, wl.m, wl.d
+    kv = decode_stored(inp.kv).copy()
+    kidx = decode_stored(inp.kidx).copy()
+    swa_k = decode_stored(inp.swa_k).copy()
+    swa_v = decode_stored(inp.swa_v).copy()
+    open_c = decode_stored(inp.open_c).copy()
+    open_z = decode_stored(inp.open_z).copy()
+    c_t, z_t = decode_stored(inp.c_t), decode_stored(inp.z_t)
+    k_t, v_t = decode_stored(inp.k_t), decode_stored(inp.v_t)
+    q, q_idx = decode_stored(inp.q), decode_stored(inp.q_idx)
+    w_ik = decode_stored(inp.w_ik)
+    outs, lses, idxs, scores, new_rows, new_keys = [], [], [], [], [], []
+    for b in range(B):
+        t = int(inp.pos[b])
+        swa_k[b, t % inp.swa_cap] = k_t[b]
+        swa_v[b, t % inp.swa_cap] = v_t[b]
+        open_c[b, t % m] = c_t[b]
+        open_z[b, t % m] = z_t[b]
+        if (t + 1) % m == 0:
+            j = (t + 1) // m - 1
+            row = compress(open_c[b], open_z[b], m)[0]
+            key = project_index_keys(row[None], w_ik)[0]
+            kv[b, j] = round_to_storage(row[None], inp.kv.dtype, inp.kv.group)[0]
+            kidx[b, j] = round_to_storage(key[None], inp.kidx.dtype, inp.kidx.group)[0]
+            new_rows.append(row)
+            new_keys.append(key)
+        nv = int(n_visible(t, m))
+        if wl.dense:
+            sel = None
+            s = None
+        else:
+            s = index_scores(q_idx[b], inp.w[b], kidx[b, :nv])
+            sel = topk(s, wl.topk)
+        o, l = sparse_swa_attention(q[b], kv[b], sel, nv, swa_k[b], swa_v[b], inp.swa_cap, t,
+                                    wl.window, inp.sink, tau)
+        outs.append(o)
+        lses.append(l)
+        idxs.append(sel)
+        scores.append(s)
+    return {
+        "out": np.stack(outs), "lse": np.stack(lses),
+        "idx": None if wl.dense else np.stack(idxs),
+        "scores": scores, "new_rows": new_rows, "new_keys": new_keys,
+    }

@@ -1,0 +1,377 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each test checks the oracle against something it does not compute: a library
+routine on a special case (torch's dtype casts, scaled_dot_product_attention,
+topk), a closed form, an invariant the pages state, a worked case of a
+printed formula (tests/golden/page_facts.json), or brute force on tiny
+inputs.  A plausible slip in the oracle (dropped term, wrong sign or index,
+transposed operand) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import csa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
+
+
+def _facts():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- formats
+def test_e4m3_table_matches_torch_cast():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = O.e4m3_to_f64(np.arange(256))
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(mine))
+    assert np.array_equal(ref[~nan], mine[~nan])
+    assert O.e4m3_to_f64(np.array([0x7E]))[0] == 448.0
+    assert O.e4m3_to_f64(np.array([0x38]))[0] == 1.0
+    assert O.e4m3_to_f64(np.array([0x01]))[0] == 2.0 ** -9
+
+
+def test_e4m3_round_matches_torch_cast():
+    g = np.random.default_rng(5)
+    x = np.concatenate([
+        g.standard_normal(20000) * 30, g.standard_normal(5000) * 0.01,
+        g.uniform(-460, 460, 5000),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(np.clip(x, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = O.e4m3_round(x.astype(np.float64))
+    # +0 / -0 codes may differ for values that round to zero; compare values
+    assert np.array_equal(O.e4m3_to_f64(ref), O.e4m3_to_f64(mine))
+
+
+def test_e4m3_round_ties_and_saturation():
+    v = O.e4m3_to_f64
+    r = lambda a: v(O.e4m3_round(np.array([a])))[0]
+    assert r(0.5 * 2 ** -9) == 0.0                # tie 0 | 2^-9 -> even (0)
+    assert r(1.5 * 2 ** -9) == 2 * 2 ** -9        # tie code1 | code2 -> code2
+    assert r(500.0) == 448.0 and r(-1e9) == -448.0
+    assert r(1.0 + 1 / 16) == 1.0                  # tie 1.0 | 1.125 -> 1.0 (even)
+    assert r(1.0 + 3 / 16) == 1.25                 # tie 1.125 | 1.25 -> 1.25 (even)
+
+
+def test_bf16_decode_and_round_match_torch():
+    g = np.random.default_rng(6)
+    x = (g.standard_normal(50000) * np.exp(g.uniform(-20, 20, 50000))).astype(np.float32)
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.bf16_to_f64(bits), ref)
+    assert np.array_equal(O.bf16_round(x.astype(np.float64)), ref)
+
+
+def test_quantize_groups_scale_and_error_bound():
+    g = np.random.default_rng(7)
+    x = g.standard_normal((13, 128))
+    codes, scale = O.quantize_groups(x, 64)
+    assert scale.shape == (13, 2)
+    amax = np.abs(x.reshape(13, 2, 64)).max(-1)
+    assert np.allclose(scale, amax / 448.0, rtol=0, atol=0)
+    deq = O.decode(codes, "fp8", scale, 64)
+    # E4M3 keeps 4 significant bits: relative error <= 2^-4, plus the
+    # subnormal step 2^-10 * scale near zero
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, np.repeat(scale, 64, -1) * 2.0 ** -10)
+    assert np.all(np.abs(deq - x) <= bound + 1e-15)
+    # the group maximum maps to exactly +-448
+    assert np.allclose(np.abs(deq).reshape(13, 2, 64).max(-1), amax, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- compressor
+def test_compress_ratio1_is_copy():
+    g = np.random.default_rng(1)
+    C, Z = g.standard_normal((37, 16)), g.standard_normal((37, 16)) * 5
+    assert np.array_equal(O.compress(C, Z, 1), C)
+
+
+def test_compress_constant_gate_is_block_mean():
+    g = np.random.default_rng(2)
+    C = g.standard_normal((24, 8))
+    Z = np.repeat(g.standard_normal((6, 1, 8)), 4, axis=1).reshape(24, 8)
+    ref = C.reshape(6, 4, 8).mean(axis=1)
+    assert np.allclose(O.compress(C, Z, 4), ref, rtol=0, atol=1e-14)
+
+
+def test_compress_m2_sigmoid_closed_form():
+    g = np.random.default_rng(3)
+    C, Z = g.standard_normal((20, 8)), g.standard_normal((20, 8)) * 3
+    c1, c2, z1, z2 = C[0::2], C[1::2], Z[0::2], Z[1::2]
+    sig = 1.0 / (1.0 + np.exp(-(z1 - z2)))
+    ref = sig * c1 + (1.0 - sig) * c2
+    assert np.allclose(O.compress(C, Z, 2), ref, rtol=0, atol=1e-14)
+
+
+def test_compress_dominant_gate_selects_row_per_channel():
+    g = np.random.default_rng(4)
+    C = g.standard_normal((8, 6))
+    Z = np.zeros((8, 6))
+    pick = g.integers(0, 4, size=(2, 6))
+    for j in range(2):
+        for c in range(6):
+            Z[j * 4 + pick[j, c], c] = 1000.0
+    out = O.compress(C, Z, 4)
+    for j in range(2):
+        for c in range(6):
+            assert out[j, c] == C[j * 4 + pick[j, c], c]
+
+
+def test_compress_gate_shift_invariance_and_tail():
+    g = np.random.default_rng(8)
+    C, Z = g.standard_normal((10, 5)), g.standard_normal((10, 5))
+    shift = np.repeat(g.standard_normal((2, 1, 5)) * 50, 4, axis=1).reshape(8, 5)
+    Z2 = Z.copy()
+    Z2[:8] += shift
+    Z2[8:] += 1e6  # rows of the partial trailing block are ignored
+    assert O.compress(C, Z, 4).shape == (2, 5)
+    assert np.allclose(O.compress(C, Z, 4), O.compress(C, Z2, 4), rtol=0, atol=1e-13)
+
+
+def test_compress_blocks_do_not_overlap():
+    """Golden: non-overlapping groups of m consecutive tokens."""
+    for case in _facts()["ratio_blocks"]["cases"]:
+        m, T = case["m"], case["T"]
+        g = np.random.default_rng(m * 100 + T)
+        C, Z = g.standard_normal((T, 3)), g.standard_normal((T, 3))
+        base = O.compress(C, Z, m)
+        assert base.shape[0] == len(case["blocks"])
+        for t in range(T):
+            C2 = C.copy()
+            C2[t] += 1.0
+            changed = np.nonzero(np.any(O.compress(C2, Z, m) != base, axis=1))[0].tolist()
+            expect = [j for j, blk in enumerate(case["blocks"]) if t in blk]
+            assert changed == expect
+
+
+def test_compress_brute_force_tiny():
+    g = np.random.default_rng(9)
+    m, n, d = 3, 4, 5
+    C, Z = g.standard_normal((m * n, d)), g.standard_normal((m * n, d))
+    out = O.compress(C, Z, m)
+    for j in range(n):
+        for c in range(d):
+            den = sum(math.exp(Z[j * m + i, c]) for i in range(m))
+            num = sum(math.exp(Z[j * m + i, c]) * C[j * m + i, c] for i in range(m))
+            assert abs(out[j, c] - num / den) < 1e-13
+
+
+def test_project_index_keys_identity_projection():
+    g = np.random.default_rng(10)
+    rows = g.standard_normal((7, 6))
+    assert np.array_equal(O.project_index_keys(rows, np.eye(6)), rows)
+    sel = np.zeros((6, 2))
+    sel[4, 0] = 1.0
+    sel[1, 1] = -2.0
+    assert np.array_equal(O.project_index_keys(rows, sel), np.stack([rows[:, 4], -2 * rows[:, 1]], 1))
+
+
+# ---------------------------------------------------------------- indexer
+def test_index_scores_single_head_is_relu_dot():
+    g = np.random.default_rng(11)
+    K, q = g.standard_normal((50, 16)), g.standard_normal((1, 16))
+    ref = torch.relu(torch.mv(torch.from_numpy(K), torch.from_numpy(q[0]))).numpy()
+    assert np.allclose(O.index_scores(q, np.ones(1), K), ref, rtol=0, atol=1e-13)
+
+
+def test_index_scores_brute_force_and_linearity():
+    g = np.random.default_rng(12)
+    K, q = g.standard_normal((9, 4)), g.standard_normal((3, 4))
+    w1, w2 = g.random(3), g.random(3)
+    s = O.index_scores(q, w1, K)
+    for j in range(9):
+        ref = 0.0
+        for h in range(3):
+            dot = sum(q[h, c] * K[j, c] for c in range(4))
+            ref += w1[h] * (dot if dot > 0 else 0.0)
+        assert abs(s[j] - ref) < 1e-13
+    assert np.allclose(O.index_scores(q, w1 + w2, K), s + O.index_scores(q, w2, K), atol=1e-13)
+
+
+def test_index_scores_all_negative_dots_are_exact_zero():
+    g = np.random.default_rng(13)
+    K = np.abs(g.standard_normal((20, 8)))
+    q = -np.abs(g.standard_normal((4, 8)))
+    assert np.all(O.index_scores(q, g.random(4), K) == 0.0)
+
+
+# ---------------------------------------------------------------- top-k
+def test_topk_matches_torch_on_distinct_scores():
+    g = np.random.default_rng(14)
+    s = g.standard_normal(1000)
+    ref = torch.topk(torch.from_numpy(s), 37).indices.numpy()
+    assert np.array_equal(O.topk(s, 37), ref)
+
+
+def test_topk_ties_lower_index_wins():
+    assert O.topk(np.zeros(10), 4).tolist() == [0, 1, 2, 3]
+    assert O.topk(np.array([0.0, -0.0, 0.0, -1.0]), 2).tolist() == [0, 1]
+    assert O.topk(np.array([1.0, 2.0, 2.0, 1.0, 2.0]), 2).tolist() == [1, 2]
+
+
+def test_topk_pads_when_fewer_candidates():
+    assert O.topk(np.array([3.0, 1.0, 2.0]), 5).tolist() == [0, 2, 1, -1, -1]
+    assert O.topk(np.zeros(0), 2).tolist() == [-1, -1]
+
+
+def test_topk_brute_force_definition():
+    g = np.random.default_rng(15)
+    s = np.round(g.standard_normal(60) * 2) / 2  # many exact ties
+    k = 17
+    chosen = set(O.topk(s, k).tolist())
+    for i in range(60):
+        rank = sum(1 for j in range(60) if s[j] > s[i] or (s[j] == s[i] and j < i))
+        assert (i in chosen) == (rank < k)
+
+
+# ---------------------------------------------------------------- attention
+def _sdpa(q, k, v, mask=None):
+    qt = torch.from_numpy(q)[None]
+    return torch.nn.functional.scaled_dot_product_attention(
+        qt, torch.from_numpy(k)[None], torch.from_numpy(v)[None], attn_mask=mask, scale=1.0)[0].numpy()
+
+
+def test_dense_no_window_no_sink_equals_sdpa():
+    g = np.random.default_rng(16)
+    q, E = g.standard_normal((8, 32)) * 0.3, g.standard_normal((50, 32))
+    out, lse = O.attend(q, E, np.zeros((0, 32)), np.zeros((0, 32)), None, 1.0)
+    assert np.allclose(out, _sdpa(q, E, E), rtol=0, atol=1e-12)
+    ref_lse = torch.logsumexp(torch.from_numpy(q @ E.T), dim=1).numpy()
+    assert np.allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_sink_is_an_extra_zero_value_key():
+    g = np.random.default_rng(17)
+    h, d = 4, 16
+    q, E = g.standard_normal((h, d)), g.standard_normal((30, d))
+    wk, wv = g.standard_normal((5, d)), g.standard_normal((5, d))
+    sink = g.standard_normal(h) * 2
+    out, _ = O.attend(q, E, wk, wv, sink, 0.7)
+    for i in range(h):
+        qa = np.concatenate([q[i] * 0.7, [1.0]])[None]
+        K = np.concatenate([np.concatenate([E, wk]), np.zeros((35, 1))], 1)
+        K = np.concatenate([K, np.concatenate([np.zeros(d), [sink[i]]])[None]])
+        V = np.concatenate([E, wv, np.zeros((1, d))])
+        assert np.allclose(out[i], _sdpa(qa, K, V)[0], rtol=0, atol=1e-12)
+
+
+def test_full_window_without_entries_is_causal_attention():
+    g = np.random.default_rng(18)
+    T, d, h = 12, 8, 3
+    q, K, V = g.standard_normal((T, h, d)), g.standard_normal((T, d)), g.standard_normal((T, d))
+    cap = 16
+    ring_k, ring_v = np.zeros((cap, d)), np.zeros((cap, d))
+    ring_k[np.arange(T) % cap], ring_v[np.arange(T) % cap] = K, V
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q.transpose(1, 0, 2)), torch.from_numpy(K)[None].expand(h, T, d),
+        torch.from_numpy(V)[None].expand(h, T, d), is_causal=True, scale=1.0).numpy()
+    for t in range(T):
+        out, _ = O.sparse_swa_attention(q[t], np.zeros((1, d)), np.zeros(0, np.int64), 0, ring_k, ring_v,
+                                        cap, t, W=T, sink=None, tau=1.0)
+        assert np.allclose(out, ref[:, t], rtol=0, atol=1e-12)
+
+
+def test_sliding_window_band_matches_masked_sdpa():
+    g = np.random.default_rng(19)
+    T, d, W = 20, 8, 5
+    q, K, V = g.standard_normal((T, 1, d)), g.standard_normal((T, d)), g.standard_normal((T, d))
+    cap = 8
+    for t in range(T):
+        ring_k, ring_v = np.zeros((cap, d)), np.zeros((cap, d))
+        for p in range(max(0, t - cap + 1), t + 1):
+            ring_k[p % cap], ring_v[p % cap] = K[p], V[p]
+        mask = torch.zeros(1, T, dtype=torch.bool)
+        mask[0, max(0, t - W + 1): t + 1] = True
+        ref = _sdpa(q[t], K, V, mask)
+        out, _ = O.sparse_swa_attention(q[t], np.zeros((1, d)), None, 0, ring_k, ring_v, cap, t, W, None, 1.0)
+        assert np.allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_window_rule_golden():
+    f = _facts()["window_rule"]
+    for c in f["cases"]:
+        pos = O.window_positions(c["i"], f["W"], c["s"])
+        assert pos[0] == c["first"] and pos[-1] == c["last"] and len(pos) == c["last"] - c["first"] + 1
+
+
+def test_split_merge_invariance():
+    g = np.random.default_rng(20)
+    q, E = g.standard_normal((6, 16)), g.standard_normal((40, 16))
+    z = np.zeros((0, 16))
+    o1, l1 = O.attend(q, E[:13], z, z, None, 1.0)
+    o2, l2 = O.attend(q, E[13:], z, z, None, 1.0)
+    o, l = O.attend(q, E, z, z, None, 1.0)
+    M = np.maximum(l1, l2)
+    a1, a2 = np.exp(l1 - M), np.exp(l2 - M)
+    assert np.allclose(o, (o1 * a1[:, None] + o2 * a2[:, None]) / (a1 + a2)[:, None], atol=1e-12)
+    assert np.allclose(l, M + np.log(a1 + a2), atol=1e-12)
+
+
+def test_selection_order_does_not_matter():
+    g = np.random.default_rng(21)
+    q, rows = g.standard_normal((4, 8)), g.standard_normal((30, 8))
+    idx = g.permutation(30)[:10]
+    ring = np.zeros((4, 8))
+    a = O.sparse_swa_attention(q, rows, idx, 30, ring, ring, 4, 0, 0, None, 1.0)[0]
+    b = O.sparse_swa_attention(q, rows, idx[::-1].copy(), 30, ring, ring, 4, 0, 0, None, 1.0)[0]
+    assert np.allclose(a, b, atol=1e-13)
+    # padding entries (-1) are ignored
+    c = O.sparse_swa_attention(q, rows, np.concatenate([idx, [-1, -1]]), 30, ring, ring, 4, 0, 0, None, 1.0)[0]
+    assert np.allclose(a, c, atol=1e-13)
+
+
+def test_degenerate_cases():
+    g = np.random.default_rng(22)
+    q, row = g.standard_normal((3, 8)), g.standard_normal((1, 8))
+    z = np.zeros((0, 8))
+    out, lse = O.attend(q, row, z, z, None, 1.0)
+    assert np.allclose(out, np.repeat(row, 3, 0), atol=1e-14)
+    sink = np.array([0.5, -1.0, 2.0])
+    out, lse = O.attend(q, z, z, z, sink, 1.0)
+    assert np.all(out == 0) and np.allclose(lse, sink)
+    out, lse = O.attend(q, z, z, z, None, 1.0)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_visibility_rule():
+    assert O.n_visible(2, 4) == 0 and O.n_visible(3, 4) == 1 and O.n_visible(7, 4) == 2
+    assert O.n_visible(0, 1) == 1 and O.n_visible(126, 128) == 0 and O.n_visible(127, 128) == 1
+
+
+# ---------------------------------------------------------------- decode step
+def _small_decode(**kw):
+    from compressed_sparse_attention_compressor_b200 import workloads as Wk
+
+    wl = Wk.WORKLOADS["decode64k"].scaled(batch=2, context=64, d=16, h_q=3, h_idx=2, d_idx=8, **kw)
+    return Wk.make_decode_inputs(wl)
+
+
+def test_decode_step_dense_no_window_equals_sdpa():
+    inp = _small_decode(topk=0, window=0, sink="zero", m=4, act_dtype="f32", kv_dtype="f32",
+                        idx_dtype="f32")
+    res = O.decode_step(inp)
+    kv = O.decode_stored(inp.kv)
+    for b in range(2):
+        rows = kv[b].copy()
+        rows[15] = res["new_rows"][b].astype(np.float32)  # stored as fp32
+        q = O.decode_stored(inp.q)[b]
+        # sink 0 is an extra key with logit 0 and value 0
+        K = np.concatenate([np.concatenate([rows, np.zeros((16, 1))], 1), [[0.0] * 16 + [1.0]]])
+        V = np.concatenate([rows, np.zeros((1, 16))])
+        qa = np.concatenate([q, np.zeros((3, 1))], 1)
+        assert np.allclose(res["out"][b], _sdpa(qa, K, V), atol=1e-10)
+
+
+def test_decode_step_ratio1_appends_the_token_row():
+    inp = _small_decode(m=1, topk=4, window=3, act_dtype="f32", kv_dtype="f32", idx_dtype="f32")
+    res = O.decode_step(inp)
+    c_t = O.decode_stored(inp.c_t)
+    for b in range(2):
+        assert np.array_equal(res["new_rows"][b], c_t[b])
+        assert np.allclose(res["new_keys"][b], c_t[b] @ O.decode_stored(inp.w_ik), atol=1e-13)
