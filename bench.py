@@ -1,0 +1,425 @@
+"""Decode-step throughput of the compressed-sparse-attention hot path on B200.
+
+One step = csa_decode_step for every request of the workload: append the new
+token (SWA ring + open block), pool the block it closes and project its
+indexer key, score all visible compressed entries, select the top-k, and run
+the single-softmax attention over the selection + window + sink.
+
+Default workload: ``decode1m`` -- batch 4 at 1,048,576 tokens, m = 4
+(262,144 compressed entries per request), FP8 E4M3 main KV (fp32 scale per
+64 channels) and FP8 indexer keys (fp32 scale per row), 64 bf16 query heads
+of dim 512, indexer 64 x 128, top-k 1,024, W = 128.  Inputs are seeded and
+synthetic; every step works on the same resident caches, and an L2 flush
+(a 256 MB write) runs between timed steps, outside their events.
+
+Metric: decode tokens/s (requests finished per second, all ranks).
+Multi-GPU: every rank runs its own batch (independent requests, no
+collective on the data path): weak scaling, max-over-ranks device time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressed_sparse_attention_compressor_b200 import workloads as Wk  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = {
+    "index_score_simt_kernel": "index_topk.cu",
+    "topk_row_kernel": "index_topk.cu",
+    "attn_simt_kernel": "attention.cu",
+    "attn_merge_kernel": "attention.cu",
+    "decode_append_kernel": "compress.cu",
+    "compress_kernel": "compress.cu",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode1m", choices=[k for k, v in Wk.WORKLOADS.items() if not v.is_prefill])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# byte accounting (algorithmic bytes: what the path must read / write once)
+# ---------------------------------------------------------------------------
+def _eb(dt):
+    return {"f32": 4, "bf16": 2, "fp8": 1}[dt]
+
+
+def key_row_bytes(wl):
+    return wl.d_idx * _eb(wl.idx_dtype) + (4 if wl.idx_dtype == "fp8" else 0)
+
+
+def kv_row_bytes(wl):
+    return wl.d * _eb(wl.kv_dtype) + (4 * wl.d // wl.kv_group if wl.kv_dtype == "fp8" else 0)
+
+
+def step_bytes(wl, n_vis):
+    """Headline bytes of one decode step: the visible indexer keys, the
+    selected (or, dense, all visible) compressed rows, the window K/V rows."""
+    B = wl.batch
+    keys = 0 if wl.dense else B * n_vis * key_row_bytes(wl)
+    rows = B * (n_vis if wl.dense else min(wl.topk, n_vis)) * kv_row_bytes(wl)
+    window = B * 2 * wl.window * wl.d * _eb(wl.act_dtype)
+    return keys + rows + window
+
+
+def kernel_bytes(name, wl, n_vis):
+    """Algorithmic bytes of one launch of a kernel of the decode step."""
+    B, ea = wl.batch, _eb(wl.act_dtype)
+    if name.startswith("index_score"):
+        return B * n_vis * key_row_bytes(wl) + B * wl.h_idx * (wl.d_idx * ea + 4)
+    if name.startswith("attn_simt"):
+        rows = n_vis if wl.dense else min(wl.topk, n_vis)
+        return (B * rows * kv_row_bytes(wl) + B * 2 * wl.window * wl.d * ea + 2 * B * wl.h_q * wl.d * ea)
+    if name.startswith("topk"):
+        return B * n_vis * 4 + B * wl.topk * 4
+    return None
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def load_traffic(name):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    source is unchanged since the capture (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(name)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, "compressed_sparse_attention_compressor_b200", "csrc", KERNEL_SOURCES[name])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha256_16"]:
+            return None
+        return float(rec["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-i", str(self.index), "-lms", "200"], stdout=subprocess.PIPE,
+                                      stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.p is not None:
+            time.sleep(0.3)
+            self.p.terminate()
+            try:
+                self.out, _ = self.p.communicate(timeout=5)
+            except Exception:
+                self.p.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from compressed_sparse_attention_compressor_b200 import csa
+    from compressed_sparse_attention_compressor_b200.csa import DevTensor
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_
+        dist = dist_
+
+    wl = Wk.WORKLOADS[args.workload].scaled(seed=Wk.WORKLOADS[args.workload].seed + 100 * rank)
+    inp = Wk.make_decode_inputs(wl)
+    B = wl.batch
+    up = DevTensor.from_stored
+    kv, kidx, swa_k, swa_v = up(inp.kv), up(inp.kidx), up(inp.swa_k), up(inp.swa_v)
+    open_c, open_z = up(inp.open_c), up(inp.open_z)
+    c_t, z_t, k_t, v_t, q, q_idx, w_ik = (up(inp.c_t), up(inp.z_t), up(inp.k_t), up(inp.v_t), up(inp.q),
+                                          up(inp.q_idx), up(inp.w_ik))
+    w = torch.from_numpy(inp.w).cuda()
+    sink = torch.from_numpy(inp.sink).cuda()
+    pos = torch.from_numpy(inp.pos).cuda()
+    p = csa.params(wl.m, wl.d, wl.d_idx, wl.h_q, wl.h_idx, wl.topk, wl.window, inp.swa_cap, 1.0)
+    out = DevTensor.empty((B, wl.h_q, wl.d), "bf16" if wl.act_dtype != "f32" else "f32")
+    lse = torch.empty((B, wl.h_q), dtype=torch.float32, device="cuda")
+    ws = csa.workspace(csa.csa_workspace_size(p, B, inp.cap))
+    caches = csa.decode_caches(kv, kidx, swa_k, swa_v, open_c, open_z, inp.cap)
+    tok = csa.decode_token(c_t, z_t, k_t, v_t, q, q_idx, w, sink, w_ik)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    n_vis = int((inp.pos[0] + 1) // wl.m)
+    del inp
+
+    def step():
+        csa.csa_decode_step(p, B, caches, tok, pos, out, lse, ws, stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region (device time per step, L2 flushed between steps) ----
+    K = args.steps
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            e0[i].record(stream)
+            step()
+            e1[i].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
+    total_ms = float(sum(step_ms))
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+
+    # ---- per-kernel times: the same K steps with events around every launch ----
+    csa.csa_profile_start(64 * K)
+    for i in range(K):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    csa.csa_profile_stop()
+    recs = csa.csa_profile_records()
+    per = {}
+    for name, ms in recs:
+        c = per.setdefault(name, [0, 0.0])
+        c[0] += 1
+        c[1] += ms
+    launches_per_step = len(recs) / K
+    dom = max(per, key=lambda n: per[n][1])
+    dom_ms = per[dom][1] / per[dom][0]
+    dom_bytes = kernel_bytes(dom, wl, n_vis)
+    peak, peak_src = load_peaks()
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_bytes else None
+
+    # ---- end to end: host inputs -> device -> step -> host output ----
+    host_in = []
+    for t in (c_t, z_t, k_t, v_t, q, q_idx):
+        host_in.append((t.data.cpu().pin_memory(), t.data))
+    host_in.append((w.cpu().pin_memory(), w))
+    host_out = torch.empty_like(out.data, device="cpu").pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    f0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    f1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        f0[i].record(stream)
+        for h, d_ in host_in:
+            d_.copy_(h, non_blocking=True)
+        step()
+        host_out.copy_(out.data, non_blocking=True)
+        f1[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(f0, f1)))
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = B * world / (e2e_ms / K * 1e-3)
+
+    value = B * world / (ms_per_step * 1e-3)
+    sbytes = step_bytes(wl, n_vis)
+    res = {
+        "metric": "decode tokens/s (CSA+SWA attention step)",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8" if wl.kv_dtype == "fp8" else wl.act_dtype,
+        "data": "synthetic (seeded Gaussian caches and queries)",
+        "config": {
+            "workload": wl.name, "batch_per_gpu": B, "context": wl.context, "m": wl.m,
+            "compressed_entries": n_vis, "topk": wl.topk, "window": wl.window, "d": wl.d, "h_q": wl.h_q,
+            "indexer": f"{wl.h_idx}x{wl.d_idx}", "kv_dtype": wl.kv_dtype, "idx_dtype": wl.idx_dtype,
+            "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (256 MB write)",
+        },
+        "step_hbm": {"bytes": sbytes, "gbs": sbytes / (ms_per_step * 1e-3) / 1e9,
+                     "frac_of_peak": sbytes / (ms_per_step * 1e-3) / 1e9 / peak,
+                     "frac_of_8tbs": sbytes / (ms_per_step * 1e-3) / 1e9 / 8000.0},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None, "traffic": load_traffic(dom),
+                     "algorithmic_bytes": dom_bytes, "avg_ms": dom_ms, "peak_source": f"{peak_src} hbm_gbs"},
+        "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
+                    for n, (c, t) in per.items()},
+        "gpu_launches": int(round(launches_per_step * K)),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+    }
+    return res
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl_name, budget_s=12.0, min_reqs=1):
+    """Times the oracle's decode step one request at a time until the budget
+    is spent; returns (requests/s, requests timed, seconds)."""
+    from oracle import csa_oracle as O
+
+    wl = Wk.WORKLOADS[wl_name]
+    inp = Wk.make_decode_inputs(wl)
+    n, t = 0, 0.0
+    while n < min_reqs or (t < budget_s and n < wl.batch * 4):
+        b = n % wl.batch
+        t0 = time.perf_counter()
+        O.decode_step(inp, requests=[b])
+        t += time.perf_counter() - t0
+        n += 1
+    return n / t, n, t
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, one request per step (a bounded
+    sample of the workload), on this host's cores."""
+    from oracle import csa_oracle as O
+
+    wl = Wk.WORKLOADS[args.workload]
+    inp = Wk.make_decode_inputs(wl)
+    for i in range(args.warmup):
+        O.decode_step(inp, requests=[i % wl.batch])
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        O.decode_step(inp, requests=[i % wl.batch])
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = 1.0 / (ms * 1e-3)
+    sample = f"one request ({wl.context} tokens, {(wl.context) // wl.m} entries) per step, requests cycled"
+    return {
+        "metric": "decode tokens/s (CSA+SWA attention step)", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Gaussian caches and queries)",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.context, "m": wl.m,
+                   "topk": wl.topk, "window": wl.window},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, t = oracle_sample(args.workload)
+        res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+                               "sample": f"{n} single-request decode steps of {args.workload} ({t:.1f} s)"}
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

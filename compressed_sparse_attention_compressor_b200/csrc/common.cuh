@@ -1,0 +1,152 @@
+// Device-side helpers shared by the kernels of the library: storage-format
+// loads/stores (fp32, bf16, FP8 E4M3 with fp32 group scales), the ordered
+// 32-bit key of an fp32 score, and host-side error plumbing.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+constexpr int kF32 = CSA_F32;
+constexpr int kBF16 = CSA_BF16;
+constexpr int kFP8 = CSA_FP8_E4M3;
+
+// --------------------------------------------------------------------------
+// scalar conversions
+// --------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Two E4M3 codes (low byte = first element) -> two floats.  E4M3 converts
+// exactly to f16 (and f16 exactly to f32).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t two_codes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes), __NV_E4M3);
+  __half2 hh;
+  hh = *reinterpret_cast<__half2*>(&h);
+  return __half22float2(hh);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+  return __half2float(*reinterpret_cast<__half*>(&h));
+}
+
+// Round-to-nearest-even, saturating to +-448.
+__device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
+  __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// --------------------------------------------------------------------------
+// 8-element vector loads (16 B of bf16, 32 B of fp32, 8 B of fp8)
+// --------------------------------------------------------------------------
+// Loads elements [col, col+8) of a row into v (fp32).  For FP8, `scale`
+// points at the row's group scales and `group` is the group length
+// (a multiple of 8, so the 8 elements share one scale).
+__device__ __forceinline__ void load8(const void* row, int dtype, int col, const float* scale, int group,
+                                      float v[8]) {
+  if (dtype == kF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(row) + col);
+    float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else if (dtype == kBF16) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(row) + col));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(row) + col));
+    float s = __ldg(scale + col / group);
+    uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFF));
+      float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
+      v[4 * i + 0] = lo.x * s; v[4 * i + 1] = lo.y * s;
+      v[4 * i + 2] = hi.x * s; v[4 * i + 3] = hi.y * s;
+    }
+  }
+}
+
+// Stores 8 fp32 values as fp32 or bf16 (not FP8: FP8 needs a group scale).
+__device__ __forceinline__ void store8(void* row, int dtype, int col, const float v[8]) {
+  if (dtype == kF32) {
+    float4* p = reinterpret_cast<float4*>(static_cast<float*>(row) + col);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w[i] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i])) |
+             (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * i + 1])) << 16);
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(row) + col) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+__device__ __forceinline__ float load1(const void* row, int dtype, int col, const float* scale, int group) {
+  if (dtype == kF32) return __ldg(static_cast<const float*>(row) + col);
+  if (dtype == kBF16) return bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(row) + col));
+  return e4m3_to_f32(__ldg(static_cast<const uint8_t*>(row) + col)) * __ldg(scale + col / group);
+}
+
+__host__ __device__ __forceinline__ int elem_bytes(int dtype) {
+  return dtype == kF32 ? 4 : (dtype == kBF16 ? 2 : 1);
+}
+
+// --------------------------------------------------------------------------
+// ordered key of an fp32 score: larger float -> larger unsigned key;
+// -0 and +0 map to the same key.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) == 0) u = 0;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_score(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+// --------------------------------------------------------------------------
+// warp helpers
+// --------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// --------------------------------------------------------------------------
+// host-side error reporting (defined in csa_api.cu)
+// --------------------------------------------------------------------------
+csa_status_t set_error(csa_status_t st, const char* fmt, ...);
+// Every kernel launch is bracketed by prof_begin(stream) before it and
+// check_launch(name, stream) after it: check_launch reports launch errors
+// and, while csa_profile_start() is active, records CUDA events around the
+// launch on its stream.
+void prof_begin(cudaStream_t stream);
+csa_status_t check_launch(const char* what, cudaStream_t stream);
+
+}  // namespace csa

@@ -1,0 +1,385 @@
+// The exported C ABI (include/csa.h): host-side validation, workspace
+// layout, and dispatch to the kernels.  Nothing here allocates device memory.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace csa {
+
+csa_status_t launch_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int batch, int64_t n_tokens, int d,
+                             int m, const csa_tensor_t* out, int64_t out_rows, const csa_tensor_t* w_ik,
+                             int d_idx, const csa_tensor_t* kidx_out, cudaStream_t stream);
+csa_status_t launch_decode_append(const csa_params_t* p, int batch, const csa_decode_caches_t* cc,
+                                  const csa_decode_token_t* tok, const int64_t* pos, int32_t* n_visible,
+                                  int64_t* q_pos, int32_t* q_req, cudaStream_t stream);
+csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
+                                const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
+                                const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
+                                cudaStream_t stream);
+csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
+                         int32_t* out_idx, float* out_score, cudaStream_t stream);
+csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
+                              int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible, const int32_t* q_req,
+                              const csa_tensor_t* swa_k, const csa_tensor_t* swa_v, const int64_t* q_pos,
+                              const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
+                              void* workspace, int max_keys, cudaStream_t stream);
+size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys);
+
+namespace {
+thread_local char g_msg[512] = "";
+
+// Workspace carve-up: consecutive 256-byte aligned regions.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t n) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+csa_status_t check_tensor(const char* name, const csa_tensor_t* t, int row_elems, bool allow_f32, bool allow_bf16,
+                          bool allow_fp8, int fp8_group) {
+  if (t == nullptr || t->data == nullptr) return set_error(CSA_ERR_INVALID_ARG, "%s: null tensor", name);
+  const int dt = t->dtype;
+  if ((dt == kF32 && !allow_f32) || (dt == kBF16 && !allow_bf16) || (dt == kFP8 && !allow_fp8) ||
+      (dt != kF32 && dt != kBF16 && dt != kFP8))
+    return set_error(CSA_ERR_INVALID_ARG, "%s: dtype %d not accepted here", name, dt);
+  if (!aligned16(t->data)) return set_error(CSA_ERR_INVALID_ARG, "%s: data not 16-byte aligned", name);
+  if ((static_cast<int64_t>(row_elems) * elem_bytes(dt)) % 16 != 0)
+    return set_error(CSA_ERR_INVALID_ARG, "%s: rows of %d elements are not a multiple of 16 bytes", name, row_elems);
+  if (dt == kFP8) {
+    if (t->scale == nullptr) return set_error(CSA_ERR_INVALID_ARG, "%s: FP8 tensor without scales", name);
+    if (fp8_group > 0 && t->scale_group != fp8_group)
+      return set_error(CSA_ERR_INVALID_ARG, "%s: FP8 scale_group must be %d (got %d)", name, fp8_group,
+                       t->scale_group);
+    if (t->scale_group <= 0 || t->scale_group % 8 != 0 || row_elems % t->scale_group != 0)
+      return set_error(CSA_ERR_INVALID_ARG, "%s: bad FP8 scale_group %d", name, t->scale_group);
+  }
+  return CSA_OK;
+}
+
+csa_status_t check_params(const csa_params_t* p, bool need_idx) {
+  if (p == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null params");
+  if (p->m < 1 || p->d < 8 || p->h_q < 1 || p->window < 0)
+    return set_error(CSA_ERR_INVALID_ARG, "bad params (m=%d d=%d h_q=%d window=%d)", p->m, p->d, p->h_q, p->window);
+  if (p->d % 8 != 0) return set_error(CSA_ERR_INVALID_ARG, "d=%d must be a multiple of 8", p->d);
+  if (p->window > 0 && p->swa_cap < p->window)
+    return set_error(CSA_ERR_INVALID_ARG, "swa_cap=%d smaller than window=%d", p->swa_cap, p->window);
+  if (need_idx && (p->h_idx < 1 || p->d_idx < 8 || p->d_idx % 8 != 0))
+    return set_error(CSA_ERR_INVALID_ARG, "bad indexer shape h_idx=%d d_idx=%d", p->h_idx, p->d_idx);
+  return CSA_OK;
+}
+
+size_t index_ws_bytes(int nq, int64_t cap) {
+  Carver c(nullptr);
+  c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
+  return c.off;
+}
+
+}  // namespace
+
+csa_status_t set_error(csa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+// ---- per-launch event profiler (csa_profile_*) ----
+namespace {
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+bool g_prof_open = false;            // a begin event is recorded, its end is not
+int g_prof_n = 0;
+std::vector<cudaEvent_t> g_prof_ev;  // 2 per record
+std::vector<const char*> g_prof_name;
+}  // namespace
+
+void prof_begin(cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on || 2 * (g_prof_n + 1) > static_cast<int>(g_prof_ev.size())) return;
+  cudaEventRecord(g_prof_ev[2 * g_prof_n], stream);
+  g_prof_open = true;
+}
+
+csa_status_t check_launch(const char* what, cudaStream_t stream) {
+  cudaError_t e = cudaGetLastError();
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_open) {
+      cudaEventRecord(g_prof_ev[2 * g_prof_n + 1], stream);
+      g_prof_name[g_prof_n] = what;
+      ++g_prof_n;
+      g_prof_open = false;
+    }
+  }
+  if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_last_error(void) { return g_msg; }
+
+size_t csa_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries) {
+  if (p == nullptr || n_queries < 0 || max_entries < 0) return 0;
+  const int max_keys = static_cast<int>((p->topk > 0 ? p->topk : max_entries) + p->window);
+  Carver c(nullptr);
+  // decode-step bookkeeping
+  c.take<int32_t>(n_queries);
+  c.take<int64_t>(n_queries);
+  c.take<int32_t>(n_queries);
+  if (p->topk > 0) {
+    c.take<int32_t>(static_cast<size_t>(n_queries) * p->topk);
+    c.take<char>(index_ws_bytes(n_queries, max_entries));
+  }
+  const size_t attn = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
+  return c.off + attn + 256;
+}
+
+csa_status_t csa_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int32_t batch, int64_t n_tokens, int32_t d,
+                          int32_t m, const csa_tensor_t* out, int64_t out_rows, const csa_tensor_t* w_ik,
+                          int32_t d_idx, const csa_tensor_t* kidx_out, csa_stream_t stream) {
+  g_msg[0] = 0;
+  if (batch < 0 || n_tokens < 0 || m < 1 || d < 8 || d % 8 != 0)
+    return set_error(CSA_ERR_INVALID_ARG, "bad shape batch=%d n_tokens=%lld d=%d m=%d", batch,
+                     static_cast<long long>(n_tokens), d, m);
+  if (out_rows < n_tokens / m) return set_error(CSA_ERR_INVALID_ARG, "out_rows smaller than n_tokens / m");
+  csa_status_t st;
+  if ((st = check_tensor("C", C, d, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("Z", Z, d, true, true, false, 0)) != CSA_OK) return st;
+  if (Z->dtype != C->dtype) return set_error(CSA_ERR_INVALID_ARG, "C and Z dtypes differ");
+  if ((st = check_tensor("out", out, d, true, true, true, 64)) != CSA_OK) return st;
+  if (w_ik != nullptr) {
+    if (d_idx < 32 || d_idx > 256 || d_idx % 32 != 0)
+      return set_error(CSA_ERR_UNSUPPORTED, "d_idx=%d: projection needs a multiple of 32 in [32, 256]", d_idx);
+    if ((st = check_tensor("w_ik", w_ik, d_idx, true, true, false, 0)) != CSA_OK) return st;
+    if ((st = check_tensor("kidx_out", kidx_out, d_idx, true, true, true, d_idx)) != CSA_OK) return st;
+    if (static_cast<size_t>(8) * d * sizeof(float) > 200 * 1024)
+      return set_error(CSA_ERR_UNSUPPORTED, "d=%d too large for the projection stage", d);
+  }
+  return launch_compress(C, Z, batch, n_tokens, d, m, out, out_rows, w_ik, d_idx, kidx_out,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int32_t* n_valid, int32_t k,
+                      int32_t* out_idx, float* out_score, void* workspace, size_t workspace_bytes,
+                      csa_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  g_msg[0] = 0;
+  if (n_rows < 0 || k < 1 || ld < 0) return set_error(CSA_ERR_INVALID_ARG, "bad shape n_rows=%d k=%d", n_rows, k);
+  if (n_rows > 0 && (scores == nullptr || n_valid == nullptr || out_idx == nullptr))
+    return set_error(CSA_ERR_INVALID_ARG, "null pointer");
+  return launch_topk(scores, n_rows, ld, n_valid, ld, k, out_idx, out_score, reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,
+                            const csa_tensor_t* k_idx, int32_t batch, int64_t cap, const int32_t* q_req, const int32_t* n_visible,
+                            int32_t* out_idx, float* out_score, void* workspace, size_t workspace_bytes,
+                            csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  if ((st = check_params(p, true)) != CSA_OK) return st;
+  if (p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "csa_index_topk needs topk >= 1");
+  if (n_queries < 0 || cap < 0 || batch < 1) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap");
+  if (n_queries == 0) return CSA_OK;
+  if ((st = check_tensor("q_idx", q_idx, p->d_idx, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("k_idx", k_idx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
+  if (w == nullptr || n_visible == nullptr || out_idx == nullptr)
+    return set_error(CSA_ERR_INVALID_ARG, "null w / n_visible / out_idx");
+  const size_t need = index_ws_bytes(n_queries, cap);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  const int64_t ld = round_up(cap, 4);
+  float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
+  if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s)) !=
+      CSA_OK)
+    return st;
+  return launch_topk(scores, n_queries, ld, n_visible, cap, p->topk, out_idx, out_score, s);
+}
+
+csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q,
+                                      const csa_tensor_t* kv, int32_t batch, int64_t cap, const int32_t* idx,
+                                      const int32_t* n_visible, const int32_t* q_req, const csa_tensor_t* swa_k,
+                                      const csa_tensor_t* swa_v, const int64_t* q_pos, const int64_t* swa_lo,
+                                      const float* sink, const csa_tensor_t* out, float* lse, void* workspace,
+                                      size_t workspace_bytes, csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  if ((st = check_params(p, false)) != CSA_OK) return st;
+  if (n_queries < 0 || cap < 0 || batch < 1) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap");
+  if (n_queries == 0) return CSA_OK;
+  if ((st = check_tensor("q", q, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("kv", kv, p->d, true, true, true, 64)) != CSA_OK) return st;
+  if ((st = check_tensor("out", out, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if (p->window > 0) {
+    if ((st = check_tensor("swa_k", swa_k, p->d, true, true, false, 0)) != CSA_OK) return st;
+    if ((st = check_tensor("swa_v", swa_v, p->d, true, true, false, 0)) != CSA_OK) return st;
+    if (swa_k->dtype != swa_v->dtype) return set_error(CSA_ERR_INVALID_ARG, "swa_k / swa_v dtypes differ");
+  }
+  if (n_visible == nullptr || q_pos == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null n_visible / q_pos");
+  if (idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "idx given with topk < 1");
+  const int max_keys = static_cast<int>((idx ? p->topk : cap) + p->window);
+  const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  return launch_attention(p, n_queries, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink, out,
+                          lse, workspace, max_keys, reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_decode_caches_t* cc,
+                             const csa_decode_token_t* tok, const int64_t* pos, const csa_tensor_t* out, float* lse,
+                             void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  const bool sparse = p && p->topk > 0;
+  // the indexer-key projection runs when the caller passes a projection (always for CSA)
+  const bool project = tok && tok->w_ik.data != nullptr;
+  if ((st = check_params(p, sparse || project)) != CSA_OK) return st;
+  if (cc == nullptr || tok == nullptr || pos == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null caches / token / pos");
+  if (batch < 0) return set_error(CSA_ERR_INVALID_ARG, "bad batch");
+  if (batch == 0) return CSA_OK;
+  if (p->window < 1) return set_error(CSA_ERR_INVALID_ARG, "decode step needs window >= 1 (the token's own SWA slot)");
+  if (sparse && !project) return set_error(CSA_ERR_INVALID_ARG, "a sparse (topk >= 1) step needs w_ik");
+  if (project && (p->d_idx < 32 || p->d_idx > 256 || p->d_idx % 32 != 0))
+    return set_error(CSA_ERR_UNSUPPORTED, "d_idx=%d: projection needs a multiple of 32 in [32, 256]", p->d_idx);
+  if ((st = check_tensor("kv", &cc->kv, p->d, true, true, true, 64)) != CSA_OK) return st;
+  if (project && (st = check_tensor("kidx", &cc->kidx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
+  if ((st = check_tensor("swa_k", &cc->swa_k, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("swa_v", &cc->swa_v, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("open_c", &cc->open_c, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("open_z", &cc->open_z, p->d, true, true, false, 0)) != CSA_OK) return st;
+  const int act = tok->c.dtype;
+  const csa_tensor_t* acts[] = {&tok->c, &tok->z, &tok->k_swa, &tok->v_swa};
+  const char* names[] = {"c", "z", "k_swa", "v_swa"};
+  for (int i = 0; i < 4; ++i) {
+    if ((st = check_tensor(names[i], acts[i], p->d, true, true, false, 0)) != CSA_OK) return st;
+    if (acts[i]->dtype != act) return set_error(CSA_ERR_INVALID_ARG, "token rows must share one dtype");
+  }
+  if (cc->open_c.dtype != act || cc->open_z.dtype != act)
+    return set_error(CSA_ERR_INVALID_ARG, "open-block buffers must have the token rows' dtype");
+  if (cc->swa_k.dtype != cc->swa_v.dtype) return set_error(CSA_ERR_INVALID_ARG, "swa_k / swa_v dtypes differ");
+  if ((st = check_tensor("q", &tok->q, p->d, true, true, false, 0)) != CSA_OK) return st;
+  if (project && (st = check_tensor("w_ik", &tok->w_ik, p->d_idx, true, true, false, 0)) != CSA_OK) return st;
+  if (sparse) {
+    if ((st = check_tensor("q_idx", &tok->q_idx, p->d_idx, true, true, false, 0)) != CSA_OK) return st;
+    if (tok->w == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null indexer weights");
+  }
+  if ((st = check_tensor("out", out, p->d, true, true, false, 0)) != CSA_OK) return st;
+  const size_t need = csa_workspace_size(p, batch, cc->cap);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  int32_t* n_vis = c.take<int32_t>(batch);
+  int64_t* q_pos = c.take<int64_t>(batch);
+  int32_t* q_req = c.take<int32_t>(batch);
+  int32_t* idx = nullptr;
+  void* index_ws = nullptr;
+  if (sparse) {
+    idx = c.take<int32_t>(static_cast<size_t>(batch) * p->topk);
+    index_ws = c.take<char>(index_ws_bytes(batch, cc->cap));
+  }
+  const int max_keys = static_cast<int>((sparse ? p->topk : cc->cap) + p->window);
+  void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys));
+
+  if ((st = launch_decode_append(p, batch, cc, tok, pos, n_vis, q_pos, q_req, s)) != CSA_OK) return st;
+  if (sparse) {
+    const int64_t ld = round_up(cc->cap, 4);
+    float* scores = static_cast<float*>(index_ws);
+    if ((st = launch_index_score(p, batch, &tok->q_idx, tok->w, &cc->kidx, batch, cc->cap, q_req, n_vis, scores, ld,
+                                 cc->cap, s)) != CSA_OK)
+      return st;
+    if ((st = launch_topk(scores, batch, ld, n_vis, cc->cap, p->topk, idx, nullptr, s)) != CSA_OK) return st;
+  }
+  return launch_attention(p, batch, &tok->q, &cc->kv, batch, cc->cap, idx, n_vis, q_req, &cc->swa_k, &cc->swa_v, q_pos,
+                          nullptr, tok->sink, out, lse, attn_ws, max_keys, s);
+}
+
+csa_status_t csa_index_score(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,
+                             const csa_tensor_t* k_idx, int32_t batch, int64_t cap, const int32_t* q_req,
+                             const int32_t* n_visible, float* scores, int64_t ld, csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  if ((st = check_params(p, true)) != CSA_OK) return st;
+  if (n_queries < 0 || cap < 0 || batch < 1 || ld < cap)
+    return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap / ld");
+  if (n_queries == 0) return CSA_OK;
+  if ((st = check_tensor("q_idx", q_idx, p->d_idx, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("k_idx", k_idx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
+  if (w == nullptr || n_visible == nullptr || scores == nullptr)
+    return set_error(CSA_ERR_INVALID_ARG, "null w / n_visible / scores");
+  return launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_profile_start(int32_t max_launches) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (max_launches < 1) return set_error(CSA_ERR_INVALID_ARG, "max_launches must be >= 1");
+  for (cudaEvent_t e : g_prof_ev) cudaEventDestroy(e);
+  g_prof_ev.assign(2 * static_cast<size_t>(max_launches), nullptr);
+  g_prof_name.assign(max_launches, nullptr);
+  for (auto& e : g_prof_ev) {
+    cudaError_t err = cudaEventCreate(&e);
+    if (err != cudaSuccess) {
+      g_prof_on = false;
+      return set_error(CSA_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(err));
+    }
+  }
+  g_prof_n = 0;
+  g_prof_open = false;
+  g_prof_on = true;
+  return CSA_OK;
+}
+
+csa_status_t csa_profile_stop(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  g_prof_open = false;
+  return CSA_OK;
+}
+
+int32_t csa_profile_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_prof_n;
+}
+
+csa_status_t csa_profile_get(int32_t i, const char** name, float* ms) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (i < 0 || i >= g_prof_n) return set_error(CSA_ERR_INVALID_ARG, "no profile record %d", i);
+  cudaError_t e = cudaEventSynchronize(g_prof_ev[2 * i + 1]);
+  if (e == cudaSuccess) e = cudaEventElapsedTime(ms, g_prof_ev[2 * i], g_prof_ev[2 * i + 1]);
+  if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "profile record %d: %s", i, cudaGetErrorString(e));
+  if (name) *name = g_prof_name[i];
+  return CSA_OK;
+}
+
+csa_status_t csa_sync_status(csa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+}  // extern "C"

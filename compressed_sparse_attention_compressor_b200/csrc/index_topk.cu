@@ -1,0 +1,251 @@
+// K2 -- lightning-indexer scores, and K3 -- exact per-query top-k.
+//
+// Atlas "Model architectures", "Trained sparse attention" entry (DSA: a
+// lightning indexer followed by fine-grained top-k selection) and
+// "compressed KV" entry (top-k over compressed entries); tech-report tour,
+// "The indexer selects, SWA covers the rest" (the indexer scores main-KV
+// entries with indexer query and indexer key and keeps the top entries of
+// every query).
+//
+//   s_j = sum_h w_h * max(0, q_h . k_j)       (FP8 keys: k_j = codes * scale_j)
+//
+// Top-k order: score descending; among exactly equal scores the lower index
+// wins (-0 == +0).  The selection is a radix select on the ordered 32-bit
+// key of each fp32 score (three histogram passes of 11/11/10 bits), which
+// yields the exact k-th key T and the number r of entries equal to T that
+// are kept; an index-ordered pass then takes every entry above T and the r
+// lowest-index entries equal to T.
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// K2, CUDA-core form: one thread per key, all heads accumulated in registers.
+// ---------------------------------------------------------------------------
+constexpr int kScoreThreads = 256;
+
+template <int H, int DI>
+__global__ void __launch_bounds__(kScoreThreads)
+index_score_simt_kernel(const void* __restrict__ q_idx, int q_dtype, const float* __restrict__ w,
+                        const void* __restrict__ keys, const float* __restrict__ kscale, int k_dtype,
+                        int batch, int64_t cap, const int32_t* __restrict__ q_req,
+                        const int32_t* __restrict__ n_visible, float* __restrict__ scores, int64_t ld) {
+  __shared__ __align__(16) float qs[H * DI];
+  __shared__ float ws[H];
+  const int qi = blockIdx.y;
+  const int r = q_req ? q_req[qi] : qi;
+  const int64_t n = (r < 0 || r >= batch) ? 0 : min(max(static_cast<int64_t>(n_visible[qi]), int64_t(0)), cap);
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kScoreThreads;
+  if (j0 >= n) return;  // uniform over the CTA
+  const char* qrow = static_cast<const char*>(q_idx) + static_cast<int64_t>(qi) * H * DI * elem_bytes(q_dtype);
+  for (int i = threadIdx.x; i < H * DI; i += kScoreThreads) qs[i] = load1(qrow, q_dtype, i, nullptr, 1);
+  for (int i = threadIdx.x; i < H; i += kScoreThreads) ws[i] = w[static_cast<int64_t>(qi) * H + i];
+  __syncthreads();
+  const int64_t j = j0 + threadIdx.x;
+  if (j >= n) return;
+  const int64_t krow = static_cast<int64_t>(r) * cap + j;
+  const char* kp = static_cast<const char*>(keys) + krow * DI * elem_bytes(k_dtype);
+  const float* sp = (k_dtype == kFP8) ? kscale + krow : nullptr;
+  float acc[H];
+#pragma unroll
+  for (int h = 0; h < H; ++h) acc[h] = 0.f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < DI; c0 += 8) {
+    float k[8];
+    if (k_dtype == kFP8) {
+      // the row scale multiplies the whole score (ReLU(s*x) = s*ReLU(x), s > 0)
+      uint2 u = __ldg(reinterpret_cast<const uint2*>(kp + c0));
+      float2 a = e4m3x2_to_f32x2(static_cast<uint16_t>(u.x & 0xFFFF));
+      float2 b = e4m3x2_to_f32x2(static_cast<uint16_t>(u.x >> 16));
+      float2 c = e4m3x2_to_f32x2(static_cast<uint16_t>(u.y & 0xFFFF));
+      float2 d = e4m3x2_to_f32x2(static_cast<uint16_t>(u.y >> 16));
+      k[0] = a.x; k[1] = a.y; k[2] = b.x; k[3] = b.y; k[4] = c.x; k[5] = c.y; k[6] = d.x; k[7] = d.y;
+    } else {
+      load8(kp, k_dtype, c0, nullptr, 1, k);
+    }
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const float4 qa = *reinterpret_cast<const float4*>(&qs[h * DI + c0]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qs[h * DI + c0 + 4]);
+      float a = acc[h];
+      a = fmaf(qa.x, k[0], a); a = fmaf(qa.y, k[1], a); a = fmaf(qa.z, k[2], a); a = fmaf(qa.w, k[3], a);
+      a = fmaf(qb.x, k[4], a); a = fmaf(qb.y, k[5], a); a = fmaf(qb.z, k[6], a); a = fmaf(qb.w, k[7], a);
+      acc[h] = a;
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int h = 0; h < H; ++h) s = fmaf(ws[h], fmaxf(acc[h], 0.f), s);
+  if (sp) s *= __ldg(sp);
+  scores[static_cast<int64_t>(qi) * ld + j] = s;
+}
+
+// ---------------------------------------------------------------------------
+// K3: one CTA per row.
+// ---------------------------------------------------------------------------
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkWarps = kTopkThreads / 32;
+
+struct TopkShared {
+  uint32_t hist[2048];
+  uint32_t warp_gt[kTopkWarps];
+  uint32_t warp_eq[kTopkWarps];
+  uint32_t sel_bin;
+  uint32_t above;
+};
+
+// Within warp 0: finds the bin b of hist[0..nb) (scanned from the top) with
+// count_above(b) < need <= count_above(b) + hist[b].
+__device__ void find_bin(TopkShared& sh, int nb, uint32_t need) {
+  const int lane = threadIdx.x & 31;
+  const int per = nb / 32;
+  const int lo = lane * per;
+  uint32_t mine = 0;
+  for (int i = 0; i < per; ++i) mine += sh.hist[lo + i];
+  // suffix sum over lanes >= lane
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += v;
+  }
+  const uint32_t excl = incl - mine;
+  if (excl < need && need <= incl) {
+    uint32_t above = excl;
+    for (int i = per - 1; i >= 0; --i) {
+      const uint32_t c = sh.hist[lo + i];
+      if (above + c >= need) {
+        sh.sel_bin = lo + i;
+        sh.above = above;
+        break;
+      }
+      above += c;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
+                int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
+  __shared__ TopkShared sh;
+  const int row = blockIdx.x;
+  const int64_t n = min(max(static_cast<int64_t>(n_valid[row]), int64_t(0)), max_n);
+  const float* s = scores + static_cast<int64_t>(row) * ld;
+  int32_t* oi = out_idx + static_cast<int64_t>(row) * k;
+  float* os = out_score ? out_score + static_cast<int64_t>(row) * k : nullptr;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (n <= k) {
+    for (int64_t j = tid; j < k; j += kTopkThreads) {
+      oi[j] = j < n ? static_cast<int32_t>(j) : -1;
+      if (os) os[j] = j < n ? s[j] : -INFINITY;
+    }
+    return;
+  }
+
+  // radix select of the k-th largest key
+  uint32_t prefix = 0, pmask = 0, need = static_cast<uint32_t>(k);
+  const int shifts[3] = {21, 10, 0};
+  const int bits[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int nb = 1 << bits[pass];
+    const int sh_ = shifts[pass];
+    for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
+    __syncthreads();
+    for (int64_t j = tid; j < n; j += kTopkThreads) {
+      const uint32_t key = score_key(s[j]);
+      if ((key & pmask) == prefix) atomicAdd(&sh.hist[(key >> sh_) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) find_bin(sh, nb, need);
+    __syncthreads();
+    prefix |= sh.sel_bin << sh_;
+    pmask |= static_cast<uint32_t>(nb - 1) << sh_;
+    need -= sh.above;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;        // exact key of the k-th largest score
+  const uint32_t take_eq = need;    // entries equal to T that are kept
+  const uint32_t n_gt = static_cast<uint32_t>(k) - take_eq;
+
+  // index-ordered selection
+  uint32_t base_gt = 0, base_eq = 0;
+  for (int64_t j0 = 0; j0 < n; j0 += kTopkThreads) {
+    const int64_t j = j0 + tid;
+    float v = 0.f;
+    uint32_t key = 0;
+    if (j < n) { v = s[j]; key = score_key(v); }
+    const bool gt = j < n && key > T;
+    const bool eq = j < n && key == T;
+    const uint32_t bgt = __ballot_sync(0xFFFFFFFFu, gt), beq = __ballot_sync(0xFFFFFFFFu, eq);
+    if (lane == 0) { sh.warp_gt[warp] = __popc(bgt); sh.warp_eq[warp] = __popc(beq); }
+    __syncthreads();
+    uint32_t off_gt = 0, off_eq = 0, tot_gt = 0, tot_eq = 0;
+    for (int w2 = 0; w2 < kTopkWarps; ++w2) {
+      const uint32_t a = sh.warp_gt[w2], b = sh.warp_eq[w2];
+      if (w2 < warp) { off_gt += a; off_eq += b; }
+      tot_gt += a; tot_eq += b;
+    }
+    const uint32_t lm = (1u << lane) - 1u;
+    if (gt) {
+      const uint32_t p = base_gt + off_gt + __popc(bgt & lm);
+      oi[p] = static_cast<int32_t>(j);
+      if (os) os[p] = v;
+    }
+    if (eq) {
+      const uint32_t r = base_eq + off_eq + __popc(beq & lm);
+      if (r < take_eq) {
+        oi[n_gt + r] = static_cast<int32_t>(j);
+        if (os) os[n_gt + r] = v;
+      }
+    }
+    base_gt += tot_gt;
+    base_eq += tot_eq;
+    __syncthreads();
+  }
+}
+
+template <int H, int DI>
+csa_status_t launch_score_t(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
+                            const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
+                            const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
+                            cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>((max_entries + kScoreThreads - 1) / kScoreThreads), nq);
+  prof_begin(stream);
+  index_score_simt_kernel<H, DI><<<grid, kScoreThreads, 0, stream>>>(
+      q_idx->data, q_idx->dtype, w, k_idx->data, k_idx->scale, k_idx->dtype, batch, cap, q_req, n_visible, scores,
+      ld);
+  return check_launch("index_score_simt_kernel", stream);
+}
+
+}  // namespace
+
+csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
+                                const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
+                                const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
+                                cudaStream_t stream) {
+  if (nq == 0 || max_entries == 0) return CSA_OK;
+#define CSA_SCORE_CASE(H, DI)                                                                                  \
+  if (p->h_idx == H && p->d_idx == DI)                                                                         \
+    return launch_score_t<H, DI>(p, nq, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, max_entries, \
+                                 stream);
+  CSA_SCORE_CASE(4, 32)
+  CSA_SCORE_CASE(8, 32)
+  CSA_SCORE_CASE(16, 64)
+  CSA_SCORE_CASE(32, 128)
+  CSA_SCORE_CASE(64, 128)
+#undef CSA_SCORE_CASE
+  return set_error(CSA_ERR_UNSUPPORTED, "indexer shape h_idx=%d d_idx=%d is not built", p->h_idx, p->d_idx);
+}
+
+csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
+                         int32_t* out_idx, float* out_score, cudaStream_t stream) {
+  if (n_rows == 0) return CSA_OK;
+  prof_begin(stream);
+  topk_row_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score);
+  return check_launch("topk_row_kernel", stream);
+}
+
+}  // namespace csa

@@ -412,3 +412,18 @@ def make_scores(seed: int, n_rows: int, n_cols: int, tie_frac: float = 0.1) -> n
     vals = np.round(g.standard_normal((n_rows, n_cols)).astype(np.float32) * 4) / 4
     s[rep] = vals[rep]
     return s
+
+
+def make_indices(seed: int, n_vis: np.ndarray, k: int, pad_frac: float = 0.0) -> np.ndarray:
+    """Random distinct entry indices per query (an explicit selection for
+    testing attention on its own): row i holds min(k, n_vis[i]) distinct
+    indices below n_vis[i] in random order, then -1 padding; with
+    ``pad_frac`` > 0 some rows hold fewer entries."""
+    g = rng(seed, "indices")
+    out = np.full((n_vis.shape[0], k), -1, np.int32)
+    for i, n in enumerate(n_vis):
+        take = min(k, int(n))
+        if pad_frac > 0 and g.random() < pad_frac:
+            take = int(g.integers(0, take + 1))
+        out[i, :take] = g.permutation(int(n))[:take]
+    return out

@@ -315,8 +315,15 @@ def sparse_swa_attention(q, kv_rows, idx, n_vis, swa_k, swa_v, swa_cap, t, W, si
 # ===========================================================================
 # a6: one decode step
 # ===========================================================================
-def decode_step(inp, tau: float = 1.0):
-    """One decode step for every request of a ``workloads.DecodeInputs``.
+def _rows(t, b: int, rows) -> np.ndarray:
+    """fp64 value of rows ``rows`` of request ``b`` of a [B][n][d] stored tensor."""
+    data = t.data[b][rows]
+    scale = None if t.scale is None else t.scale[b][rows]
+    return decode(data, t.dtype, scale, t.group)
+
+
+def decode_step(inp, tau: float = 1.0, requests=None):
+    """One decode step for the requests of a ``workloads.DecodeInputs``.
 
     Tech-report tour, "Full, Reindex, and Reuse" (Full mode: compute main KV,
     project indexer K, select a fresh top-k) and "The indexer selects, SWA
@@ -329,46 +336,57 @@ def decode_step(inp, tau: float = 1.0):
       4. one softmax over selected entries + window + sink.
     The new entry and its indexer key are stored in the caches' formats
     (``round_to_storage``) before they are scored and attended, as the
-    caches hold them in storage format.
-    Returns dict with out [B][h_q][d], lse [B][h_q], idx [B][k] (or None),
-    scores [B][n] and the new cache rows (fp64, before storage rounding).
+    caches hold them in storage format.  ``requests`` restricts the work to
+    some requests (all by default); only the cache rows a request touches
+    are decoded.
+    Returns dict with out [R][h_q][d], lse [R][h_q], idx [R][k] (or None),
+    scores (list), and the new cache rows / keys (fp64, before storage
+    rounding) of the requests that closed a block.
     """
     wl = inp.wl
-    B, m, d = wl.batch, wl.m, wl.d
-    kv = decode_stored(inp.kv).copy()
-    kidx = decode_stored(inp.kidx).copy()
-    swa_k = decode_stored(inp.swa_k).copy()
-    swa_v = decode_stored(inp.swa_v).copy()
-    open_c = decode_stored(inp.open_c).copy()
-    open_z = decode_stored(inp.open_z).copy()
-    c_t, z_t = decode_stored(inp.c_t), decode_stored(inp.z_t)
-    k_t, v_t = decode_stored(inp.k_t), decode_stored(inp.v_t)
-    q, q_idx = decode_stored(inp.q), decode_stored(inp.q_idx)
-    w_ik = decode_stored(inp.w_ik)
+    m = wl.m
+    reqs = list(range(wl.batch)) if requests is None else list(requests)
     outs, lses, idxs, scores, new_rows, new_keys = [], [], [], [], [], []
-    for b in range(B):
+    w_ik = decode_stored(inp.w_ik)
+    for b in reqs:
         t = int(inp.pos[b])
-        swa_k[b, t % inp.swa_cap] = k_t[b]
-        swa_v[b, t % inp.swa_cap] = v_t[b]
-        open_c[b, t % m] = c_t[b]
-        open_z[b, t % m] = z_t[b]
+        swa_k = _rows(inp.swa_k, b, slice(None)).copy()
+        swa_v = _rows(inp.swa_v, b, slice(None)).copy()
+        swa_k[t % inp.swa_cap] = decode(inp.k_t.data[b], inp.k_t.dtype)
+        swa_v[t % inp.swa_cap] = decode(inp.v_t.data[b], inp.v_t.dtype)
+        nv = int(n_visible(t, m))
+        new_row = new_key = None
         if (t + 1) % m == 0:
-            j = (t + 1) // m - 1
-            row = compress(open_c[b], open_z[b], m)[0]
+            open_c = _rows(inp.open_c, b, slice(None)).copy()
+            open_z = _rows(inp.open_z, b, slice(None)).copy()
+            open_c[t % m] = decode(inp.c_t.data[b], inp.c_t.dtype)
+            open_z[t % m] = decode(inp.z_t.data[b], inp.z_t.dtype)
+            row = compress(open_c, open_z, m)[0]
             key = project_index_keys(row[None], w_ik)[0]
-            kv[b, j] = round_to_storage(row[None], inp.kv.dtype, inp.kv.group)[0]
-            kidx[b, j] = round_to_storage(key[None], inp.kidx.dtype, inp.kidx.group)[0]
+            new_row = round_to_storage(row[None], inp.kv.dtype, inp.kv.group)[0]
+            new_key = round_to_storage(key[None], inp.kidx.dtype, inp.kidx.group)[0]
             new_rows.append(row)
             new_keys.append(key)
-        nv = int(n_visible(t, m))
         if wl.dense:
-            sel = None
-            s = None
+            sel, s = None, None
+            ent = _rows(inp.kv, b, slice(0, nv)).copy()
+            if new_row is not None:
+                ent[nv - 1] = new_row
         else:
-            s = index_scores(q_idx[b], inp.w[b], kidx[b, :nv])
+            keys = _rows(inp.kidx, b, slice(0, nv)).copy()
+            if new_key is not None:
+                keys[nv - 1] = new_key
+            q_idx = decode(inp.q_idx.data[b], inp.q_idx.dtype)
+            s = index_scores(q_idx, inp.w[b], keys)
             sel = topk(s, wl.topk)
-        o, l = sparse_swa_attention(q[b], kv[b], sel, nv, swa_k[b], swa_v[b], inp.swa_cap, t,
-                                    wl.window, inp.sink, tau)
+            take = sel[sel >= 0]
+            ent = _rows(inp.kv, b, take)
+            if new_row is not None:
+                ent[take == nv - 1] = new_row
+        q = decode(inp.q.data[b], inp.q.dtype)
+        pos = window_positions(t, wl.window)
+        slots = pos % inp.swa_cap
+        o, l = attend(q, ent, swa_k[slots], swa_v[slots], inp.sink, tau)
         outs.append(o)
         lses.append(l)
         idxs.append(sel)
@@ -378,3 +396,65 @@ def decode_step(inp, tau: float = 1.0):
         "idx": None if wl.dense else np.stack(idxs),
         "scores": scores, "new_rows": new_rows, "new_keys": new_keys,
     }
+
+
+def pipeline(inp, queries=None, tau: float = 1.0):
+    """The path from the compressor for a ``workloads.PipelineInputs``
+    (single request): pool the new C/Z rows into entries appended after the
+    ``n_cached`` cached ones (stored in the cache format), project their
+    indexer keys, then for each query i (all, or ``queries``) at position
+    q_pos[i]: scores over its n_visible entries, top-k, and attention over
+    the selection + window + sink.  Causal visibility: block j is visible to
+    position t iff (j+1)m - 1 <= t ("Compressed Sparse Attention 2": each
+    query attends over causally visible entries)."""
+    wl = inp.wl
+    m = wl.m
+    C = decode_stored(inp.C)[0]
+    Z = decode_stored(inp.Z)[0]
+    rows = compress(C, Z, m)
+    keys = project_index_keys(rows, decode_stored(inp.w_ik))
+    n_new = rows.shape[0]
+    kv_dt = wl.kv_dtype
+    idx_dt = wl.idx_dtype
+    stored_rows = round_to_storage(rows, kv_dt, wl.kv_group)
+    stored_keys = round_to_storage(keys, idx_dt, wl.d_idx)
+    n0 = inp.n_cached
+    if n0 > 0:
+        cached_keys = _rows(inp.kidx_cached, 0, slice(0, n0))
+        all_keys = np.concatenate([cached_keys, stored_keys])
+    else:
+        all_keys = stored_keys
+
+    def kv_rows(sel):
+        sel = np.asarray(sel, np.int64)
+        out = np.empty((sel.shape[0], wl.d))
+        old = sel < n0
+        if old.any():
+            out[old] = _rows(inp.kv_cached, 0, sel[old])
+        out[~old] = stored_rows[sel[~old] - n0]
+        return out
+
+    swa_k = decode_stored(inp.swa_k)[0]
+    swa_v = decode_stored(inp.swa_v)[0]
+    q_all, qi_all = inp.q, inp.q_idx
+    qs = range(inp.q_pos.shape[0]) if queries is None else queries
+    outs, lses, idxs, scores = [], [], [], []
+    for i in qs:
+        t = int(inp.q_pos[i])
+        nv = int(n_visible(t, m))
+        if wl.dense:
+            sel, s = None, None
+            ent = kv_rows(np.arange(nv))
+        else:
+            s = index_scores(decode(qi_all.data[i], qi_all.dtype), inp.w[i], all_keys[:nv])
+            sel = topk(s, wl.topk)
+            ent = kv_rows(sel[sel >= 0])
+        pos = window_positions(t, wl.window)
+        slots = pos % inp.swa_cap
+        o, l = attend(decode(q_all.data[i], q_all.dtype), ent, swa_k[slots], swa_v[slots], inp.sink, tau)
+        outs.append(o)
+        lses.append(l)
+        idxs.append(sel)
+        scores.append(s)
+    return {"rows": rows, "keys": keys, "n_new": n_new, "out": np.stack(outs), "lse": np.stack(lses),
+            "idx": None if wl.dense else np.stack(idxs), "scores": scores}

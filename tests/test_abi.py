@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/csa.h declares, and host validation rejects bad
+arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_sparse_attention_compressor_b200 import csa
+from compressed_sparse_attention_compressor_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return csa.load()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(csa_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "csa_compress" in names and "csa_decode_step" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(csa.EXPORTS) <= set(names)
+
+
+def test_exports_are_c_symbols():
+    out = os.popen(f"nm -D --defined-only {csa.LIB_PATH}").read()
+    for n in declared_functions():
+        assert re.search(rf"\bT {n}$", out, flags=re.M), f"{n} is not an extern \"C\" text symbol"
+
+
+def _t(ptr=16, dtype=csa.CSA_BF16, scale=None, group=0):
+    return csa.Tensor(ptr, scale, dtype, group)
+
+
+def test_compress_rejects_bad_arguments(lib):
+    C, Z, out = _t(), _t(), _t()
+    st = lib.csa_compress(ctypes.byref(C), ctypes.byref(Z), 1, 64, 100, 4, ctypes.byref(out), 16, None, 0, None, None)
+    assert st == 1 and b"d=100" in lib.csa_last_error() or b"shape" in lib.csa_last_error()
+    bad = _t(ptr=18)  # not 16-byte aligned
+    st = lib.csa_compress(ctypes.byref(bad), ctypes.byref(Z), 1, 64, 128, 4, ctypes.byref(out), 16, None, 0, None, None)
+    assert st == 1 and b"aligned" in lib.csa_last_error()
+    fp8_out = _t(dtype=csa.CSA_FP8_E4M3, scale=32, group=32)
+    st = lib.csa_compress(ctypes.byref(C), ctypes.byref(Z), 1, 64, 128, 4, ctypes.byref(fp8_out), 16, None, 0, None,
+                          None)
+    assert st == 1 and b"scale_group" in lib.csa_last_error()
+    st = lib.csa_compress(ctypes.byref(C), ctypes.byref(Z), 1, 64, 128, 4, ctypes.byref(out), 8, None, 0, None, None)
+    assert st == 1 and b"out_rows" in lib.csa_last_error()
+
+
+def test_index_topk_rejects_bad_arguments(lib):
+    p = csa.params(4, 512, 128, 64, 64, 0, 128, 128)
+    q, k = _t(), _t()
+    st = lib.csa_index_topk(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 100, None, 16, 16, None, 16,
+                            1 << 20, None)
+    assert st == 1 and b"topk" in lib.csa_last_error()
+    p.topk = 64
+    st = lib.csa_index_topk(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16, 16, None, 16,
+                            64, None)
+    assert st == 3 and b"workspace" in lib.csa_last_error()
+    fp8k = _t(dtype=csa.CSA_FP8_E4M3, scale=None, group=128)
+    st = lib.csa_index_topk(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(fp8k), 1, 1000, None, 16, 16, None, 16,
+                            1 << 30, None)
+    assert st == 1 and b"scales" in lib.csa_last_error()
+
+
+def test_attention_rejects_bad_arguments(lib):
+    p = csa.params(4, 512, 128, 64, 64, 64, 128, 64)  # swa_cap < window
+    q, kv, out = _t(), _t(), _t()
+    st = lib.csa_sparse_swa_attention(ctypes.byref(p), 2, ctypes.byref(q), ctypes.byref(kv), 1, 100, 16, 16, None, None,
+                                      None, 16, None, None, ctypes.byref(out), None, 16, 1 << 30, None)
+    assert st == 1 and b"swa_cap" in lib.csa_last_error()
+    p.swa_cap = 128
+    st = lib.csa_sparse_swa_attention(ctypes.byref(p), 2, ctypes.byref(q), ctypes.byref(kv), 1, 100, 16, 16, None, None,
+                                      None, 16, None, None, ctypes.byref(out), None, 16, 1 << 30, None)
+    assert st == 1 and b"swa_k" in lib.csa_last_error()
+
+
+def test_workspace_size_grows_with_problem(lib):
+    p = csa.params(4, 512, 128, 64, 64, 1024, 128, 128)
+    a = csa.csa_workspace_size(p, 4, 262144)
+    b = csa.csa_workspace_size(p, 8, 262144)
+    assert a >= 4 * 262144 * 4 and b > a
+    p.topk = 0
+    assert csa.csa_workspace_size(p, 4, 2048) > 0

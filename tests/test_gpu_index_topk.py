@@ -1,0 +1,91 @@
+"""a2 indexer + a3 top-k: CUDA path vs the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+from compressed_sparse_attention_compressor_b200 import csa
+from compressed_sparse_attention_compressor_b200 import workloads as Wk
+from oracle import csa_oracle as O
+from tests._harness import check_selection, gpu_index_topk, i32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("k,n_cols", [(1, 10), (64, 1000), (512, 20000), (1024, 100000), (7, 5)])
+def test_topk_alone_is_bit_exact_with_ties(k, n_cols, cuda_lib):
+    """Same fp32 scores on both sides: selection must match exactly,
+    including planted exact ties, -0 vs +0, and rows with n_valid <= k."""
+    rows = 6
+    s = Wk.make_scores(3000 + k, rows, n_cols)
+    n_valid = np.array([n_cols, n_cols - 1, min(n_cols, k), min(n_cols, k + 1), 0, max(n_cols // 3, 1)], np.int32)
+    ld = n_cols + 5
+    buf = np.zeros((rows, ld), np.float32)
+    buf[:, :n_cols] = s
+    scores = torch.from_numpy(buf).cuda()
+    out_idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
+    out_score = torch.empty((rows, k), dtype=torch.float32, device="cuda")
+    csa.csa_topk(scores, rows, ld, i32(n_valid), k, out_idx, out_score)
+    torch.cuda.synchronize()
+    gi, gs = out_idx.cpu().numpy(), out_score.cpu().numpy()
+    for r in range(rows):
+        n = int(n_valid[r])
+        ref = O.topk(buf[r, :n].astype(np.float64), k)
+        assert np.array_equal(np.sort(gi[r]), np.sort(ref)), f"row {r}"
+        sel = gi[r] >= 0
+        assert np.array_equal(gs[r][sel], buf[r, gi[r][sel]])
+        assert np.all(np.isneginf(gs[r][~sel]))
+
+
+def test_topk_all_equal_scores_takes_lowest_indices(cuda_lib):
+    n, k = 5000, 300
+    scores = torch.zeros((2, n), dtype=torch.float32, device="cuda")
+    scores[1, ::2] = -0.0
+    out_idx = torch.empty((2, k), dtype=torch.int32, device="cuda")
+    csa.csa_topk(scores, 2, n, i32([n, n]), k, out_idx)
+    torch.cuda.synchronize()
+    for r in range(2):
+        assert np.array_equal(np.sort(out_idx[r].cpu().numpy()), np.arange(k))
+
+
+IDX_CASES = {
+    # name: (workload, n_queries, batch, cap)
+    "tiny_f32": (Wk.WORKLOADS["tiny"], 3, 3, 1024 + 37),
+    "bf16": (Wk.WORKLOADS["decode64k"], 4, 2, 3000),
+    "fp8": (Wk.WORKLOADS["decode1m"], 3, 3, 5000),
+    "bf16_ratio1": (Wk.WORKLOADS["hybrid_ratio1"].scaled(topk=256), 2, 2, 2500),
+}
+
+
+@pytest.mark.parametrize("name", list(IDX_CASES))
+def test_index_topk_matches_oracle(name, cuda_lib):
+    wl, nq, B, cap = IDX_CASES[name]
+    seed = 3100 + len(name)
+    sI = 1 / np.sqrt(wl.d_idx)
+    kidx = Wk.store(Wk.normal(seed, "kidx", (B, cap, wl.d_idx), sI), wl.idx_dtype, wl.d_idx)
+    q_idx = Wk.store(Wk.normal(seed, "q_idx", (nq, wl.h_idx, wl.d_idx), sI), wl.act_dtype)
+    w = Wk.uniform(seed, "w", (nq, wl.h_idx))
+    q_req = np.arange(nq, dtype=np.int32) % B
+    n_vis = np.array([cap, cap - 17, max(wl.topk // 2, 1), cap - 1][:nq], np.int32)
+    gi, gs = gpu_index_topk(wl, q_idx, w, kidx, B, cap, q_req, n_vis)
+    exact = wl.idx_dtype == "f32"
+    qd = O.decode_stored(q_idx)
+    swaps = 0
+    for i in range(nq):
+        keys = O.decode(kidx.data[q_req[i], : n_vis[i]], kidx.dtype,
+                        None if kidx.scale is None else kidx.scale[q_req[i], : n_vis[i]], kidx.group)
+        s = O.index_scores(qd[i], w[i], keys)
+        swaps += check_selection(gi[i], s, wl.topk, exact, gs[i])
+    print(f"{name}: boundary swaps {swaps}")
+
+
+def test_index_topk_all_negative_dots_select_first_indices(cuda_lib):
+    """Every score is exactly 0 (ReLU of negative dots): the tie rule picks
+    indices 0..k-1."""
+    wl = Wk.WORKLOADS["decode64k"]
+    cap, k = 2000, 512
+    keys = np.abs(Wk.normal(7, "k", (1, cap, wl.d_idx))) / 10
+    q = -np.abs(Wk.normal(7, "q", (1, wl.h_idx, wl.d_idx))) / 10
+    gi, gs = gpu_index_topk(wl, Wk.store(q, "bf16"), Wk.uniform(7, "w", (1, wl.h_idx)), Wk.store(keys, "bf16"), 1, cap,
+                            None, np.array([cap], np.int32), k=k)
+    assert np.array_equal(np.sort(gi[0]), np.arange(k))
+    assert np.all(gs[0] == 0)
