@@ -39,6 +39,7 @@ from compressed_sparse_attention_compressor_b200 import workloads as Wk  # noqa:
 
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = {
+    "index_topk_tc_kernel": "index_tc.cu",
     "index_score_simt_kernel": "index_topk.cu",
     "topk_row_kernel": "index_topk.cu",
     "attn_simt_kernel": "attention.cu",
@@ -87,7 +88,7 @@ def step_bytes(wl, n_vis):
 def kernel_bytes(name, wl, n_vis):
     """Algorithmic bytes of one launch of a kernel of the decode step."""
     B, ea = wl.batch, _eb(wl.act_dtype)
-    if name.startswith("index_score"):
+    if name.startswith("index_"):
         return B * n_vis * key_row_bytes(wl) + B * wl.h_idx * (wl.d_idx * ea + 4)
     if name.startswith("attn_simt"):
         rows = n_vis if wl.dense else min(wl.topk, n_vis)

@@ -266,41 +266,49 @@ attn_simt_kernel(AttnArgs a) {
   }
 }
 
-// Combines the per-split partial states of one query (all heads).
-__global__ void __launch_bounds__(kAttnThreads)
+// Combines the per-split partial states of one (query, head): one CTA each.
+constexpr int kMaxSplits = 256;
+__global__ void __launch_bounds__(128)
 attn_merge_kernel(const float* __restrict__ part, int n_splits, int hq, int d, const float* __restrict__ sink,
                   void* out, int out_dtype, float* lse) {
-  const int qi = blockIdx.x;
-  const int oeb = elem_bytes(out_dtype);
-  for (int h = 0; h < hq; ++h) {
-    const float* base = part + (static_cast<int64_t>(qi) * n_splits * hq + h) * (d + 2);
-    const int64_t sstride = static_cast<int64_t>(hq) * (d + 2);
+  __shared__ float wgt[kMaxSplits];
+  __shared__ float s_ml[2];
+  const int qi = blockIdx.x / hq, h = blockIdx.x % hq;
+  const float* base = part + (static_cast<int64_t>(qi) * n_splits * hq + h) * (d + 2);
+  const int64_t sstride = static_cast<int64_t>(hq) * (d + 2);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     const float sk = sink ? sink[h] : -INFINITY;
     float M = sk;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, base[s * sstride]);
+    for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, __ldg(base + s * sstride));
+    M = warp_max(M);
     float L = 0.f;
     if (M != -INFINITY) {
-      L = (sk == -INFINITY) ? 0.f : __expf(sk - M);
-      for (int s = 0; s < n_splits; ++s) {
-        const float ms = base[s * sstride];
-        if (ms != -INFINITY) L += __expf(ms - M) * base[s * sstride + 1];
+      for (int s = lane; s < n_splits; s += 32) {
+        const float ms = __ldg(base + s * sstride);
+        const float wv = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+        wgt[s] = wv;
+        L += wv * __ldg(base + s * sstride + 1);
       }
+      L = warp_sum(L);
+      if (sk != -INFINITY) L += __expf(sk - M);
     }
-    char* orow = static_cast<char*>(out) + (static_cast<int64_t>(qi) * hq + h) * d * oeb;
-    for (int c = threadIdx.x; c < d; c += kAttnThreads) {
-      float v = 0.f;
-      if (M != -INFINITY) {
-        for (int s = 0; s < n_splits; ++s) {
-          const float ms = base[s * sstride];
-          if (ms != -INFINITY) v = fmaf(__expf(ms - M), base[s * sstride + 2 + c], v);
-        }
-        v /= L;
-      }
-      if (out_dtype == kF32) reinterpret_cast<float*>(orow)[c] = v;
-      else reinterpret_cast<uint16_t*>(orow)[c] = f32_to_bf16_bits(v);
-    }
-    if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(qi) * hq + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
+    if (lane == 0) { s_ml[0] = M; s_ml[1] = L; }
   }
+  __syncthreads();
+  const float M = s_ml[0], L = s_ml[1];
+  const int oeb = elem_bytes(out_dtype);
+  char* orow = static_cast<char*>(out) + (static_cast<int64_t>(qi) * hq + h) * d * oeb;
+  const float inv = (M != -INFINITY) ? 1.f / L : 0.f;
+  for (int c = threadIdx.x; c < d; c += 128) {
+    float v = 0.f;
+    if (M != -INFINITY)
+      for (int s = 0; s < n_splits; ++s) v = fmaf(wgt[s], __ldg(base + s * sstride + 2 + c), v);
+    v *= inv;
+    if (out_dtype == kF32) reinterpret_cast<float*>(orow)[c] = v;
+    else reinterpret_cast<uint16_t*>(orow)[c] = f32_to_bf16_bits(v);
+  }
+  if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(qi) * hq + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
 }
 
 template <int HQ, int D>
@@ -316,7 +324,7 @@ csa_status_t launch_attn_t(AttnArgs a, int nq, cudaStream_t stream) {
   csa_status_t st = check_launch("attn_simt_kernel", stream);
   if (st != CSA_OK || a.n_splits == 1) return st;
   prof_begin(stream);
-  attn_merge_kernel<<<nq, kAttnThreads, 0, stream>>>(a.part, a.n_splits, HQ, D, a.sink, a.out, a.out_dtype, a.lse);
+  attn_merge_kernel<<<nq * HQ, 128, 0, stream>>>(a.part, a.n_splits, HQ, D, a.sink, a.out, a.out_dtype, a.lse);
   return check_launch("attn_merge_kernel", stream);
 }
 
@@ -329,6 +337,7 @@ int attn_splits(int nq, int max_keys) {
   int s = (target + nq - 1) / nq;
   const int max_s = (max_keys + 63) / 64;  // a partial state costs as much as ~128 bf16 rows
   if (s > max_s) s = max_s;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s < 1) s = 1;
   return s;
 }

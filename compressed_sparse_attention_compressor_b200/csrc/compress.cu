@@ -128,6 +128,76 @@ __device__ __forceinline__ void project_row(const float* pooled, int d, const vo
   }
 }
 
+// Largest W_IK staged in shared memory by the projection (bytes).
+constexpr int kMaxWSmem = 160 * 1024;
+
+// All threads: copy W_IK [d][d_idx] into shared memory (16-byte vectors).
+__device__ __forceinline__ void stage_w(uint8_t* wsm, const void* w_ik, int bytes) {
+  const uint4* src = static_cast<const uint4*>(w_ik);
+  uint4* dst = reinterpret_cast<uint4*>(wsm);
+  for (int i = threadIdx.x; i < bytes / 16; i += kCompressThreads) dst[i] = __ldg(src + i);
+}
+
+// All threads: kout[0..d_idx) = pooled[0..d) . W (W staged in shared memory).
+// Thread t owns output pair t % (d_idx/2) over a slice of the d rows; the
+// slices are summed through red[] (256 * 2 floats).  d_idx in {32, 64,
+// 128, 256}.
+__device__ void project_smem(const float* pooled, int d, const uint8_t* wsm, int w_dtype, int d_idx, float* red,
+                             float* kout) {
+  const int P = d_idx / 2, S = kCompressThreads / P;
+  const int t = threadIdx.x, o2 = t % P, sl = t / P;
+  const int r0 = sl * d / S, r1 = (sl + 1) * d / S;
+  float a0 = 0.f, a1 = 0.f;
+  if (w_dtype == kBF16) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(wsm);
+#pragma unroll 8
+    for (int c = r0; c < r1; ++c) {
+      const uint32_t u = w[c * P + o2];
+      const float x = pooled[c];
+      a0 = fmaf(x, __uint_as_float(u << 16), a0);
+      a1 = fmaf(x, __uint_as_float(u & 0xFFFF0000u), a1);
+    }
+  } else {
+    const float2* w = reinterpret_cast<const float2*>(wsm);
+#pragma unroll 8
+    for (int c = r0; c < r1; ++c) {
+      const float2 u = w[c * P + o2];
+      const float x = pooled[c];
+      a0 = fmaf(x, u.x, a0);
+      a1 = fmaf(x, u.y, a1);
+    }
+  }
+  red[sl * d_idx + 2 * o2] = a0;
+  red[sl * d_idx + 2 * o2 + 1] = a1;
+  __syncthreads();
+  if (t < d_idx) {
+    float v = 0.f;
+    for (int q = 0; q < S; ++q) v += red[q * d_idx + t];
+    kout[t] = v;
+  }
+  __syncthreads();
+}
+
+// One warp stores a projected key row (fp32 values in shared memory).
+__device__ __forceinline__ void store_key_row(const float* kv, int d_idx, const OutSpec& ko, int64_t row) {
+  const int lane = threadIdx.x & 31;
+  if (ko.dtype == kFP8) {
+    float amax = 0.f;
+    for (int i = lane; i < d_idx; i += 32) amax = fmaxf(amax, fabsf(kv[i]));
+    amax = warp_max(amax);
+    const float s = amax > 0.f ? amax / 448.f : 1.f;
+    uint8_t* dst = static_cast<uint8_t*>(ko.data) + row * ko.row_stride;
+    for (int i = lane; i < d_idx; i += 32) dst[i] = f32_to_e4m3(kv[i] / s);
+    if (lane == 0) ko.scale[row * ko.scale_stride] = s;
+  } else if (ko.dtype == kBF16) {
+    uint16_t* dst = static_cast<uint16_t*>(ko.data) + row * ko.row_stride;
+    for (int i = lane; i < d_idx; i += 32) dst[i] = f32_to_bf16_bits(kv[i]);
+  } else {
+    float* dst = static_cast<float*>(ko.data) + row * ko.row_stride;
+    for (int i = lane; i < d_idx; i += 32) dst[i] = kv[i];
+  }
+}
+
 __global__ void __launch_bounds__(kCompressThreads)
 compress_kernel(const void* __restrict__ C, const void* __restrict__ Z, int in_dtype, int64_t n_tokens, int d,
                 int m, int64_t n_blocks, OutSpec out, int64_t out_rows, const void* __restrict__ w_ik,
@@ -163,6 +233,22 @@ compress_kernel(const void* __restrict__ C, const void* __restrict__ Z, int in_d
     store_pooled8(out, static_cast<int64_t>(b) * out_rows + j, col, v, valid);
   }
   if (w_ik == nullptr) return;
+  const int wbytes = d * d_idx * elem_bytes(w_dtype);
+  if (wbytes <= kMaxWSmem) {
+    uint8_t* wsm = reinterpret_cast<uint8_t*>(pooled + kCompressNB * d);
+    float* red = reinterpret_cast<float*>(wsm + wbytes);
+    float* kvec = red + 2 * kCompressThreads;
+    stage_w(wsm, w_ik, wbytes);
+    __syncthreads();
+    for (int lb = 0; lb < kCompressNB; ++lb) {
+      const int64_t j = blk0 + lb;
+      if (j >= n_blocks) break;  // uniform over the CTA
+      project_smem(pooled + lb * d, d, wsm, w_dtype, d_idx, red, kvec);
+      if (threadIdx.x < 32) store_key_row(kvec, d_idx, kout, static_cast<int64_t>(b) * out_rows + j);
+      __syncthreads();
+    }
+    return;
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   for (int lb = warp; lb < kCompressNB; lb += kCompressThreads / 32) {
@@ -183,9 +269,15 @@ decode_append_kernel(const int64_t* __restrict__ pos, int m, int d, int act_dtyp
                      void* open_c, void* open_z, void* swa_k, void* swa_v, int swa_dtype, int swa_cap,
                      OutSpec kv, int64_t cap, const void* __restrict__ w_ik, int w_dtype, int d_idx,
                      OutSpec kidx, int32_t* __restrict__ n_visible_out, int64_t* __restrict__ q_pos_out,
-                     int32_t* __restrict__ q_req_out) {
+                     int32_t* __restrict__ q_req_out, uint4* __restrict__ zero, int64_t zero_n16) {
   extern __shared__ float pooled[];  // [d]
   const int b = blockIdx.x;
+  // zero this CTA's share of the caller's control words (later kernels'
+  // counters and histograms)
+  if (zero != nullptr) {
+    const int64_t z0 = zero_n16 * b / gridDim.x, z1 = zero_n16 * (b + 1) / gridDim.x;
+    for (int64_t i = z0 + threadIdx.x; i < z1; i += kCompressThreads) zero[i] = make_uint4(0, 0, 0, 0);
+  }
   const int64_t t = pos[b];
   const int slot_m = static_cast<int>(t % m);
   const int64_t slot_w = t % swa_cap;
@@ -234,6 +326,17 @@ decode_append_kernel(const int64_t* __restrict__ pos, int m, int d, int act_dtyp
     store_pooled8(kv, row, valid ? vec * 8 : 0, v, valid);
   }
   if (w_ik == nullptr) return;
+  const int wbytes = d * d_idx * elem_bytes(w_dtype);
+  if (wbytes <= kMaxWSmem) {
+    uint8_t* wsm = reinterpret_cast<uint8_t*>(pooled + d);
+    float* red = reinterpret_cast<float*>(wsm + wbytes);
+    float* kvec = red + 2 * kCompressThreads;
+    stage_w(wsm, w_ik, wbytes);
+    __syncthreads();
+    project_smem(pooled, d, wsm, w_dtype, d_idx, red, kvec);
+    if (threadIdx.x < 32) store_key_row(kvec, d_idx, kidx, row);
+    return;
+  }
   __syncthreads();
   if (threadIdx.x < 32) project_row(pooled, d, w_ik, w_dtype, d_idx, kidx, row);
 }
@@ -257,7 +360,11 @@ csa_status_t launch_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int b
   const int64_t n_blocks = n_tokens / m;
   if (n_blocks == 0 || batch == 0) return CSA_OK;
   dim3 grid(static_cast<unsigned>((n_blocks + kCompressNB - 1) / kCompressNB), batch);
-  const size_t smem = w_ik ? static_cast<size_t>(kCompressNB) * d * sizeof(float) : 0;
+  size_t smem = w_ik ? static_cast<size_t>(kCompressNB) * d * sizeof(float) : 0;
+  if (w_ik) {
+    const size_t wb = static_cast<size_t>(d) * d_idx * elem_bytes(w_ik->dtype);
+    if (wb <= kMaxWSmem) smem += wb + (2 * kCompressThreads + d_idx) * sizeof(float);
+  }
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   prof_begin(stream);
@@ -269,14 +376,21 @@ csa_status_t launch_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int b
 
 csa_status_t launch_decode_append(const csa_params_t* p, int batch, const csa_decode_caches_t* cc,
                                   const csa_decode_token_t* tok, const int64_t* pos, int32_t* n_visible,
-                                  int64_t* q_pos, int32_t* q_req, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(p->d) * sizeof(float);
+                                  int64_t* q_pos, int32_t* q_req, void* zero, size_t zero_bytes,
+                                  cudaStream_t stream) {
+  size_t smem = static_cast<size_t>(p->d) * sizeof(float);
+  if (tok->w_ik.data) {
+    const size_t wb = static_cast<size_t>(p->d) * p->d_idx * elem_bytes(tok->w_ik.dtype);
+    if (wb <= kMaxWSmem) smem += wb + (2 * kCompressThreads + p->d_idx) * sizeof(float);
+  }
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(decode_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   prof_begin(stream);
   decode_append_kernel<<<batch, kCompressThreads, smem, stream>>>(
       pos, p->m, p->d, tok->c.dtype, tok->c.data, tok->z.data, tok->k_swa.data, tok->v_swa.data,
       cc->open_c.data, cc->open_z.data, cc->swa_k.data, cc->swa_v.data, cc->swa_k.dtype, p->swa_cap,
       make_out(&cc->kv, p->d), cc->cap, tok->w_ik.data, tok->w_ik.dtype, p->d_idx, make_out(&cc->kidx, p->d_idx),
-      n_visible, q_pos, q_req);
+      n_visible, q_pos, q_req, static_cast<uint4*>(zero), static_cast<int64_t>(zero_bytes / 16));
   return check_launch("decode_append_kernel", stream);
 }
 

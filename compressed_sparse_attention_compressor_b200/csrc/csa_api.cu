@@ -15,7 +15,15 @@ csa_status_t launch_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int b
                              int d_idx, const csa_tensor_t* kidx_out, cudaStream_t stream);
 csa_status_t launch_decode_append(const csa_params_t* p, int batch, const csa_decode_caches_t* cc,
                                   const csa_decode_token_t* tok, const int64_t* pos, int32_t* n_visible,
-                                  int64_t* q_pos, int32_t* q_req, cudaStream_t stream);
+                                  int64_t* q_pos, int32_t* q_req, void* zero, size_t zero_bytes,
+                                  cudaStream_t stream);
+bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dtype, int k_dtype);
+size_t index_tc_control_bytes(int batch);
+size_t index_tc_workspace_bytes(int batch, int64_t cap, int k);
+csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
+                                  const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
+                                  float* out_score, void* ws, cudaStream_t stream);
+uint32_t index_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                                 const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
                                 const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
@@ -149,7 +157,12 @@ size_t csa_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_
   c.take<int32_t>(n_queries);
   if (p->topk > 0) {
     c.take<int32_t>(static_cast<size_t>(n_queries) * p->topk);
-    c.take<char>(index_ws_bytes(n_queries, max_entries));
+    size_t ib = index_ws_bytes(n_queries, max_entries);
+    if (p->h_idx > 0 && p->d_idx > 0) {
+      const size_t tb = index_tc_workspace_bytes(n_queries, max_entries, p->topk);
+      if (tb > ib) ib = tb;
+    }
+    c.take<char>(ib);
   }
   const size_t attn = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
   return c.off + attn + 256;
@@ -206,10 +219,19 @@ csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_
   if ((st = check_tensor("k_idx", k_idx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
   if (w == nullptr || n_visible == nullptr || out_idx == nullptr)
     return set_error(CSA_ERR_INVALID_ARG, "null w / n_visible / out_idx");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (q_req == nullptr && n_queries == batch && index_tc_supported(p, batch, cap, q_idx->dtype, k_idx->dtype)) {
+    // one query per request: the fused tensor-core kernel
+    const size_t need = index_tc_workspace_bytes(batch, cap, p->topk);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, index_tc_control_bytes(batch), s);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    return launch_index_topk_tc(p, batch, q_idx, w, k_idx, cap, n_visible, out_idx, out_score, workspace, s);
+  }
   const size_t need = index_ws_bytes(n_queries, cap);
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Carver c(workspace);
   const int64_t ld = round_up(cap, 4);
   float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
@@ -298,15 +320,24 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
   int32_t* q_req = c.take<int32_t>(batch);
   int32_t* idx = nullptr;
   void* index_ws = nullptr;
+  const bool tc = sparse && index_tc_supported(p, batch, cc->cap, tok->q_idx.dtype, cc->kidx.dtype);
   if (sparse) {
     idx = c.take<int32_t>(static_cast<size_t>(batch) * p->topk);
-    index_ws = c.take<char>(index_ws_bytes(batch, cc->cap));
+    size_t ib = index_ws_bytes(batch, cc->cap);
+    const size_t tb = index_tc_workspace_bytes(batch, cc->cap, p->topk);
+    index_ws = c.take<char>(ib > tb ? ib : tb);
   }
   const int max_keys = static_cast<int>((sparse ? p->topk : cc->cap) + p->window);
   void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys));
 
-  if ((st = launch_decode_append(p, batch, cc, tok, pos, n_vis, q_pos, q_req, s)) != CSA_OK) return st;
-  if (sparse) {
+  if ((st = launch_decode_append(p, batch, cc, tok, pos, n_vis, q_pos, q_req, tc ? index_ws : nullptr,
+                                 tc ? index_tc_control_bytes(batch) : 0, s)) != CSA_OK)
+    return st;
+  if (tc) {
+    if ((st = launch_index_topk_tc(p, batch, &tok->q_idx, tok->w, &cc->kidx, cc->cap, n_vis, idx, nullptr, index_ws,
+                                   s)) != CSA_OK)
+      return st;
+  } else if (sparse) {
     const int64_t ld = round_up(cc->cap, 4);
     float* scores = static_cast<float*>(index_ws);
     if ((st = launch_index_score(p, batch, &tok->q_idx, tok->w, &cc->kidx, batch, cc->cap, q_req, n_vis, scores, ld,
@@ -379,6 +410,8 @@ csa_status_t csa_profile_get(int32_t i, const char** name, float* ms) {
 csa_status_t csa_sync_status(csa_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  if (index_tc_take_error() != 0)
+    return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the indexer gave up");
   return CSA_OK;
 }
 

@@ -170,7 +170,10 @@ def check_rows(gpu_vals: np.ndarray, ref: np.ndarray, dtype: str, group: int = 0
             f"bf16 rows differ by {np.abs(gpu_vals - ref).max():g}"
     else:
         codes, scale = O.quantize_groups(ref, group)
-        assert np.allclose(gpu_scale, scale, rtol=1e-6, atol=0), "FP8 scales differ"
+        # the kernel's group maximum is an fp32 pooled value: a few fp32 ulps
+        # of the block's inputs away from the fp64 one
+        rel = np.abs(gpu_scale - scale) / scale
+        assert np.all(rel <= 1e-5), f"FP8 scales differ by {rel.max():.3g} relative"
         gv = O.e4m3_to_f64(gpu_codes)
         ov = O.e4m3_to_f64(codes)
         off = gv != ov

@@ -89,3 +89,60 @@ def test_index_topk_all_negative_dots_select_first_indices(cuda_lib):
                             None, np.array([cap], np.int32), k=k)
     assert np.array_equal(np.sort(gi[0]), np.arange(k))
     assert np.all(gs[0] == 0)
+
+
+# one query per request, q_req = NULL: the fused tensor-core kernel
+TC_CASES = {
+    "fp8_ragged": (Wk.WORKLOADS["decode1m"], 3, 5000, [5000, 4983, 700]),
+    "bf16": (Wk.WORKLOADS["decode64k"], 2, 3000, [3000, 2999]),
+    "fp8_one_request_many_ctas": (Wk.WORKLOADS["decode1m"], 1, 20000, [19999]),
+    "bf16_k2048": (Wk.WORKLOADS["hybrid_ratio1"], 2, 9000, [9000, 8000]),
+    "bf16_fewer_than_k": (Wk.WORKLOADS["decode64k"], 2, 700, [300, 512]),
+}
+
+
+@pytest.mark.parametrize("name", list(TC_CASES))
+def test_index_topk_tensor_core_path(name, cuda_lib):
+    wl, B, cap, n_vis = TC_CASES[name]
+    seed = 3300 + len(name)
+    sI = 1 / np.sqrt(wl.d_idx)
+    kidx = Wk.store(Wk.normal(seed, "kidx", (B, cap, wl.d_idx), sI), wl.idx_dtype, wl.d_idx)
+    q_idx = Wk.store(Wk.normal(seed, "q_idx", (B, wl.h_idx, wl.d_idx), sI), wl.act_dtype)
+    w = Wk.uniform(seed, "w", (B, wl.h_idx))
+    n_vis = np.array(n_vis, np.int32)
+    gi, gs = gpu_index_topk(wl, q_idx, w, kidx, B, cap, None, n_vis)
+    qd = O.decode_stored(q_idx)
+    swaps = 0
+    for i in range(B):
+        keys = O.decode(kidx.data[i, : n_vis[i]], kidx.dtype,
+                        None if kidx.scale is None else kidx.scale[i, : n_vis[i]], kidx.group)
+        s = O.index_scores(qd[i], w[i], keys)
+        swaps += check_selection(gi[i], s, wl.topk, False, gs[i])
+    print(f"{name}: boundary swaps {swaps}")
+
+
+@pytest.mark.parametrize("dt", ["fp8", "bf16"])
+def test_index_topk_tensor_core_all_ties(dt, cuda_lib):
+    """Every score is exactly 0 across many CTAs: the selection is the k
+    lowest indices, assembled by the last CTA of each request."""
+    wl = Wk.WORKLOADS["decode1m" if dt == "fp8" else "decode64k"]
+    B, cap = 2, 30000
+    keys = np.abs(Wk.normal(8, "k", (B, cap, wl.d_idx))) / 10
+    q = -np.abs(Wk.normal(8, "q", (B, wl.h_idx, wl.d_idx))) / 10
+    gi, gs = gpu_index_topk(wl, Wk.store(q, "bf16"), Wk.uniform(8, "w", (B, wl.h_idx)),
+                            Wk.store(keys, dt, wl.d_idx), B, cap, None, np.array([cap, cap - 5], np.int32))
+    for i in range(B):
+        assert np.array_equal(gi[i], np.arange(wl.topk)), "ties must keep the lowest indices, in index order"
+        assert np.all(gs[i] == 0)
+
+
+def test_index_topk_tensor_core_is_deterministic(cuda_lib):
+    wl = Wk.WORKLOADS["decode1m"]
+    B, cap = 2, 40000
+    kidx = Wk.store(Wk.normal(9, "kidx", (B, cap, wl.d_idx)), "fp8", wl.d_idx)
+    q_idx = Wk.store(Wk.normal(9, "q", (B, wl.h_idx, wl.d_idx)), "bf16")
+    w = Wk.uniform(9, "w", (B, wl.h_idx))
+    n_vis = np.array([cap, cap], np.int32)
+    a, sa = gpu_index_topk(wl, q_idx, w, kidx, B, cap, None, n_vis)
+    b, sb = gpu_index_topk(wl, q_idx, w, kidx, B, cap, None, n_vis)
+    assert np.array_equal(a, b) and np.array_equal(sa, sb)
