@@ -25,7 +25,7 @@ STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "C
 
 EXPORTS = ["csa_workspace_size", "csa_compress", "csa_index_topk", "csa_index_score", "csa_topk",
            "csa_sparse_swa_attention", "csa_decode_step", "csa_last_error", "csa_sync_status", "csa_profile_start",
-           "csa_profile_stop", "csa_profile_count", "csa_profile_get"]
+           "csa_profile_stop", "csa_profile_count", "csa_profile_get", "csa_sparse_swa_attention_noalloc"]
 
 
 class CsaError(RuntimeError):
@@ -76,6 +76,7 @@ def load() -> ctypes.CDLL:
         "csa_index_score": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, V, I64, V]),
         "csa_topk": (I32, [V, I32, I64, V, I32, V, V, V, SZ, V]),
         "csa_sparse_swa_attention": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V, SZ, V]),
+        "csa_sparse_swa_attention_noalloc": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V]),
         "csa_decode_step": (I32, [P(Params), I32, P(DecodeCaches), P(DecodeToken), V, T, V, V, SZ, V]),
         "csa_last_error": (ctypes.c_char_p, []),
         "csa_sync_status": (I32, [V]),
@@ -218,6 +219,22 @@ def csa_sparse_swa_attention(p: Params, n_queries: int, q: DevTensor, kv: DevTen
         _ptr(q_req), sk, sv, _ptr(q_pos), _ptr(swa_lo), _ptr(sink), ctypes.byref(out.c()), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
         _stream(stream)), "csa_sparse_swa_attention")
+
+
+def csa_sparse_swa_attention_noalloc(p: Params, n_queries: int, q: DevTensor, kv: DevTensor, batch: int, cap: int,
+                                     idx: torch.Tensor | None, n_visible: torch.Tensor, q_req: torch.Tensor | None,
+                                     swa_k: DevTensor | None, swa_v: DevTensor | None, q_pos: torch.Tensor,
+                                     swa_lo: torch.Tensor | None, sink: torch.Tensor | None, out: DevTensor,
+                                     lse: torch.Tensor | None, stream=None):
+    """csa_sparse_swa_attention without a workspace: for callers that cannot
+    allocate device memory; its scratch is a fixed array inside the library
+    (see include/csa.h)."""
+    sk = ctypes.byref(swa_k.c()) if swa_k is not None else None
+    sv = ctypes.byref(swa_v.c()) if swa_v is not None else None
+    _check(load().csa_sparse_swa_attention_noalloc(
+        ctypes.byref(p), n_queries, ctypes.byref(q.c()), ctypes.byref(kv.c()), batch, cap, _ptr(idx),
+        _ptr(n_visible), _ptr(q_req), sk, sv, _ptr(q_pos), _ptr(swa_lo), _ptr(sink), ctypes.byref(out.c()),
+        _ptr(lse), _stream(stream)), "csa_sparse_swa_attention_noalloc")
 
 
 def decode_caches(kv, kidx, swa_k, swa_v, open_c, open_z, cap) -> DecodeCaches:

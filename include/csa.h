@@ -216,6 +216,29 @@ csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries,
                                       const csa_tensor_t* out, float* lse, void* workspace,
                                       size_t workspace_bytes, csa_stream_t stream);
 
+/* a4 + a5 without a caller workspace -- the pages have no counterpart; this
+ * entry point exists for callers that cannot allocate device memory: a
+ * plugin whose host application owns every byte of device memory, or a
+ * serving loop that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation.  Same arguments, semantics and results as
+ * csa_sparse_swa_attention, minus (workspace, workspace_bytes).  Its scratch
+ * is a fixed 16 MiB device array inside the library, held by every GPU that
+ * loads the library until the process exits; problems that need more
+ * return CSA_ERR_CAPACITY with a message (use csa_sparse_swa_attention
+ * then).  The first call made with a given device current looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  All calls share the one array: calls that overlap on
+ * the GPU (concurrent streams) race, so serialise them.  The call itself
+ * allocates nothing.                                                        */
+csa_status_t csa_sparse_swa_attention_noalloc(const csa_params_t* p, int32_t n_queries,
+                                              const csa_tensor_t* q, const csa_tensor_t* kv,
+                                              int32_t batch, int64_t cap, const int32_t* idx,
+                                              const int32_t* n_visible, const int32_t* q_req,
+                                              const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
+                                              const int64_t* q_pos, const int64_t* swa_lo,
+                                              const float* sink, const csa_tensor_t* out, float* lse,
+                                              csa_stream_t stream);
+
 /* Caches of a decode step (all per request, updated in place). */
 typedef struct csa_decode_caches {
   csa_tensor_t kv;       /* [batch][cap][d] compressed entries                */

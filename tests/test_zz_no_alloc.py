@@ -1,0 +1,67 @@
+"""csa_sparse_swa_attention_noalloc: the attention entry point for callers
+that cannot allocate device memory (a plugin whose host application owns all
+device memory, or a loop that cannot pay cudaMalloc's device-wide
+synchronisation).  It must give the same results as the workspace entry
+point, call after call, and refuse problems larger than its fixed scratch.
+
+This file sorts last so that a run stopping at the first failure has already
+run every other test; it also passes on its own in a fresh process."""
+import numpy as np
+import pytest
+import torch
+
+from compressed_sparse_attention_compressor_b200 import csa
+from compressed_sparse_attention_compressor_b200 import workloads as Wk
+from compressed_sparse_attention_compressor_b200.csa import CsaError, DevTensor
+from tests._harness import ATT_TOL, dev, f32, i32, i64, params_of, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(nq=4, cap=20000):
+    wl = Wk.WORKLOADS["decode1m"]
+    d = wl.d
+    kv = Wk.store(Wk.normal(51, "kv", (nq, cap, d)), "fp8", 64)
+    sk = Wk.store(Wk.normal(51, "sk", (nq, 128, d), 1 / np.sqrt(d)), "bf16")
+    sv = Wk.store(Wk.normal(51, "sv", (nq, 128, d), 1 / np.sqrt(d)), "bf16")
+    q = Wk.store(Wk.normal(51, "q", (nq, wl.h_q, d), 1 / np.sqrt(d)), "bf16")
+    n_vis = np.full(nq, cap, np.int32)
+    idx = Wk.make_indices(51, n_vis, wl.topk)
+    args = dict(q=dev(q), kv=dev(kv), idx=i32(idx), n_vis=i32(n_vis), swa_k=dev(sk), swa_v=dev(sv),
+                q_pos=i64(np.full(nq, 4 * cap - 1)), sink=f32(Wk.normal(51, "sink", (wl.h_q,))))
+    return wl, params_of(wl, 128), nq, cap, args
+
+
+def _run(fn, wl, p, nq, cap, a, with_ws):
+    out = DevTensor.empty((nq, wl.h_q, wl.d), "bf16")
+    lse = torch.empty((nq, wl.h_q), dtype=torch.float32, device="cuda")
+    extra = [csa.workspace(csa.csa_workspace_size(p, nq, cap))] if with_ws else []
+    fn(p, nq, a["q"], a["kv"], nq, cap, a["idx"], a["n_vis"], None, a["swa_k"], a["swa_v"], a["q_pos"], None,
+       a["sink"], out, lse, *extra)
+    torch.cuda.synchronize()
+    return to_f64(out), lse.double().cpu().numpy()
+
+
+def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
+    wl, p, nq, cap, a = _problem()
+    ref_out, ref_lse = _run(csa.csa_sparse_swa_attention, wl, p, nq, cap, a, True)
+    tol = ATT_TOL["fp8"]
+    for _ in range(2):  # the scratch keeps the previous call's contents
+        out, lse = _run(csa.csa_sparse_swa_attention_noalloc, wl, p, nq, cap, a, False)
+        assert np.abs(out - ref_out).max() <= tol
+        assert np.abs(lse - ref_lse).max() <= tol
+
+
+def test_noalloc_refuses_problems_beyond_its_scratch(cuda_lib):
+    """Two queries, dense over a very long claimed context: many splits per
+    query, whose partial states need more than the fixed scratch.  The call
+    is refused before any launch (nothing visible is read either way)."""
+    wl, p, nq, cap, a = _problem(nq=4, cap=4000)
+    two = 2
+    q = DevTensor.empty((two, wl.h_q, wl.d), "bf16")
+    out = DevTensor.empty((two, wl.h_q, wl.d), "bf16")
+    p.topk = 0
+    with pytest.raises(CsaError) as e:
+        csa.csa_sparse_swa_attention_noalloc(p, two, q, a["kv"], nq, 1 << 20, None, i32(np.zeros(two)), None,
+                                             a["swa_k"], a["swa_v"], i64(np.zeros(two)), None, None, out, None)
+    assert "scratch" in str(e.value) and e.value.status == 3
