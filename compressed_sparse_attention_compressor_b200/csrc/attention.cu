@@ -300,13 +300,35 @@ attn_merge_kernel(const float* __restrict__ part, int n_splits, int hq, int d, c
   const int oeb = elem_bytes(out_dtype);
   char* orow = static_cast<char*>(out) + (static_cast<int64_t>(qi) * hq + h) * d * oeb;
   const float inv = (M != -INFINITY) ? 1.f / L : 0.f;
-  for (int c = threadIdx.x; c < d; c += 128) {
-    float v = 0.f;
-    if (M != -INFINITY)
-      for (int s = 0; s < n_splits; ++s) v = fmaf(wgt[s], __ldg(base + s * sstride + 2 + c), v);
-    v *= inv;
-    if (out_dtype == kF32) reinterpret_cast<float*>(orow)[c] = v;
-    else reinterpret_cast<uint16_t*>(orow)[c] = f32_to_bf16_bits(v);
+  // columns c, c+128, ... of this thread; the split states are read in
+  // batches of 8 splits, all loads of a batch issued before use
+  for (int c0 = threadIdx.x; c0 < d; c0 += 128 * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+      for (int s0 = 0; s0 < n_splits; s0 += 8) {
+        float v[8][4];
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int s = s0 + b, c = c0 + q * 128;
+            v[b][q] = (s < n_splits && c < d) ? __ldg(base + s * sstride + 2 + c) : 0.f;
+          }
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (s0 + b < n_splits) acc[q] = fmaf(wgt[s0 + b], v[b][q], acc[q]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = c0 + q * 128;
+      if (c >= d) continue;
+      const float o = acc[q] * inv;
+      if (out_dtype == kF32) reinterpret_cast<float*>(orow)[c] = o;
+      else reinterpret_cast<uint16_t*>(orow)[c] = f32_to_bf16_bits(o);
+    }
   }
   if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(qi) * hq + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
 }
@@ -330,6 +352,14 @@ csa_status_t launch_attn_t(AttnArgs a, int nq, cudaStream_t stream) {
 
 }  // namespace
 
+csa_status_t launch_attn_merge(const float* part, int nq, int n_splits, int hq, int d, const float* sink, void* out,
+                               int out_dtype, float* lse, cudaStream_t stream) {
+  if (n_splits > kMaxSplits) return set_error(CSA_ERR_UNSUPPORTED, "%d attention splits (max %d)", n_splits, kMaxSplits);
+  prof_begin(stream);
+  attn_merge_kernel<<<nq * hq, 128, 0, stream>>>(part, n_splits, hq, d, sink, out, out_dtype, lse);
+  return check_launch("attn_merge_kernel", stream);
+}
+
 // Splits per query: enough CTAs to cover the GPU twice for small query
 // counts; one split (no merge pass) once the queries alone fill it.
 int attn_splits(int nq, int max_keys) {
@@ -342,10 +372,30 @@ int attn_splits(int nq, int max_keys) {
   return s;
 }
 
+bool attn_tc_supported(const csa_params_t* p, int q_dtype, int kv_dtype, int swa_dtype, bool has_window);
+size_t attn_tc_workspace_bytes(int nq, int max_keys);
+int attn_tc_splits(int max_keys);
+csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
+                                 int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
+                                 const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
+                                 const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
+                                 const csa_tensor_t* out, float* lse, void* workspace, int max_keys,
+                                 cudaStream_t stream);
+
+// The tensor-core attention takes few queries, each cut into 128-key
+// splits (decode); many queries (prefill) use the CUDA-core kernel.
+static bool attn_tc_shape(int nq, int hq, int d, int max_keys) {
+  return hq == 64 && d == 512 && nq <= 64 && attn_tc_splits(max_keys) <= kMaxSplits;
+}
+
 size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys) {
   const int s = attn_splits(nq, max_keys);
-  if (s <= 1) return 0;
-  return static_cast<size_t>(nq) * s * hq * (d + 2) * sizeof(float);
+  size_t b = s <= 1 ? 0 : static_cast<size_t>(nq) * s * hq * (d + 2) * sizeof(float);
+  if (attn_tc_shape(nq, hq, d, max_keys)) {
+    const size_t t = attn_tc_workspace_bytes(nq, max_keys);
+    if (t > b) b = t;
+  }
+  return b;
 }
 
 csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
@@ -354,6 +404,10 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
                               void* workspace, int max_keys, cudaStream_t stream) {
   if (nq == 0) return CSA_OK;
+  if (attn_tc_shape(nq, p->h_q, p->d, max_keys) &&
+      attn_tc_supported(p, q->dtype, kv->dtype, swa_k ? swa_k->dtype : kBF16, p->window > 0))
+    return launch_attention_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink,
+                               out, lse, workspace, max_keys, stream);
   AttnArgs a;
   a.q = q->data; a.q_dtype = q->dtype;
   a.kv = kv->data; a.kv_scale = kv->scale; a.kv_dtype = kv->dtype;

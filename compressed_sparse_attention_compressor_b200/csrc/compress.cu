@@ -17,6 +17,7 @@
 // max|x| / 448.  The optional indexer-key projection (entry . W_IK) runs
 // from the fp32 pooled entries held in shared memory, one warp per entry.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -35,27 +36,42 @@ struct OutSpec {
 };
 
 // Pools 8 channels [col, col+8) of one block.  rowC(i) / rowZ(i) give the
-// i-th row of the block (i < m).
+// i-th row of the block (i < m).  Rows are loaded four at a time, all four
+// loads issued before their use: first the block maximum, then the
+// exp-weighted sums.
 template <class RowC, class RowZ>
 __device__ __forceinline__ void pool8(RowC rowC, RowZ rowZ, int in_dtype, int m, int col, float out[8]) {
   float mx[8], den[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; den[e] = 0.f; out[e] = 0.f; }
-  float z[8], c[8];
-  for (int i = 0; i < m; ++i) {
-    load8(rowZ(i), in_dtype, col, nullptr, 1, z);
+  for (int i0 = 0; i0 < m; i0 += 4) {
+    float z[4][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], z[e]);
+    for (int b = 0; b < 4; ++b)
+      if (i0 + b < m) load8(rowZ(i0 + b), in_dtype, col, nullptr, 1, z[b]);
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if (i0 + b < m)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], z[b][e]);
   }
-  for (int i = 0; i < m; ++i) {
-    load8(rowZ(i), in_dtype, col, nullptr, 1, z);
-    load8(rowC(i), in_dtype, col, nullptr, 1, c);
+  for (int i0 = 0; i0 < m; i0 += 4) {
+    float z[4][8], c[4][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float a = expf(z[e] - mx[e]);
-      den[e] += a;
-      out[e] = fmaf(a, c[e], out[e]);
-    }
+    for (int b = 0; b < 4; ++b)
+      if (i0 + b < m) {
+        load8(rowZ(i0 + b), in_dtype, col, nullptr, 1, z[b]);
+        load8(rowC(i0 + b), in_dtype, col, nullptr, 1, c[b]);
+      }
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if (i0 + b < m)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a = expf(z[b][e] - mx[e]);
+          den[e] += a;
+          out[e] = fmaf(a, c[b][e], out[e]);
+        }
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = out[e] / den[e];
@@ -270,15 +286,29 @@ decode_append_kernel(const int64_t* __restrict__ pos, int m, int d, int act_dtyp
                      OutSpec kv, int64_t cap, const void* __restrict__ w_ik, int w_dtype, int d_idx,
                      OutSpec kidx, int32_t* __restrict__ n_visible_out, int64_t* __restrict__ q_pos_out,
                      int32_t* __restrict__ q_req_out, uint4* __restrict__ zero, int64_t zero_n16) {
-  extern __shared__ float pooled[];  // [d]
+  extern __shared__ __align__(16) float pooled[];  // [d], then W_IK, reduction scratch
+  __shared__ uint64_t wbar;
   const int b = blockIdx.x;
+  const int64_t t = pos[b];
+  const bool closes = (t + 1) % m == 0;
+  const int wbytes = w_ik ? d * d_idx * elem_bytes(w_dtype) : 0;
+  const bool w_smem = w_ik != nullptr && closes && wbytes <= kMaxWSmem;
+  uint8_t* wsm = reinterpret_cast<uint8_t*>(pooled + d);
+  if (w_smem && threadIdx.x == 0) {
+    // W_IK by TMA bulk copies, in flight while the block is pooled
+    sm100::mbar_init(&wbar, 1);
+    sm100::fence_barrier_init();
+    sm100::mbar_arrive_expect_tx(&wbar, wbytes);
+    for (int off = 0; off < wbytes; off += 32768)
+      sm100::bulk_load(wsm + off, static_cast<const uint8_t*>(w_ik) + off, min(32768, wbytes - off), &wbar);
+  }
+  __syncthreads();  // the barrier's initialisation is visible to every waiter
   // zero this CTA's share of the caller's control words (later kernels'
   // counters and histograms)
   if (zero != nullptr) {
     const int64_t z0 = zero_n16 * b / gridDim.x, z1 = zero_n16 * (b + 1) / gridDim.x;
     for (int64_t i = z0 + threadIdx.x; i < z1; i += kCompressThreads) zero[i] = make_uint4(0, 0, 0, 0);
   }
-  const int64_t t = pos[b];
   const int slot_m = static_cast<int>(t % m);
   const int64_t slot_w = t % swa_cap;
   const int ea = elem_bytes(act_dtype), es = elem_bytes(swa_dtype);
@@ -304,7 +334,7 @@ decode_append_kernel(const int64_t* __restrict__ pos, int m, int d, int act_dtyp
     q_pos_out[b] = t;
     q_req_out[b] = b;
   }
-  if ((t + 1) % m != 0) return;  // uniform across the CTA
+  if (!closes) return;  // uniform across the CTA
   const int64_t row = static_cast<int64_t>(b) * cap + (t + 1) / m - 1;
   // The current token's row is read from c_t / z_t, the others from the
   // open-block buffer (written by earlier steps).
@@ -326,13 +356,11 @@ decode_append_kernel(const int64_t* __restrict__ pos, int m, int d, int act_dtyp
     store_pooled8(kv, row, valid ? vec * 8 : 0, v, valid);
   }
   if (w_ik == nullptr) return;
-  const int wbytes = d * d_idx * elem_bytes(w_dtype);
-  if (wbytes <= kMaxWSmem) {
-    uint8_t* wsm = reinterpret_cast<uint8_t*>(pooled + d);
+  if (w_smem) {
     float* red = reinterpret_cast<float*>(wsm + wbytes);
     float* kvec = red + 2 * kCompressThreads;
-    stage_w(wsm, w_ik, wbytes);
-    __syncthreads();
+    // bounded wait; on a timeout the key row is left unwritten
+    if (!__syncthreads_and(sm100::mbar_wait(&wbar, 0, 1u << 22) ? 1 : 0)) return;
     project_smem(pooled, d, wsm, w_dtype, d_idx, red, kvec);
     if (threadIdx.x < 32) store_key_row(kvec, d_idx, kidx, row);
     return;

@@ -24,6 +24,7 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
                                   float* out_score, void* ws, cudaStream_t stream);
 uint32_t index_tc_take_error();
+uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                                 const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
                                 const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
@@ -412,6 +413,8 @@ csa_status_t csa_sync_status(csa_stream_t stream) {
   if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
   if (index_tc_take_error() != 0)
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the indexer gave up");
+  if (attn_tc_take_error() != 0)
+    return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the attention gave up");
   return CSA_OK;
 }
 
