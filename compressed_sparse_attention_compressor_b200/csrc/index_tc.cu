@@ -30,14 +30,20 @@
 //
 // Top-k (score descending, lower index first on exact ties): a radix select
 // on the ordered 32-bit key of each fp32 score, distributed over the CTAs
-// of a request: pass 1 histograms bits 31..20, pass 2 bits 19..8 of the keys
-// in the boundary bin, each CTA adding its shared-memory histogram into a
-// global one, separated by bounded per-request grid barriers.  Every CTA
-// then stages, in index order, its keys above the 24-bit boundary prefix and
-// those equal to it; the last CTA of the request to finish (atomic counter,
-// no waiting) concatenates them in chunk order -- which is index order --
-// and resolves the remaining boundary entries exactly (low 8 bits, then
-// lowest indices), so the output order is deterministic.
+// of a request.  The histogram of key bits 31..20 is built while the keys
+// stream; each CTA adds it into a global per-request histogram, and after a
+// bounded per-request grid barrier every CTA finds the boundary bin (a
+// crowded bin takes one more distributed level, bits 19..8).  Each CTA then
+// classifies its scores once: entries above the boundary prefix stay in its
+// shared memory, entries at the prefix are published to global memory, both
+// lists in index order; the per-chunk counts are exchanged at a second
+// barrier.  From the chunk prefix sums every CTA writes its own entries
+// above the boundary straight to their output slots, loads the request's
+// boundary entries (a few thousand) into shared memory, resolves the
+// remaining key bits with shared-memory radix levels -- all CTAs reach the
+// same threshold key T and count -- and writes its own selected boundary
+// entries.  The output is deterministic: entries above the boundary in
+// index order, then the selected boundary entries in index order.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -56,45 +62,52 @@ constexpr int kDI = 128;
 constexpr int kEpiWarps = 8;                     // two groups of four, alternating tiles
 constexpr int kThreads = 32 * (2 + kEpiWarps);   // producer, MMA, epilogue
 constexpr int kPrep = kThreads - 32;             // threads preparing the query (warps 1..)
-constexpr int kNAcc = 4;                         // accumulator buffers (64 TMEM columns each)
-constexpr int kScoreCol = kNAcc * kHeads;        // first TMEM column holding scores (one per tile)
-constexpr int kMaxChunkTiles = 512 - kScoreCol;
+constexpr int kNAcc = 2;                         // accumulator buffers, one per epilogue group
+constexpr int kAccCols = 128;                    // TMEM columns per accumulator
+constexpr int kScoreCol = kNAcc * kAccCols;      // first TMEM column holding scores (one per tile)
+constexpr int kMaxChunkTiles = 224;              // tiles of one CTA (TMEM columns, shared-memory scores)
 constexpr int kTmemCols = 512;
 constexpr int kHistBins = 4096;
 constexpr int kEqCache = 8192;                   // boundary entries resolved in shared memory
+constexpr int kACache = 2048;                    // entries above the boundary kept in shared memory
+constexpr int kMaxChunks = 148;                  // CTAs of one request (<= SMs)
+constexpr int kSStages = 16;                     // FP8 row-scale ring (one 512-byte tile each)
 constexpr uint32_t kWaitLimit = 1u << 22;        // mbarrier polls
 constexpr uint32_t kSpinLimit = 1u << 22;        // grid-barrier polls (~64 ns apart)
+static_assert(kScoreCol + kMaxChunkTiles <= kTmemCols, "TMEM columns");
 
 __device__ uint32_t g_index_tc_error = 0;  // bit 0: a bounded wait gave up
 
 template <bool FP8>
 struct Cfg {
-  static constexpr int kStageBytes = FP8 ? 16384 : 32768;
-  static constexpr int kStages = FP8 ? 9 : 5;
-  static constexpr int kScaleBytes = FP8 ? kTileM * 4 : 0;  // per stage
+  // one TMA stage = 32 KB: two FP8 key tiles (one 256-row box) or one bf16 tile
+  static constexpr int kTPS = FP8 ? 2 : 1;
+  static constexpr int kStageBytes = 32768;
+  static constexpr int kStages = 5;
   static constexpr int oStages = 0;
-  static constexpr int oScales = kStages * kStageBytes;
-  static constexpr int oB = oScales + (kStages * kScaleBytes + 1023) / 1024 * 1024;
-  static constexpr int oQ = oB + 16384;            // raw query staging (bf16)
-  static constexpr int oHist = oQ + 16384;          // two group histograms
+  static constexpr int oScales = kStages * kStageBytes;                 // FP8: [kSStages][128] fp32
+  static constexpr int oB = oScales + (FP8 ? kSStages * kTileM * 4 : 0);
+  static constexpr int oHist = oB + 16384;          // two group histograms; the raw query before them
+  static constexpr int oQ = oHist;
   static constexpr int oW = oHist + 2 * kHistBins * 4;
   static constexpr int oBars = oW + kHeads * 4;
   static constexpr int oMisc = oBars + 512;
   static constexpr int kSmem = oMisc + 256 + 1024;
-  static constexpr uint32_t kIdesc = FP8 ? idesc(0, 0, kTileM, kHeads) : idesc(1, 1, kTileM, kHeads);
-  static constexpr uint32_t kEmptyCount = FP8 ? 1 + 128 : 1;  // MMA commit (+ epilogue scale reads)
-  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kNAcc + 2) <= 512, "mbarrier area");
+  // FP8: N = 128 = both E4M3 terms of the split query (rows 0..63 and 64..127 of B)
+  static constexpr uint32_t kIdesc = FP8 ? idesc(0, 0, kTileM, 2 * kHeads) : idesc(1, 1, kTileM, kHeads);
+  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 4) <= 512, "mbarrier area");
   static_assert(oB % 1024 == 0, "operand alignment");
-  // phase-2 scratch, inside the (then idle) stage ring
-  static constexpr int pHist = 0;                         // merged histogram
-  static constexpr int pScratch = kHistBins * 4;          // 256 words
-  static constexpr int pCpre = pScratch + 1024;           // 320 words
-  static constexpr int pCntA = pCpre + 1536;              // [kMaxChunkTiles][4] words each
-  static constexpr int pCntE = pCntA + kMaxChunkTiles * 16;
-  static constexpr int pOffA = pCntE + kMaxChunkTiles * 16;
-  static constexpr int pOffE = pOffA + kMaxChunkTiles * 16;
-  static constexpr int pEq = pOffE + kMaxChunkTiles * 16;
-  static_assert(pEq + kEqCache * 8 <= oScales, "phase-2 scratch must fit in the stage ring");
+  static_assert(kSmem <= 232448, "shared memory");
+  // phase-2 scratch, inside the (then idle) stage and scale rings
+  static constexpr int pHist = 0;                              // [kHistBins] histogram
+  static constexpr int pScratch = pHist + kHistBins * 4;       // 512 words
+  static constexpr int pCpre = pScratch + 2048;                // [2][kMaxChunks + 4] chunk prefixes
+  static constexpr int pACache = pCpre + 2 * (kMaxChunks + 4) * 4;   // this chunk's entries above the boundary
+  static constexpr int pScores = pACache + kACache * 8;        // this chunk's scores, index order
+  static constexpr int pEq = pScores;                          // later: the request's boundary entries
+  static_assert(pScores + kMaxChunkTiles * kTileM * 4 <= oB, "phase-2 scores must fit in the rings");
+  static_assert(pEq + kEqCache * 8 <= oB, "phase-2 boundary list must fit in the rings");
+  static_assert(pACache % 16 == 0 && pScores % 16 == 0, "phase-2 alignment");
 };
 
 struct IdxArgs {
@@ -108,12 +121,10 @@ struct IdxArgs {
   int32_t* out_idx;
   float* out_score;
   uint32_t* ghist;         // [batch][2][4096]  (zero on entry)
-  uint32_t* sync;          // [batch][4]        (zero on entry): barrier, done
-  uint32_t* cnt;           // [batch][chunks][2]
-  int32_t* st_idx;         // [batch][chunks][k]
-  float* st_score;
-  int32_t* eq_idx;         // [batch][chunks][kMaxChunkTiles * 128]
-  float* eq_score;
+  uint32_t* sync;          // [batch][4]        (zero on entry): barrier counter
+  uint32_t* cnt;           // [batch][chunks][2] entries above / at the boundary per chunk
+  uint2* st;               // [batch][chunks][k] (index, score bits) above the boundary, beyond kACache
+  uint2* eq;               // [batch][chunks][kMaxChunkTiles * 128] (index, score bits) at the boundary
 };
 
 struct Shared {
@@ -151,21 +162,26 @@ __device__ bool request_barrier(uint32_t* ctr, uint32_t target, Shared& sh) {
   return sh.bcast[7] != 0;
 }
 
-// Whole block: bin b of a shared-memory histogram of kHistBins bins,
-// scanned from the top, with above(b) < need <= above(b) + hist[b]; writes
-// (b, above) to bcast[0..1].  Threads 0..127 own 32 consecutive bins each.
-__device__ void find_bin_block(const uint32_t* hist, uint32_t need, Shared& sh, uint32_t* scratch) {
+// Whole block: bin b of a shared-memory histogram of `nbins` bins (a power
+// of two, 128..kHistBins), scanned from the top, with
+// above(b) < need <= above(b) + hist[b]; writes (b, above) to bcast[0..1].
+// Threads 0..127 own nbins / 128 consecutive bins each.
+__device__ void find_bin_block(const uint32_t* hist, int nbins, uint32_t need, Shared& sh, uint32_t* scratch) {
   const int tid = threadIdx.x;
-  constexpr int per = kHistBins / 128;
+  const int per = nbins / 128;
   uint32_t mine = 0;
-  if (tid < 128) {
-#pragma unroll
-    for (int i = 0; i < per; i += 4) {
-      const uint4 v = *reinterpret_cast<const uint4*>(hist + tid * per + i);
-      mine += v.x + v.y + v.z + v.w;
-    }
-    scratch[tid] = mine;
+  // a histogram that holds fewer than `need` entries (never produced by the
+  // kernel: the counts add up to the visible entries) selects bin 0
+  if (tid == 0) {
+    sh.bcast[0] = 0;
+    sh.bcast[1] = 0;
   }
+  if (tid < 128)
+    for (int i = 0; i < per; i += 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(hist + tid * per + i);
+      mine += v.x + v.y;
+    }
+  if (tid < 128) scratch[tid] = mine;
   __syncthreads();
   if (tid < 32) {
     uint32_t t4[4], s4 = 0;
@@ -206,6 +222,44 @@ __device__ void find_bin_block(const uint32_t* hist, uint32_t need, Shared& sh, 
   __syncthreads();
 }
 
+// Whole block: exclusive prefix sums over the block (thread order) of two
+// per-thread counts, and their totals.  scratch: 2 * warps words.
+__device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, uint32_t& oa, uint32_t& ob, uint32_t& ta,
+                                            uint32_t& tb, uint32_t* scratch) {
+  constexpr int W = kThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t xa = __shfl_up_sync(0xFFFFFFFFu, ia, o), xb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+    if (lane >= o) {
+      ia += xa;
+      ib += xb;
+    }
+  }
+  if (lane == 31) {
+    scratch[warp] = ia;
+    scratch[W + warp] = ib;
+  }
+  __syncthreads();
+  uint32_t pa = 0, pb = 0, sa = 0, sb = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const uint32_t x = scratch[w], y = scratch[W + w];
+    if (w < warp) {
+      pa += x;
+      pb += y;
+    }
+    sa += x;
+    sb += y;
+  }
+  oa = pa + ia - a;
+  ob = pb + ib - b;
+  ta = sa;
+  tb = sb;
+  __syncthreads();
+}
+
 // Block-wide index-ordered compaction step: rank of this thread's flagged
 // item among the block's flagged items, and the block totals, for two flags.
 __device__ __forceinline__ void block_rank2(bool f0, bool f1, uint32_t& r0, uint32_t& r1, uint32_t& t0,
@@ -234,26 +288,68 @@ __device__ __forceinline__ void block_rank2(bool f0, bool f1, uint32_t& r0, uint
   __syncthreads();
 }
 
-// One warp: exclusive prefix sums of cnt[0..n) into off[0..n); returns the
-// total (valid in every lane).
-__device__ uint32_t warp_exclusive_scan(const uint32_t* cnt, uint32_t* off, int n) {
+// One warp: in-place exclusive prefix sums of v[0..n); returns the total
+// (valid in every lane).
+__device__ uint32_t warp_scan_inplace(uint32_t* v, int n) {
   const int lane = threadIdx.x & 31;
   const int seg = (n + 31) / 32;
   const int lo = min(n, lane * seg), hi = min(n, lo + seg);
   uint32_t mine = 0;
-  for (int i = lo; i < hi; ++i) mine += cnt[i];
+  for (int i = lo; i < hi; ++i) mine += v[i];
   uint32_t incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
+    const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += x;
   }
   uint32_t run = incl - mine;
   for (int i = lo; i < hi; ++i) {
-    off[i] = run;
-    run += cnt[i];
+    const uint32_t x = v[i];
+    v[i] = run;
+    run += x;
   }
+  __syncwarp();
   return __shfl_sync(0xFFFFFFFFu, incl, 31);
+}
+
+// Whole block: a global histogram of kHistBins words into shared memory,
+// every load issued before the first store.
+__device__ __forceinline__ void load_hist(uint32_t* dst, const uint32_t* src) {
+  constexpr int N4 = kHistBins / 4, R = (N4 + kThreads - 1) / kThreads;
+  uint4 v[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    const int i = threadIdx.x + j * kThreads;
+    if (i < N4) v[j] = __ldcg(reinterpret_cast<const uint4*>(src) + i);
+  }
+#pragma unroll
+  for (int j = 0; j < R; ++j) {
+    const int i = threadIdx.x + j * kThreads;
+    if (i < N4) reinterpret_cast<uint4*>(dst)[i] = v[j];
+  }
+}
+
+// Whole block: sum of two per-thread counts over the block (scratch: 2 * warps words).
+__device__ __forceinline__ void block_sum2(uint32_t& a, uint32_t& b, uint32_t* scratch) {
+  constexpr int W = kThreads / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+    b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    scratch[threadIdx.x >> 5] = a;
+    scratch[W + (threadIdx.x >> 5)] = b;
+  }
+  __syncthreads();
+  a = 0;
+  b = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    a += scratch[w];
+    b += scratch[W + w];
+  }
+  __syncthreads();
 }
 
 template <bool FP8>
@@ -268,9 +364,11 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   float* ws = reinterpret_cast<float*>(smem + C::oW);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::oBars);
   uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
-  uint64_t* tempty = tfull + kNAcc;
-  uint64_t* qbar = tempty + kNAcc;
+  uint64_t* sfull = empty + C::kStages;
+  uint64_t* sempty = sfull + kSStages;
+  uint64_t* tfull = sempty + kSStages;  // a pair of tiles' accumulators are ready
+  uint64_t* tempty = tfull + 1;          // ... and have been read back
+  uint64_t* qbar = tempty + 1;
   uint64_t* mdone = qbar + 1;
   uint8_t* Bs = smem + C::oB;
   const float* scale_ring = reinterpret_cast<const float*>(smem + C::oScales);
@@ -288,18 +386,19 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::kEmptyCount);
+      mbar_init(&empty[s], 1);  // the MMA commit
     }
-    for (int b = 0; b < kNAcc; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 128);  // the epilogue group that read the scales
     }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, kNAcc * 128);
     mbar_init(qbar, 1);
     mbar_init(mdone, 1);
     sh.fail = 0;
     fence_barrier_init();
   }
-  for (int i = tid; i < 2 * kHistBins; i += kThreads) ghist0[i] = 0;
   __syncthreads();
 
   // ================= phase 1: stream the keys, scores into TMEM =================
@@ -308,30 +407,47 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       // the query first, so that it is not queued behind the key stream
       mbar_arrive_expect_tx(qbar, kHeads * kDI * 2);
       bulk_load(smem + C::oQ, a.q_idx + static_cast<int64_t>(r) * kHeads * kDI, kHeads * kDI * 2, qbar);
-      int issued = 0;
-      for (int t = 0; t < nt; ++t) {
-        const int s = t % C::kStages;
-        const uint32_t ph = (t / C::kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, kWaitLimit)) {
+      int issued = 0, sissued = 0;
+      const int nst = (nt + C::kTPS - 1) / C::kTPS;
+      for (int p = 0; p < nst && !sh.fail; ++p) {
+        const int s = p % C::kStages;
+        if (!mbar_wait(&empty[s], ((p / C::kStages) & 1) ^ 1, kWaitLimit)) {
           atomicOr(&g_index_tc_error, 1u);
           sh.fail = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes + C::kScaleBytes);
-        const int64_t row0 = static_cast<int64_t>(t0 + t) * kTileM;
-        const int y = static_cast<int>(r * a.cap + row0);
+        const int t = p * C::kTPS;
+        const int y = static_cast<int>(r * a.cap + static_cast<int64_t>(t0 + t) * kTileM);
         uint8_t* dst = smem + C::oStages + s * C::kStageBytes;
-        tma_load_2d(dst, &kmap, &full[s], 0, y);
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         if constexpr (FP8) {
-          tma_load_2d(smem + C::oScales + s * C::kScaleBytes, &smap, &full[s], static_cast<int>(row0), r);
+          tma_load_2d(dst, &kmap, &full[s], 0, y);  // 256 rows: tiles t and t + 1
         } else {
+          tma_load_2d(dst, &kmap, &full[s], 0, y);
           tma_load_2d(dst + 16384, &kmap, &full[s], 64, y);
         }
-        issued = t + 1;
+        issued = p + 1;
+        if constexpr (FP8) {
+          for (int j = 0; j < C::kTPS && t + j < nt; ++j) {
+            const int u = t + j, ss = u % kSStages;
+            if (!mbar_wait(&sempty[ss], ((u / kSStages) & 1) ^ 1, kWaitLimit)) {
+              atomicOr(&g_index_tc_error, 1u);
+              sh.fail = 1;
+              break;
+            }
+            mbar_arrive_expect_tx(&sfull[ss], kTileM * 4);
+            tma_load_2d(smem + C::oScales + ss * kTileM * 4, &smap, &sfull[ss],
+                        static_cast<int>(static_cast<int64_t>(t0 + u) * kTileM), r);
+            sissued = u + 1;
+          }
+        }
       }
-      if (sh.fail)  // let the copies still in flight land before the CTA winds down
-        for (int t = max(0, issued - C::kStages); t < issued; ++t)
-          mbar_wait(&full[t % C::kStages], (t / C::kStages) & 1, kWaitLimit);
+      if (sh.fail) {  // let the copies still in flight land before the CTA winds down
+        for (int p = max(0, issued - C::kStages); p < issued; ++p)
+          mbar_wait(&full[p % C::kStages], (p / C::kStages) & 1, kWaitLimit);
+        for (int u = max(0, sissued - kSStages); u < sissued; ++u)
+          mbar_wait(&sfull[u % kSStages], (u / kSStages) & 1, kWaitLimit);
+      }
     }
   } else {
     // warps 1..: TMEM, head weights, query operand
@@ -400,92 +516,132 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     const uint32_t tmem = sh.tmem_base;
 
     if (warp == 1) {
-      // MMA issuer
+      // MMA issuer.  Tiles go in pairs (2p -> accumulator 0, 2p + 1 -> 1)
+      // with their K steps interleaved; per pair it polls one barrier for
+      // the keys (FP8) and one for the accumulators, and commits twice (an
+      // mbarrier poll in this thread stalls the MMA issue for ~150 cycles).
       if (lane == 0 && !sh.fail) {
         const uint32_t b_base = smem_u32(Bs);
-        for (int t = 0; t < nt; ++t) {
-          const int s = t % C::kStages;
-          const uint32_t ph = (t / C::kStages) & 1;
-          const int acc = t % kNAcc;
-          const uint32_t aph = (t / kNAcc) & 1;
-          if (!mbar_wait(&full[s], ph, kWaitLimit) || !mbar_wait(&tempty[acc], aph ^ 1, kWaitLimit)) {
+        for (int p = 0; 2 * p < nt; ++p) {
+          const int ta = 2 * p;
+          const bool two = ta + 1 < nt;
+          int sa, sb;
+          bool ok;
+          if constexpr (FP8) {
+            sa = sb = p % C::kStages;
+            ok = mbar_wait(&full[sa], (p / C::kStages) & 1, kWaitLimit);
+          } else {
+            sa = ta % C::kStages;
+            sb = (ta + 1) % C::kStages;
+            ok = mbar_wait(&full[sa], (ta / C::kStages) & 1, kWaitLimit);
+            if (ok && two) ok = mbar_wait(&full[sb], ((ta + 1) / C::kStages) & 1, kWaitLimit);
+          }
+          if (ok) ok = mbar_wait(tempty, (p & 1) ^ 1, kWaitLimit);
+          if (!ok) {
             atomicOr(&g_index_tc_error, 1u);
             sh.fail = 1;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + acc * kHeads;
-          const uint32_t a_base = smem_u32(smem + C::oStages + s * C::kStageBytes);
+          const uint32_t a0 = smem_u32(smem + C::oStages + sa * C::kStageBytes);
+          const uint32_t a1 = FP8 ? a0 + 16384 : smem_u32(smem + C::oStages + sb * C::kStageBytes);
           if constexpr (FP8) {
+            // N = 128: the key tile is read once for both query terms
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = desc_k_sw128(a_base + kk * 32);
-              mma_f8f6f4(d, ad, desc_k_sw128(b_base + kk * 32), C::kIdesc, kk > 0 ? 1u : 0u);
-              mma_f8f6f4(d, ad, desc_k_sw128(b_base + 8192 + kk * 32), C::kIdesc, 1u);
+              const uint64_t bd = desc_k_sw128(b_base + kk * 32);
+              mma_f8f6f4(tmem, desc_k_sw128(a0 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              if (two) mma_f8f6f4(tmem + kAccCols, desc_k_sw128(a1 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
             }
+            mma_commit(&empty[sa]);
           } else {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t half = kk >> 2, off = (kk & 3) * 32;
-              mma_f16(d, desc_k_sw128(a_base + half * 16384 + off), desc_k_sw128(b_base + half * 8192 + off),
-                      C::kIdesc, kk > 0 ? 1u : 0u);
+              const uint64_t bd = desc_k_sw128(b_base + half * 8192 + off);
+              mma_f16(tmem, desc_k_sw128(a0 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              if (two) mma_f16(tmem + kAccCols, desc_k_sw128(a1 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
             }
+            mma_commit(&empty[sa]);
+            if (two) mma_commit(&empty[sb]);
           }
-          mma_commit(&empty[s]);
-          mma_commit(&tfull[acc]);
+          mma_commit(tfull);
         }
         // every MMA of this CTA has completed before TMEM is read back or released
         mma_commit(mdone);
         mbar_wait(mdone, 0, kWaitLimit);
       }
-    } else if (!sh.fail) {
-      // epilogue: two groups of four warps take alternate tiles; warp w owns
-      // TMEM lanes 32 (w % 4) .. +31
-      const int grp = (warp - 2) >> 2;
-      const int sub = warp & 3;
-      const int row = sub * 32 + lane;
-      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-      const float qinv = sh.qinv;
-      uint32_t* hist = ghist0 + grp * kHistBins;
-      float w_r[kHeads];
+    } else {
+      // epilogue: the raw query is consumed, its space becomes the histograms
+      for (int i = tid - 64; i < 2 * kHistBins; i += kEpiWarps * 32) ghist0[i] = 0;
+      named_barrier(3, kEpiWarps * 32);
+      if (!sh.fail) {
+        // two groups of four warps take alternate tiles; warp w owns TMEM
+        // lanes 32 (w % 4) .. +31
+        const int grp = (warp - 2) >> 2;
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+        const float qinv = sh.qinv;
+        uint32_t* hist = ghist0 + grp * kHistBins;
+        float w_r[kHeads];
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) w_r[h] = ws[h];
-      for (int t = grp; t < nt; t += 2) {
-        const int acc = t % kNAcc;
-        const uint32_t aph = (t / kNAcc) & 1;
-        // the whole warp takes the same branch (warp-wide TMEM ops below)
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], aph, kWaitLimit))) {
-          atomicOr(&g_index_tc_error, 1u);
-          sh.fail = 1;
-          break;
-        }
-        tc_fence_after();
-        float ks = 1.f;
-        if constexpr (FP8) {
-          const int s = t % C::kStages;
-          mbar_wait(&full[s], (t / C::kStages) & 1, kWaitLimit);  // complete: makes the scales visible
-          ks = scale_ring[s * kTileM + row] * qinv;
-          mbar_arrive(&empty[s]);
-        }
-        uint32_t v0[32], v1[32];
-        tmem_ld32(lane_addr + acc * kHeads, v0);
-        tmem_ld32(lane_addr + acc * kHeads + 32, v1);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&tempty[acc]);
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int h = 0; h < kHeads; ++h) w_r[h] = ws[h];
+        for (int t = grp; t < nt; t += 2) {
+          const int acc = grp;
+          // the whole warp takes the same branch (warp-wide TMEM ops below)
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(tfull, (t >> 1) & 1, kWaitLimit))) {
+            atomicOr(&g_index_tc_error, 1u);
+            sh.fail = 1;
+            break;
+          }
+          tc_fence_after();
+          float ks = 1.f;
+          if constexpr (FP8) {
+            const int ss = t % kSStages;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[ss], (t / kSStages) & 1, kWaitLimit))) {
+              atomicOr(&g_index_tc_error, 1u);
+              sh.fail = 1;
+              break;
+            }
+            ks = scale_ring[ss * kTileM + row] * qinv;
+            mbar_arrive(&sempty[ss]);
+          }
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          const uint32_t acc_addr = lane_addr + acc * kAccCols;
 #pragma unroll
-        for (int h = 0; h < 32; h += 2) {
-          s0 = fmaf(w_r[h], fmaxf(__uint_as_float(v0[h]), 0.f), s0);
-          s1 = fmaf(w_r[h + 1], fmaxf(__uint_as_float(v0[h + 1]), 0.f), s1);
-          s2 = fmaf(w_r[32 + h], fmaxf(__uint_as_float(v1[h]), 0.f), s2);
-          s3 = fmaf(w_r[33 + h], fmaxf(__uint_as_float(v1[h + 1]), 0.f), s3);
+          for (int hh = 0; hh < kHeads; hh += 32) {
+            // heads hh..hh+31: FP8 adds the two query terms (columns h and 64 + h)
+            uint32_t v0[32], v1[32];
+            tmem_ld32(acc_addr + hh, v0);
+            if constexpr (FP8) tmem_ld32(acc_addr + kHeads + hh, v1);
+            tmem_wait_ld();
+            if (hh + 32 == kHeads) {
+              tc_fence_before();
+              mbar_arrive(tempty);
+            }
+#pragma unroll
+            for (int h = 0; h < 32; h += 2) {
+              float x0 = __uint_as_float(v0[h]), x1 = __uint_as_float(v0[h + 1]);
+              if constexpr (FP8) {
+                x0 += __uint_as_float(v1[h]);
+                x1 += __uint_as_float(v1[h + 1]);
+              }
+              if (hh == 0) {
+                s0 = fmaf(w_r[h], fmaxf(x0, 0.f), s0);
+                s1 = fmaf(w_r[h + 1], fmaxf(x1, 0.f), s1);
+              } else {
+                s2 = fmaf(w_r[hh + h], fmaxf(x0, 0.f), s2);
+                s3 = fmaf(w_r[hh + h + 1], fmaxf(x1, 0.f), s3);
+              }
+            }
+          }
+          const float sc = ((s0 + s1) + (s2 + s3)) * ks;
+          tmem_st1(lane_addr + kScoreCol + t, __float_as_uint(sc));
+          if (static_cast<int64_t>(t0 + t) * kTileM + row < n) atomicAdd(&hist[score_key(sc) >> 20], 1u);
         }
-        const float sc = ((s0 + s1) + (s2 + s3)) * ks;
-        tmem_st1(lane_addr + kScoreCol + t, __float_as_uint(sc));
-        if (static_cast<int64_t>(t0 + t) * kTileM + row < n) atomicAdd(&hist[score_key(sc) >> 20], 1u);
+        tmem_wait_st();
       }
-      tmem_wait_st();
     }
   }
   tc_fence_before();
@@ -496,280 +652,266 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   if (!sh.fail) {
     // ================= phase 2: exact top-k over the request =================
     const int k = a.k;
+    const int nch = a.chunks;
     int32_t* oi = a.out_idx + static_cast<int64_t>(r) * k;
     float* os = a.out_score ? a.out_score + static_cast<int64_t>(r) * k : nullptr;
-    uint8_t* p2 = smem + C::oStages;  // the stage ring is idle now
+    uint8_t* p2 = smem + C::oStages;  // the rings are idle now
     uint32_t* hist = reinterpret_cast<uint32_t*>(p2 + C::pHist);
     uint32_t* scratch = reinterpret_cast<uint32_t*>(p2 + C::pScratch);
-    uint32_t* cpre = reinterpret_cast<uint32_t*>(p2 + C::pCpre);
-    uint32_t* cntA = reinterpret_cast<uint32_t*>(p2 + C::pCntA);
-    uint32_t* cntE = reinterpret_cast<uint32_t*>(p2 + C::pCntE);
-    uint32_t* offA = reinterpret_cast<uint32_t*>(p2 + C::pOffA);
-    uint32_t* offE = reinterpret_cast<uint32_t*>(p2 + C::pOffE);
-    int32_t* eq_cache_i = reinterpret_cast<int32_t*>(p2 + C::pEq);
-    float* eq_cache_s = reinterpret_cast<float*>(eq_cache_i + kEqCache);
-    uint32_t* gh_g = ghist0;  // the two group histograms
-    // TMEM readers in phase 2: the four warps 2..5 (one per lane quarter)
-    const bool rd = warp >= 2 && warp < 6;
-    const int sub = warp & 3;
-    const uint32_t score_addr = tmem + (static_cast<uint32_t>(sub * 32) << 16) + kScoreCol;
-    auto local_of = [&](int t) { return t * kTileM + sub * 32 + lane; };
+    uint32_t* preA = reinterpret_cast<uint32_t*>(p2 + C::pCpre);  // [nch + 1] chunk prefixes
+    uint32_t* preE = preA + kMaxChunks + 4;
+    uint2* acache = reinterpret_cast<uint2*>(p2 + C::pACache);
+    float* sc = reinterpret_cast<float*>(p2 + C::pScores);
+    uint2* ecache = reinterpret_cast<uint2*>(p2 + C::pEq);
+    auto put = [&](uint32_t pos, uint2 e) {
+      if (pos < static_cast<uint32_t>(k)) {
+        oi[pos] = static_cast<int32_t>(e.x);
+        if (os) os[pos] = __uint_as_float(e.y);
+      }
+    };
+
+    // scores TMEM -> shared memory in index order: warps 2..9, two per lane quarter
+    if (warp >= 2) {
+      const int q = warp & 3, half = (warp - 2) >> 2;
+      const uint32_t qaddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kScoreCol;
+      for (int tb = half * 32; tb < nt; tb += 64) {
+        uint32_t v[32];
+        tmem_ld32(qaddr + tb, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          if (tb + u < nt) sc[(tb + u) * kTileM + q * 32 + lane] = __uint_as_float(v[u]);
+      }
+    }
+    __syncthreads();
+    // every thread owns a contiguous, 4-aligned segment of the chunk's entries
+    const int seg = ((nloc + kThreads - 1) / kThreads + 3) & ~3;
+    const int i0 = min(nloc, tid * seg), i1 = min(nloc, i0 + seg);
 
     if (n <= k) {
-      if (rd)
-        for (int tb = 0; tb < nt; tb += 32) {
-          uint32_t v[32];
-          tmem_ld32(score_addr + tb, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int t = tb + u, loc = local_of(t);
-            if (t < nt && loc < nloc) {
-              oi[base + loc] = static_cast<int32_t>(base + loc);
-              if (os) os[base + loc] = __uint_as_float(v[u]);
-            }
-          }
-        }
+      for (int i = tid; i < nloc; i += kThreads) {
+        oi[base + i] = static_cast<int32_t>(base + i);
+        if (os) os[base + i] = sc[i];
+      }
       if (c == 0)
         for (int64_t j = n + tid; j < k; j += kThreads) {
           oi[j] = -1;
           if (os) os[j] = -INFINITY;
         }
     } else {
+      uint32_t* gh_g = ghist0;  // the two group histograms
       uint32_t* gh1 = a.ghist + static_cast<int64_t>(r) * 2 * kHistBins;
       uint32_t* gh2 = gh1 + kHistBins;
       uint32_t* bar = a.sync + r * 4;
-      // pass 1 (bits 31..20): built while streaming
+      uint32_t nbar = 1;
+      // level 1 (bits 31..20): the histogram built while streaming
       for (int i = tid; i < kHistBins; i += kThreads) {
         const uint32_t v = gh_g[i] + gh_g[kHistBins + i];
         if (v) atomicAdd(&gh1[i], v);
       }
       bool alive = request_barrier(&bar[0], a.chunks, sh);
-      uint32_t shift = 20, prefix = 0, need = 0;
+      uint32_t shift = 20, prefix = 0;
       if (alive) {
-        for (int i = tid; i < kHistBins / 4; i += kThreads)
-          reinterpret_cast<uint4*>(hist)[i] = __ldcg(reinterpret_cast<const uint4*>(gh1) + i);
+        load_hist(hist, gh1);
         __syncthreads();
-        find_bin_block(hist, static_cast<uint32_t>(k), sh, scratch);
+        find_bin_block(hist, kHistBins, static_cast<uint32_t>(k), sh, scratch);
         prefix = sh.bcast[0];
-        need = static_cast<uint32_t>(k) - sh.bcast[1];
         if (hist[prefix] > static_cast<uint32_t>(kEqCache)) {
-          // a crowded boundary bin: one more distributed pass (bits 19..8)
-          for (int i = tid; i < 2 * kHistBins; i += kThreads) gh_g[i] = 0;
+          // a crowded boundary bin: one more distributed level (bits 19..8)
+          const uint32_t need = static_cast<uint32_t>(k) - sh.bcast[1];
+          for (int i = tid; i < kHistBins; i += kThreads) gh_g[i] = 0;
           __syncthreads();
-          if (rd)
-            for (int tb = 0; tb < nt; tb += 32) {
-              uint32_t v[32];
-              tmem_ld32(score_addr + tb, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                const uint32_t key = score_key(__uint_as_float(v[u]));
-                if (tb + u < nt && local_of(tb + u) < nloc && (key >> 20) == prefix)
-                  atomicAdd(&gh_g[(key >> 8) & 0xFFFu], 1u);
-              }
-            }
+          for (int i = i0; i < i1; ++i) {
+            const uint32_t key = score_key(sc[i]);
+            if ((key >> 20) == prefix) atomicAdd(&gh_g[(key >> 8) & 0xFFFu], 1u);
+          }
           __syncthreads();
           for (int i = tid; i < kHistBins; i += kThreads)
             if (gh_g[i]) atomicAdd(&gh2[i], gh_g[i]);
+          nbar = 2;
           alive = request_barrier(&bar[0], 2u * a.chunks, sh);
           if (alive) {
-            for (int i = tid; i < kHistBins / 4; i += kThreads)
-              reinterpret_cast<uint4*>(hist)[i] = __ldcg(reinterpret_cast<const uint4*>(gh2) + i);
+            load_hist(hist, gh2);
             __syncthreads();
-            find_bin_block(hist, need, sh, scratch);
+            find_bin_block(hist, kHistBins, need, sh, scratch);
             prefix = (prefix << 12) | sh.bcast[0];
-            need -= sh.bcast[1];
             shift = 8;
           }
         }
       }
+      const int64_t slot = static_cast<int64_t>(r) * nch + c;
+      uint2* st = a.st + slot * k;
+      uint2* eqg = a.eq + slot * (kMaxChunkTiles * kTileM);
+      uint32_t my_a = 0, my_e = 0;
       if (alive) {
-        // stage this chunk's keys above the boundary prefix and at it, in
-        // index order: per (tile, quarter) counts, prefix sums, then writes
-        const int64_t slot = static_cast<int64_t>(r) * a.chunks + c;
-        int32_t* sti = a.st_idx + slot * k;
-        float* sts = a.st_score + slot * k;
-        int32_t* eqi = a.eq_idx + slot * (kMaxChunkTiles * kTileM);
-        float* eqs = a.eq_score + slot * (kMaxChunkTiles * kTileM);
-        for (int pass = 0; pass < 2; ++pass) {
-          if (rd)
-            for (int tb = 0; tb < nt; tb += 32) {
-              uint32_t v[32];
-              tmem_ld32(score_addr + tb, v);
-              tmem_wait_ld();
+        // this chunk's entries above the boundary prefix (kept here) and at
+        // it (published), both lists in index order: counts per segment,
+        // block prefix sums, writes
+        uint32_t na = 0, ne = 0;
+        for (int i = i0; i < i1; i += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(sc + i);
+          const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                const int t = tb + u;
-                const int loc = local_of(t);
-                const bool valid = t < nt && loc < nloc;
-                const float sv = __uint_as_float(v[u]);
-                const uint32_t kp = score_key(sv) >> shift;
-                const bool above = valid && kp > prefix, eq = valid && kp == prefix;
-                const uint32_t ba = __ballot_sync(0xFFFFFFFFu, above), be = __ballot_sync(0xFFFFFFFFu, eq);
-                if (t < nt) {
-                  if (pass == 0) {
-                    if (lane == 0) {
-                      cntA[t * 4 + sub] = __popc(ba);
-                      cntE[t * 4 + sub] = __popc(be);
-                    }
-                  } else {
-                    const uint32_t lm = (1u << lane) - 1u;
-                    if (above) {
-                      const uint32_t pos = offA[t * 4 + sub] + __popc(ba & lm);
-                      if (pos < static_cast<uint32_t>(k)) {
-                        sti[pos] = static_cast<int32_t>(base + loc);
-                        sts[pos] = sv;
-                      }
-                    }
-                    if (eq) {
-                      const uint32_t pos = offE[t * 4 + sub] + __popc(be & lm);
-                      eqi[pos] = static_cast<int32_t>(base + loc);
-                      eqs[pos] = sv;
-                    }
-                  }
-                }
-              }
-            }
-          __syncthreads();
-          if (pass == 0) {
-            if (warp == 0) {
-              const uint32_t ta = warp_exclusive_scan(cntA, offA, nt * 4);
-              const uint32_t te = warp_exclusive_scan(cntE, offE, nt * 4);
-              if (lane == 0) {
-                sh.bcast[5] = ta;
-                sh.bcast[6] = te;
-              }
-            }
-            __syncthreads();
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t kp = score_key(fv[e]) >> shift;
+            const bool ok = i + e < i1;
+            na += ok && kp > prefix;
+            ne += ok && kp == prefix;
           }
         }
-        if (tid == 0) {
-          a.cnt[slot * 2] = sh.bcast[5];
-          a.cnt[slot * 2 + 1] = sh.bcast[6];
-          __threadfence();
-          const uint32_t prev = atomicAdd(&bar[1], 1u);
-          sh.bcast[2] = (prev == static_cast<uint32_t>(a.chunks) - 1) ? 1u : 0u;
+        uint32_t pa, pe;
+        block_scan2(na, ne, pa, pe, my_a, my_e, scratch);
+        for (int i = i0; i < i1; i += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(sc + i);
+          const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (i + e >= i1) break;
+            const uint32_t kp = score_key(fv[e]) >> shift;
+            const uint2 en = make_uint2(static_cast<uint32_t>(base + i + e), __float_as_uint(fv[e]));
+            if (kp > prefix) {
+              if (pa < static_cast<uint32_t>(kACache)) acache[pa] = en;
+              else if (pa < static_cast<uint32_t>(k)) st[pa] = en;
+              ++pa;
+            } else if (kp == prefix) {
+              eqg[pe++] = en;
+            }
+          }
+        }
+        if (tid == 0) reinterpret_cast<uint2*>(a.cnt)[slot] = make_uint2(my_a, my_e);
+        ++nbar;
+        alive = request_barrier(&bar[0], nbar * a.chunks, sh);
+      }
+      if (alive) {
+        // ---- every CTA: chunk offsets, then its own share of the output ----
+        const uint2* cnt = reinterpret_cast<const uint2*>(a.cnt) + static_cast<int64_t>(r) * nch;
+        for (int i = tid; i < nch; i += kThreads) {
+          const uint2 ce = __ldcg(cnt + i);
+          preA[i] = ce.x;
+          preE[i] = ce.y;
         }
         __syncthreads();
-        if (sh.bcast[2]) {
-          // ---------- last CTA of the request: assemble in chunk (= index) order ----------
-          __threadfence();
-          const uint32_t* cnt = a.cnt + static_cast<int64_t>(r) * a.chunks * 2;
-          const int nch = a.chunks;
-          for (int cc = tid; cc < nch; cc += kThreads) {
-            cpre[cc] = __ldcg(cnt + cc * 2);
-            cpre[160 + cc] = __ldcg(cnt + cc * 2 + 1);
+        if (warp == 0) {
+          const uint32_t ta = warp_scan_inplace(preA, nch);
+          if (lane == 0) preA[nch] = ta;
+        } else if (warp == 1) {
+          const uint32_t te = warp_scan_inplace(preE, nch);
+          if (lane == 0) preE[nch] = te;
+        }
+        __syncthreads();
+        const uint32_t A_tot = preA[nch], E_tot = preE[nch];
+        // entries above the boundary: straight to their place
+        for (uint32_t i = tid; i < my_a; i += kThreads)
+          put(preA[c] + i, i < static_cast<uint32_t>(kACache) ? acache[i] : __ldcg(st + i));
+        const uint32_t take = A_tot < static_cast<uint32_t>(k) ? static_cast<uint32_t>(k) - A_tot : 0u;
+        // chunk of boundary entry i (i < E_tot): fixed-step binary search
+        auto eq_src = [&](uint32_t i) {
+          int lo = 0;
+#pragma unroll
+          for (int step = 128; step > 0; step >>= 1) {
+            const int m = lo + step;
+            if (m < nch && preE[m] <= i) lo = m;
+          }
+          return a.eq + (static_cast<int64_t>(r) * nch + lo) * (kMaxChunkTiles * kTileM) + (i - preE[lo]);
+        };
+        if (E_tot <= take) {
+          // every boundary entry is taken
+          for (uint32_t i = tid; i < my_e; i += kThreads) put(A_tot + preE[c] + i, __ldcg(eqg + i));
+        } else if (E_tot <= static_cast<uint32_t>(kEqCache)) {
+          // the request's boundary entries, in index order, into shared memory
+          constexpr int LB = 8;
+          for (uint32_t j0 = 0; j0 < E_tot; j0 += kThreads * LB) {
+            uint2 e[LB];
+#pragma unroll
+            for (int b = 0; b < LB; ++b) {
+              const uint32_t i = j0 + b * kThreads + tid;
+              if (i < E_tot) e[b] = __ldcg(eq_src(i));
+            }
+#pragma unroll
+            for (int b = 0; b < LB; ++b) {
+              const uint32_t i = j0 + b * kThreads + tid;
+              if (i < E_tot) ecache[i] = e[b];
+            }
           }
           __syncthreads();
-          if (tid == 0) {
-            uint32_t sa = 0, se = 0;
-            for (int cc = 0; cc < nch; ++cc) {
-              const uint32_t x = cpre[cc], y = cpre[160 + cc];
-              cpre[cc] = sa;
-              cpre[160 + cc] = se;
-              sa += x;
-              se += y;
-            }
-            cpre[nch] = sa;
-            cpre[160 + nch] = se;
-          }
-          __syncthreads();
-          const uint32_t A = min(cpre[nch], static_cast<uint32_t>(k));
-          const uint32_t E = cpre[160 + nch];
-          const int64_t eq_stride = kMaxChunkTiles * kTileM;
-          auto chunk_of = [&](const uint32_t* pre, uint32_t i) {
-            int lo = 0, hi = nch - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (pre[mid] <= i) lo = mid; else hi = mid - 1;
-            }
-            return lo;
-          };
-          for (uint32_t i = tid; i < A; i += kThreads) {
-            const int cc = chunk_of(cpre, i);
-            const int64_t src = (static_cast<int64_t>(r) * nch + cc) * k + (i - cpre[cc]);
-            oi[i] = __ldcg(a.st_idx + src);
-            if (os) os[i] = __ldcg(a.st_score + src);
-          }
-          const uint32_t take = min(need, static_cast<uint32_t>(k) - A);
-          if (E <= take) {
-            for (uint32_t i = tid; i < E; i += kThreads) {
-              const int cc = chunk_of(cpre + 160, i);
-              const int64_t src = (static_cast<int64_t>(r) * nch + cc) * eq_stride + (i - cpre[160 + cc]);
-              oi[A + i] = __ldcg(a.eq_idx + src);
-              if (os) os[A + i] = __ldcg(a.eq_score + src);
-            }
-          } else {
-            // more boundary entries than places left: radix passes over the
-            // low `shift` bits of their keys, then the lowest indices
-            // (entries are in index order)
-            const uint32_t ncache = min(E, static_cast<uint32_t>(kEqCache));
-            for (uint32_t i = tid; i < ncache; i += kThreads) {
-              const int cc = chunk_of(cpre + 160, i);
-              const int64_t src = (static_cast<int64_t>(r) * nch + cc) * eq_stride + (i - cpre[160 + cc]);
-              eq_cache_i[i] = __ldcg(a.eq_idx + src);
-              eq_cache_s[i] = __ldcg(a.eq_score + src);
+          // radix levels over the low `shift` key bits (10 + 10, or 8): the
+          // take-th largest key T and how many entries equal to T are taken
+          uint32_t pfx = prefix, rb = shift, tk = take;
+          while (rb > 0) {
+            const uint32_t nb = rb > 10 ? 10 : rb;
+            const uint32_t sft = rb - nb;
+            for (int i = tid; i < (1 << nb); i += kThreads) hist[i] = 0;
+            __syncthreads();
+            for (uint32_t i = tid; i < E_tot; i += kThreads) {
+              const uint32_t key = score_key(__uint_as_float(ecache[i].y));
+              if ((key >> rb) == pfx) atomicAdd(&hist[(key >> sft) & ((1u << nb) - 1u)], 1u);
             }
             __syncthreads();
-            auto eq_at = [&](uint32_t i, int32_t& j, float& v) {
-              if (i < ncache) {
-                j = eq_cache_i[i];
-                v = eq_cache_s[i];
-              } else {
-                const int cc = chunk_of(cpre + 160, i);
-                const int64_t src = (static_cast<int64_t>(r) * nch + cc) * eq_stride + (i - cpre[160 + cc]);
-                j = __ldcg(a.eq_idx + src);
-                v = __ldcg(a.eq_score + src);
-              }
-            };
-            uint32_t pfx = prefix, rb = shift, tk = take;
-            while (rb > 0) {
-              const uint32_t nb = rb > 12 ? 12 : rb;
-              const uint32_t sft = rb - nb;
-              for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
-              __syncthreads();
-              for (uint32_t i = tid; i < E; i += kThreads) {
-                int32_t j;
-                float v;
-                eq_at(i, j, v);
-                const uint32_t key = score_key(v);
-                if ((key >> rb) == pfx) atomicAdd(&hist[(key >> sft) & ((1u << nb) - 1u)], 1u);
-              }
-              __syncthreads();
-              find_bin_block(hist, tk, sh, scratch);
-              pfx = (pfx << nb) | sh.bcast[0];
-              tk -= sh.bcast[1];
-              rb = sft;
+            find_bin_block(hist, 1 << nb, tk, sh, scratch);
+            pfx = (pfx << nb) | sh.bcast[0];
+            tk -= sh.bcast[1];
+            rb = sft;
+          }
+          const uint32_t T = pfx;
+          // taken: key > T, and the first tk (lowest indices) with key == T
+          const uint32_t e0 = preE[c], e1 = preE[c + 1];
+          uint32_t g = 0, q = 0;
+          for (uint32_t i = tid; i < e0; i += kThreads) {
+            const uint32_t key = score_key(__uint_as_float(ecache[i].y));
+            g += key > T;
+            q += key == T;
+          }
+          block_sum2(g, q, scratch);
+          uint32_t out = A_tot + g + min(q, tk), eq_seen = q;
+          for (uint32_t j0 = e0; j0 < e1; j0 += kThreads) {
+            const uint32_t i = j0 + tid;
+            const uint2 e = i < e1 ? ecache[i] : make_uint2(0u, 0u);
+            const uint32_t key = score_key(__uint_as_float(e.y));
+            const bool gt = i < e1 && key > T, eq = i < e1 && key == T;
+            uint32_t re, rz, te, tz;
+            block_rank2(eq, false, re, rz, te, tz, scratch);
+            const bool sel = gt || (eq && eq_seen + re < tk);
+            uint32_t rs, ts;
+            block_rank2(sel, false, rs, rz, ts, tz, scratch);
+            if (sel) put(out + rs, e);
+            out += ts;
+            eq_seen += te;
+          }
+        } else if (c == 0) {
+          // very many boundary entries (massive ties): one CTA streams them
+          // from global memory through the same radix levels and writes the
+          // whole boundary part of the output
+          uint32_t pfx = prefix, rb = shift, tk = take;
+          while (rb > 0) {
+            const uint32_t nb = rb > 10 ? 10 : rb;
+            const uint32_t sft = rb - nb;
+            for (int i = tid; i < (1 << nb); i += kThreads) hist[i] = 0;
+            __syncthreads();
+            for (uint32_t i = tid; i < E_tot; i += kThreads) {
+              const uint32_t key = score_key(__uint_as_float(__ldcg(eq_src(i)).y));
+              if ((key >> rb) == pfx) atomicAdd(&hist[(key >> sft) & ((1u << nb) - 1u)], 1u);
             }
-            // every boundary entry with key > T, then the first tk equal to T
-            const uint32_t T = pfx, take_eq = tk;
-            uint32_t out = A, got_eq = 0;
-            for (uint32_t i0 = 0; i0 < E; i0 += kThreads) {
-              const uint32_t i = i0 + tid;
-              int32_t j = 0;
-              float v = 0.f;
-              uint32_t key = 0;
-              if (i < E) {
-                eq_at(i, j, v);
-                key = score_key(v);
-              }
-              const bool gt = i < E && key > T, eq = i < E && key == T;
-              uint32_t rg, re, tg, te;
-              block_rank2(gt, eq, rg, re, tg, te, scratch);
-              if (gt && out + rg < static_cast<uint32_t>(k)) {
-                oi[out + rg] = j;
-                if (os) os[out + rg] = v;
-              }
-              out += tg;
-              if (eq && got_eq + re < take_eq && out + re < static_cast<uint32_t>(k)) {
-                oi[out + re] = j;
-                if (os) os[out + re] = v;
-              }
-              const uint32_t add = min(te, take_eq - got_eq);
-              got_eq += add;
-              out += add;
-            }
+            __syncthreads();
+            find_bin_block(hist, 1 << nb, tk, sh, scratch);
+            pfx = (pfx << nb) | sh.bcast[0];
+            tk -= sh.bcast[1];
+            rb = sft;
+          }
+          const uint32_t T = pfx;
+          uint32_t out = A_tot, eq_seen = 0;
+          for (uint32_t j0 = 0; j0 < E_tot; j0 += kThreads) {
+            const uint32_t i = j0 + tid;
+            const uint2 e = i < E_tot ? __ldcg(eq_src(i)) : make_uint2(0u, 0u);
+            const uint32_t key = score_key(__uint_as_float(e.y));
+            const bool gt = i < E_tot && key > T, eq = i < E_tot && key == T;
+            uint32_t re, rz, te, tz;
+            block_rank2(eq, false, re, rz, te, tz, scratch);
+            const bool sel = gt || (eq && eq_seen + re < tk);
+            uint32_t rs, ts;
+            block_rank2(sel, false, rs, rz, ts, tz, scratch);
+            if (sel) put(out + rs, e);
+            out += ts;
+            eq_seen += te;
           }
         }
       }
@@ -822,7 +964,7 @@ bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dty
   if (static_cast<int64_t>(batch) * cap >= (int64_t(1) << 31)) return false;
   const int ch = index_tc_chunks(batch, cap);
   const int64_t tiles = (cap + kTileM - 1) / kTileM;
-  return (tiles + ch - 1) / ch <= kMaxChunkTiles && p->topk >= 1;
+  return ch <= kMaxChunks && (tiles + ch - 1) / ch <= kMaxChunkTiles && p->topk >= 1;
 }
 
 size_t index_tc_control_bytes(int batch) { return static_cast<size_t>(batch) * (2 * kHistBins + 4) * 4; }
@@ -848,7 +990,8 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(batch) * cap};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDI) * (fp8 ? 1 : 2)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(kTileM)};
+  // FP8: one 256-row box = two key tiles per stage; bf16: two 64-column boxes per tile
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(fp8 ? 2 * kTileM : kTileM)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult cr = L.encode(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                          k_idx->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -891,10 +1034,8 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.sync = reinterpret_cast<uint32_t*>(base + static_cast<size_t>(batch) * 2 * kHistBins * 4);
   off = (index_tc_control_bytes(batch) + 255) & ~static_cast<size_t>(255);
   a.cnt = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(batch) * ch * 2 * 4));
-  a.st_idx = reinterpret_cast<int32_t*>(take(static_cast<size_t>(batch) * ch * p->topk * 4));
-  a.st_score = reinterpret_cast<float*>(take(static_cast<size_t>(batch) * ch * p->topk * 4));
-  a.eq_idx = reinterpret_cast<int32_t*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 4));
-  a.eq_score = reinterpret_cast<float*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 4));
+  a.st = reinterpret_cast<uint2*>(take(static_cast<size_t>(batch) * ch * p->topk * 8));
+  a.eq = reinterpret_cast<uint2*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 8));
 
   const int smem = fp8 ? Cfg<true>::kSmem : Cfg<false>::kSmem;
   void* fn = fp8 ? reinterpret_cast<void*>(index_topk_tc_kernel<true>) : reinterpret_cast<void*>(index_topk_tc_kernel<false>);

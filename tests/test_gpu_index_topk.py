@@ -146,3 +146,42 @@ def test_index_topk_tensor_core_is_deterministic(cuda_lib):
     a, sa = gpu_index_topk(wl, q_idx, w, kidx, B, cap, None, n_vis)
     b, sb = gpu_index_topk(wl, q_idx, w, kidx, B, cap, None, n_vis)
     assert np.array_equal(a, b) and np.array_equal(sa, sb)
+
+
+@pytest.mark.parametrize("dt", ["fp8", "bf16"])
+def test_index_topk_tensor_core_zero_ties_resolved_in_shared_memory(dt, cuda_lib):
+    """A few hundred keys score above zero, every other key scores exactly 0
+    and the zeros fit the shared-memory boundary list: the selection is every
+    positive key plus the lowest-index zeros, bit-exact."""
+    wl = Wk.WORKLOADS["decode1m" if dt == "fp8" else "decode64k"]
+    cap, k, n_pos = 8000, 512, 300
+    rng = np.random.default_rng(11)
+    pos_rows = np.sort(rng.choice(cap, n_pos, replace=False))
+    keys = np.abs(Wk.normal(11, "k", (1, cap, wl.d_idx))) / 10
+    keys[0, pos_rows] *= -1.0  # q < 0 everywhere: these rows have positive dots
+    q = -np.abs(Wk.normal(11, "q", (1, wl.h_idx, wl.d_idx))) / 10
+    gi, gs = gpu_index_topk(wl, Wk.store(q, "bf16"), Wk.uniform(11, "w", (1, wl.h_idx)),
+                            Wk.store(keys, dt, wl.d_idx), 1, cap, None, np.array([cap], np.int32), k=k)
+    zeros = np.setdiff1d(np.arange(cap), pos_rows)[: k - n_pos]
+    assert np.array_equal(np.sort(gi[0]), np.sort(np.concatenate([pos_rows, zeros])))
+    sel_zero = np.isin(gi[0], zeros)
+    assert np.all(gs[0][sel_zero] == 0) and np.all(gs[0][~sel_zero] > 0)
+
+
+def test_index_topk_tensor_core_crowded_bin_takes_second_level(cuda_lib):
+    """All scores within a few per cent of each other: the top 12 key bits
+    put more than the shared-memory list holds into the boundary bin, so the
+    kernel narrows the boundary with a second distributed histogram level."""
+    wl = Wk.WORKLOADS["decode64k"]
+    cap = 30000
+    sI = 1 / np.sqrt(wl.d_idx)
+    base = Wk.normal(12, "base", (1, 1, wl.d_idx), sI)
+    keys = base + 0.03 * Wk.normal(12, "noise", (1, cap, wl.d_idx), sI)
+    kidx = Wk.store(keys, "bf16")
+    q_idx = Wk.store(Wk.normal(12, "q", (1, wl.h_idx, wl.d_idx), sI), "bf16")
+    w = Wk.uniform(12, "w", (1, wl.h_idx))
+    gi, gs = gpu_index_topk(wl, q_idx, w, kidx, 1, cap, None, np.array([cap], np.int32))
+    s = O.index_scores(O.decode_stored(q_idx)[0], w[0], O.decode(kidx.data[0], "bf16", None, 0))
+    top = np.sort(s)[::-1]
+    assert top[0] / top[-1] < 1.1, "the scores are meant to crowd one 12-bit key bin"
+    check_selection(gi[0], s, wl.topk, False, gs[0])
