@@ -214,6 +214,10 @@ def run_ours(args, rank, world, local_rank):
     def flush_l2():
         flush.zero_()         # evicts the inputs ...
         evict.sum()           # ... and replaces the flush's dirty lines with clean ones
+        # the GPU idles ~100 us after the flush, so that the host has queued the
+        # step's launches before the step's first event is timestamped: the
+        # events then time the kernels, not the host's launch calls
+        torch.cuda._sleep(200_000)
     stream = torch.cuda.current_stream()
     n_vis = int((inp.pos[0] + 1) // wl.m)
     del inp

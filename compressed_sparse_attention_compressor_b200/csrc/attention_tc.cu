@@ -26,6 +26,8 @@
 
 #include <cstring>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -45,8 +47,9 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 // shared-memory layout
 constexpr int oK = 0;                        // 8 x 16 KB key tile
 constexpr int oQ = oK + 8 * kTK * 128;       // 8 x 8 KB query (later: logits, P^T, stats)
-constexpr int oS = oQ;                       // fp32 [64][128] logits (after S is done)
-constexpr int oP = oQ + kH * kTK * 4;        // 2 x 8 KB P^T
+constexpr int oS = oQ;                       // fp32 logits [64 heads][4 blocks of 33] (after S is done)
+constexpr int kSbStride = 4 * 33;            // padded head row: conflict-free writes and reads
+constexpr int oP = oQ + (kH * kSbStride * 4 + 1023) / 1024 * 1024;  // 2 x 8 KB P^T
 constexpr int oML = oP + 2 * kH * 128;       // per-head (max, sum)
 constexpr int oEnt = oQ + 8 * kH * 128;      // [128] entry codes
 constexpr int oBars = oEnt + kTK * 4;
@@ -67,6 +70,8 @@ struct AttnTcArgs {
   float tau;
   float* part;     // [nq][splits][64][512 + 2]: (m, l, O)
   int splits;
+  // cluster path: the merged output
+  const float* sink; void* out; int out_dtype; float* lse;
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -164,6 +169,92 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const AttnTcArgs&
   }
 }
 
+// CLUSTER = false: one CTA per 128-key split of a query's key list, the
+// split's (max, sum, O) to the global workspace, merged by another kernel.
+// CLUSTER = true: the gridDim.x CTAs of one cluster serve one query; CTA r
+// takes the r-th even slice of the selected entries and of the window, keeps
+// its (max, sum, O) in its own shared memory, and the cluster merges them
+// through distributed shared memory (CTA r finishes heads r, r + R, ...).
+// Cluster path, all threads: the tile's rows [0, nsr) from their compressed
+// entries (FP8 dequantised to bf16) and rows [nsr, nsr + nwr) from the
+// window keys, every load of a batch of 16 per thread issued before any is
+// used; the window rows' values go to vw[] (registers) in the same batch
+// (nwr <= 16), to replace the keys once the logits are out.  Rows
+// [nsr + nwr, nk16) are zeroed (the PV product reads them with weight 0).
+__device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const AttnTcArgs& a, int64_t kv_row0,
+                               int64_t sw_row0, int nsr, int nwr, int nk16, uint4 (&vw)[4]) {
+  const int per_sel = a.kv_fp8 ? 32 : 64;  // 16-byte chunks per selected row
+  const int T1 = nsr * per_sel, T = T1 + nwr * 64;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int task = threadIdx.x + b * kThreads;
+    vw[b] = make_uint4(0, 0, 0, 0);
+    if (task < nwr * 64) {
+      const int e = ent[nsr + (task >> 6)];
+      if (e <= -2) vw[b] = __ldg(reinterpret_cast<const uint4*>(a.swa_v + (sw_row0 + (-2 - e)) * kD) + (task & 63));
+    }
+  }
+  constexpr int B = 16;
+  for (int t0 = threadIdx.x; t0 < T; t0 += kThreads * B) {
+    uint4 u[B];
+    float sc[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int task = t0 + b * kThreads;
+      u[b] = make_uint4(0, 0, 0, 0);
+      sc[b] = 0.f;
+      if (task < T1) {
+        const int r = task / per_sel, c = task % per_sel;
+        const int32_t e = ent[r];
+        if (e >= 0) {
+          const int64_t gr = kv_row0 + e;
+          if (a.kv_fp8) {
+            u[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * kD) + c);
+            sc[b] = __ldg(a.kv_scale + gr * (kD / 64) + (c >> 2));
+          } else {
+            u[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + gr * kD) + c);
+          }
+        }
+      } else if (task < T) {
+        const int w = task - T1;
+        const int32_t e = ent[nsr + (w >> 6)];
+        if (e <= -2) u[b] = __ldg(reinterpret_cast<const uint4*>(a.swa_k + (sw_row0 + (-2 - e)) * kD) + (w & 63));
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int task = t0 + b * kThreads;
+      if (task < T1) {
+        const int r = task / per_sel, c = task % per_sel;
+        if (a.kv_fp8) {
+          const uint32_t w[4] = {u[b].x, u[b].y, u[b].z, u[b].w};
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFF));
+            const float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
+            const __nv_bfloat162 bl = __floats2bfloat162_rn(lo.x * sc[b], lo.y * sc[b]);
+            const __nv_bfloat162 bh = __floats2bfloat162_rn(hi.x * sc[b], hi.y * sc[b]);
+            o[2 * i] = *reinterpret_cast<const uint32_t*>(&bl);
+            o[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&bh);
+          }
+          put_chunk(tile, r, c * 16, make_uint4(o[0], o[1], o[2], o[3]));
+          put_chunk(tile, r, c * 16 + 8, make_uint4(o[4], o[5], o[6], o[7]));
+        } else {
+          put_chunk(tile, r, c * 8, u[b]);
+        }
+      } else if (task < T) {
+        const int w = task - T1;
+        put_chunk(tile, nsr + (w >> 6), (w & 63) * 8, u[b]);
+      }
+    }
+  }
+  // zero rows between the last valid key and the next multiple of 16
+  for (int task = (nsr + nwr) * 64 + threadIdx.x; task < nk16 * 64; task += kThreads)
+    put_chunk(tile, task >> 6, (task & 63) * 8, make_uint4(0, 0, 0, 0));
+}
+
+template <bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -192,11 +283,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   const int n_win = (a.window > 0 && t >= p_lo) ? static_cast<int>(t - p_lo + 1) : 0;
   const int total = live ? n_sel + n_win : 0;
   const int x0 = split * kTK;
+  // cluster slices: selected [s0, s1), window [w0, w1) (window offsets)
+  const int R = static_cast<int>(gridDim.x);
+  const int s0 = live ? static_cast<int>(static_cast<int64_t>(split) * n_sel / R) : 0;
+  const int s1 = live ? static_cast<int>(static_cast<int64_t>(split + 1) * n_sel / R) : 0;
+  const int w0 = live ? static_cast<int>(static_cast<int64_t>(split) * n_win / R) : 0;
+  const int w1 = live ? static_cast<int>(static_cast<int64_t>(split + 1) * n_win / R) : 0;
   const int64_t kv_row0 = live ? static_cast<int64_t>(r) * a.cap : 0;
   const int64_t sw_row0 = live ? static_cast<int64_t>(r) * a.swa_cap : 0;
   float* pp = a.part + (static_cast<int64_t>(qi) * a.splits + split) * kH * (kD + 2);
 
-  if (x0 >= total) {  // an empty split: m = -inf
+  if (!CLUSTER && x0 >= total) {  // an empty split: m = -inf
     for (int h = tid; h < kH; h += kThreads) {
       pp[h * (kD + 2)] = -INFINITY;
       pp[h * (kD + 2) + 1] = 0.f;
@@ -213,15 +310,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     fence_barrier_init();
   }
   if (tid < kTK) {
-    const int x = x0 + tid;
     int32_t e = -1;
-    if (x < total) {
-      if (x < n_sel) {
-        const int32_t j = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
-        e = (j >= 0 && j < nv) ? j : -1;
-      } else {
-        e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
+    int xs = -1, xw = -1;  // selected-list position / window offset of this row
+    if (CLUSTER) {
+      if (tid < s1 - s0) xs = s0 + tid;
+      else if (tid < (s1 - s0) + (w1 - w0)) xw = w0 + tid - (s1 - s0);
+    } else {
+      const int x = x0 + tid;
+      if (x < total) {
+        if (x < n_sel) xs = x;
+        else xw = x - n_sel;
       }
+    }
+    if (xs >= 0) {
+      const int32_t j = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + xs] : xs;
+      e = (j >= 0 && j < nv) ? j : -1;
+    } else if (xw >= 0) {
+      e = -2 - static_cast<int32_t>((p_lo + xw) % a.swa_cap);
     }
     ent[tid] = e;
   }
@@ -232,7 +337,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + oQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
   }
   if (tid < kTK && ent[tid] <= -2) s_flags[0] = 1;
-  gather_rows(Kt, ent, a, kv_row0, sw_row0, 0);
+  const int nsr = s1 - s0, nwr = w1 - w0;
+  const int nk16 = CLUSTER ? ((nsr + nwr + 15) & ~15) : kTK;  // keys the PV product covers
+  const bool vregs = CLUSTER && nwr <= 16;                     // window values held in registers
+  uint4 vw[4];
+  if (vregs) gather_cluster(Kt, ent, a, kv_row0, sw_row0, nsr, nwr, nk16, vw);
+  else gather_rows(Kt, ent, a, kv_row0, sw_row0, 0);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -256,11 +366,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
                 kIdescS, (blk | kk) ? 1u : 0u);
     mma_commit(sbar);
   }
-  // logits -> shared memory, transposed to [head][key]
-  if (!__all_sync(0xFFFFFFFFu, mbar_wait(sbar, 0, kWaitLimit))) {
+  // logits -> shared memory, transposed to [head][key]; one thread polls
+  // the MMA's barrier and the CTA barrier releases the others
+  if (tid == 0 && !mbar_wait(sbar, 0, kWaitLimit)) {
     atomicOr(&g_attn_tc_error, 1u);
     s_flags[1] = 1;
   }
+  __syncthreads();
   tc_fence_after();
   if (warp >= 4) {
     const int sub = warp & 3, row = sub * 32 + lane;
@@ -272,17 +384,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     const bool ok = ent[row] != -1;
 #pragma unroll
     for (int h = 0; h < 32; ++h) {
-      Sb[h * kTK + row] = ok ? __uint_as_float(v0[h]) * a.tau : -INFINITY;
-      Sb[(32 + h) * kTK + row] = ok ? __uint_as_float(v1[h]) * a.tau : -INFINITY;
+      Sb[h * kSbStride + sub * 33 + lane] = ok ? __uint_as_float(v0[h]) * a.tau : -INFINITY;
+      Sb[(32 + h) * kSbStride + sub * 33 + lane] = ok ? __uint_as_float(v1[h]) * a.tau : -INFINITY;
     }
   }
   __syncthreads();
   // window rows: values replace keys in the tile (the S MMA has read it)
-  if (s_flags[0]) gather_rows(Kt, ent, a, kv_row0, sw_row0, 1);
+  if (vregs) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int task = tid + b * kThreads;
+      if (task < nwr * 64) put_chunk(Kt, nsr + (task >> 6), (task & 63) * 8, vw[b]);
+    }
+  } else if (s_flags[0]) {
+    gather_rows(Kt, ent, a, kv_row0, sw_row0, 1);
+  }
   // softmax statistics and P^T: four threads per head, 32 keys each
   {
     const int h = tid >> 2, q4 = tid & 3;
-    const float* srow = Sb + h * kTK + q4 * 32;
+    const float* srow = Sb + h * kSbStride + q4 * 33;
     float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < 32; ++i) m = fmaxf(m, srow[i]);
@@ -322,36 +442,114 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int kk = 0; kk < kTK / 16; ++kk)
+      for (int kk = 0; kk < nk16 / 16; ++kk)
         mma_f16(dO + mt * kH, desc_mn_sw128(kb + (2 * mt) * kTK * 128 + kk * 16 * 128, kTK * 128),
                 desc_k_sw128(pb + (kk >> 2) * kH * 128 + (kk & 3) * 32), kIdescO, kk > 0 ? 1u : 0u);
     mma_commit(obar);
   }
-  if (tid < kH) {
+  if (!CLUSTER && tid < kH) {
     pp[tid * (kD + 2)] = ml[2 * tid];
     pp[tid * (kD + 2) + 1] = ml[2 * tid + 1];
   }
-  if (!__all_sync(0xFFFFFFFFu, mbar_wait(obar, 0, kWaitLimit))) {
+  if (tid == 0 && !mbar_wait(obar, 0, kWaitLimit)) {
     atomicOr(&g_attn_tc_error, 1u);
     s_flags[1] = 1;
   }
+  __syncthreads();
   tc_fence_after();
-  if (warp >= 4) {
-    const int sub = warp & 3;
+  if constexpr (!CLUSTER) {
+    if (warp >= 4) {
+      const int sub = warp & 3;
 #pragma unroll 1
-    for (int mt = 0; mt < 4; ++mt) {
-      const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
-      uint32_t v0[32], v1[32];
-      tmem_ld32(ta, v0);
-      tmem_ld32(ta + 32, v1);
-      tmem_wait_ld();
-      const int dim = mt * 128 + sub * 32 + lane;
+      for (int mt = 0; mt < 4; ++mt) {
+        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
+        uint32_t v0[32], v1[32];
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_wait_ld();
+        const int dim = mt * 128 + sub * 32 + lane;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) {
-        pp[h * (kD + 2) + 2 + dim] = __uint_as_float(v0[h]);
-        pp[(32 + h) * (kD + 2) + 2 + dim] = __uint_as_float(v1[h]);
+        for (int h = 0; h < 32; ++h) {
+          pp[h * (kD + 2) + 2 + dim] = __uint_as_float(v0[h]);
+          pp[(32 + h) * (kD + 2) + 2 + dim] = __uint_as_float(v1[h]);
+        }
       }
     }
+  } else {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    // this CTA's O (unnormalised) into its own shared memory as [head][dim]
+    // fp32, over the key tile (both MMAs have completed)
+    float* Osm = reinterpret_cast<float*>(smem + oK);
+    {
+      const int sub = warp & 3, mh = warp >> 2;  // two warps per TMEM lane quarter
+#pragma unroll 1
+      for (int mt = mh * 2; mt < mh * 2 + 2; ++mt) {
+        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
+        uint32_t v0[32], v1[32];
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_wait_ld();
+        const int dim = mt * 128 + sub * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          Osm[h * kD + dim] = __uint_as_float(v0[h]);
+          Osm[(32 + h) * kD + dim] = __uint_as_float(v1[h]);
+        }
+      }
+    }
+    cluster.sync();
+    // heads split + r * R for r = 0, 1, ...: warp w weighs head split + w R
+    float* wgt = reinterpret_cast<float*>(smem + oS);  // [head][16 CTAs], then [head][2] (M, 1/L); logits are dead
+    const int nh = (kH - split + R - 1) / R;
+    for (int w = warp; w < nh; w += kThreads / 32) {
+      const int h = split + w * R;
+      float mj = -INFINITY, lj = 0.f;
+      if (lane < R) {
+        const float* pml = cluster.map_shared_rank(ml, lane);
+        mj = pml[2 * h];
+        lj = pml[2 * h + 1];
+      }
+      const float sk = a.sink ? a.sink[h] : -INFINITY;
+      const float M = fmaxf(warp_max(mj), sk);
+      const float wj = (mj == -INFINITY) ? 0.f : __expf(mj - M);
+      float L = warp_sum(wj * lj);
+      if (sk != -INFINITY) L += __expf(sk - M);
+      if (lane < R) wgt[w * 16 + lane] = wj;
+      if (lane == 0) {
+        wgt[kH * 16 + w * 2] = M;
+        wgt[kH * 16 + w * 2 + 1] = (M == -INFINITY) ? 0.f : 1.f / L;
+        if (a.lse) a.lse[static_cast<int64_t>(qi) * kH + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
+      }
+    }
+    __syncthreads();
+    // two consecutive dims per thread, R peers each
+    for (int w = 0; w < nh; ++w) {
+      const int h = split + w * R;
+      const int dim = tid * 2;
+      float2 v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)  // every peer's load in flight before the sums
+        if (j < R) v[j] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(Osm, j) + h * kD + dim);
+      float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < R) {
+          const float wj = wgt[w * 16 + j];
+          o0 = fmaf(wj, v[j].x, o0);
+          o1 = fmaf(wj, v[j].y, o1);
+        }
+      const float inv = wgt[kH * 16 + w * 2 + 1];
+      o0 *= inv;
+      o1 *= inv;
+      const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
+      if (a.out_dtype == kF32) {
+        *reinterpret_cast<float2*>(static_cast<float*>(a.out) + off) = make_float2(o0, o1);
+      } else {
+        *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0, o1);
+      }
+    }
+    cluster.sync();  // every peer has read this CTA's partial
   }
   tc_fence_before();
   __syncthreads();
@@ -361,7 +559,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
 
 struct TcLauncher {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  bool attr = false;
+  bool attr[2] = {false, false};
+  int cluster_ok[17] = {0};  // per cluster size: 0 unknown, else co-resident clusters (-1: none)
 };
 
 TcLauncher& tc_launcher() {
@@ -379,6 +578,14 @@ TcLauncher& tc_launcher() {
 }  // namespace
 
 int attn_tc_splits(int max_keys) { return (max_keys + kTK - 1) / kTK; }
+
+// Smallest cluster whose even slices of `sel_max` selected entries and
+// `window` window positions fit one 128-key tile per CTA; 0 if none <= 16.
+int attn_cluster_min(int sel_max, int window) {
+  for (int r = 1; r <= 16; ++r)
+    if ((sel_max + r - 1) / r + (window + r - 1) / r <= kTK) return r;
+  return 0;
+}
 
 bool attn_tc_supported(const csa_params_t* p, int q_dtype, int kv_dtype, int swa_dtype, bool has_window) {
   if (p->h_q != kH || p->d != kD || q_dtype != kBF16) return false;
@@ -430,13 +637,68 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
   a.tau = p->softmax_scale;
   a.part = static_cast<float*>(workspace);
   a.splits = attn_tc_splits(max_keys);
-  if (!L.attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    L.attr = true;
+  a.sink = sink;
+  a.out = out->data;
+  a.out_dtype = out->dtype;
+  a.lse = lse;
+  for (int c = 0; c < 2; ++c)
+    if (!L.attr[c]) {
+      void* fn = c ? reinterpret_cast<void*>(attn_tc_kernel<true>) : reinterpret_cast<void*>(attn_tc_kernel<false>);
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+      if (e == cudaSuccess && c) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      L.attr[c] = true;
+    }
+  // One cluster per query when its keys fit 16 CTAs of one tile each: the
+  // largest size (least work per CTA) whose nq clusters are co-resident.
+  const int rmin = attn_cluster_min(max_keys - p->window, p->window);
+  int R = 0;
+  for (int r = 16; rmin > 0 && r >= rmin && R == 0; --r) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(r, nq);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = r;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (L.cluster_ok[r] == 0) {
+      int ncl = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveClusters(&ncl, attn_tc_kernel<true>, &cfg);
+      L.cluster_ok[r] = (e == cudaSuccess && ncl >= 1) ? ncl : -1;
+      cudaGetLastError();
+    }
+    if (L.cluster_ok[r] >= nq || (r == rmin && L.cluster_ok[r] > 0)) R = r;
+  }
+  if (R > 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(R, nq);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = R;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+      prof_begin(stream);
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, qmap, a);
+      if (e != cudaSuccess) {
+        check_launch("attn_tc_cluster_kernel", stream);
+        return set_error(CSA_ERR_CUDA, "attn_tc_kernel (cluster) launch: %s", cudaGetErrorString(e));
+      }
+      return check_launch("attn_tc_cluster_kernel", stream);
+    }
   }
   prof_begin(stream);
-  attn_tc_kernel<<<dim3(a.splits, nq), kThreads, kSmem, stream>>>(qmap, a);
+  attn_tc_kernel<false><<<dim3(a.splits, nq), kThreads, kSmem, stream>>>(qmap, a);
   csa_status_t st = check_launch("attn_tc_kernel", stream);
   if (st != CSA_OK) return st;
   return launch_attn_merge(a.part, nq, a.splits, kH, kD, sink, out->data, out->dtype, lse, stream);

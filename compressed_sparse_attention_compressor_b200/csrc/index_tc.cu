@@ -589,8 +589,11 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         for (int h = 0; h < kHeads; ++h) w_r[h] = ws[h];
         for (int t = grp; t < nt; t += 2) {
           const int acc = grp;
-          // the whole warp takes the same branch (warp-wide TMEM ops below)
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(tfull, (t >> 1) & 1, kWaitLimit))) {
+          // lane 0 polls, the warp follows its verdict (warp-wide TMEM ops below)
+          bool tok = true;
+          if (lane == 0) tok = mbar_wait(tfull, (t >> 1) & 1, kWaitLimit);
+          __syncwarp();  // orders the other lanes after lane 0's acquire
+          if (!__shfl_sync(0xFFFFFFFFu, tok, 0)) {
             atomicOr(&g_index_tc_error, 1u);
             sh.fail = 1;
             break;
@@ -599,7 +602,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
           float ks = 1.f;
           if constexpr (FP8) {
             const int ss = t % kSStages;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sfull[ss], (t / kSStages) & 1, kWaitLimit))) {
+            bool sok = true;
+            if (lane == 0) sok = mbar_wait(&sfull[ss], (t / kSStages) & 1, kWaitLimit);
+            __syncwarp();
+            if (!__shfl_sync(0xFFFFFFFFu, sok, 0)) {
               atomicOr(&g_index_tc_error, 1u);
               sh.fail = 1;
               break;

@@ -22,6 +22,9 @@ CASES = {
     "bf16_sharp": (Wk.WORKLOADS["decode64k"], 2, 2, 1500, 128, False, True, False, float(np.sqrt(512))),
     "f32_prefill_like": (Wk.WORKLOADS["tiny"].scaled(h_q=16), 40, 1, 300, 512, False, True, True, 1.0),
     "bf16_no_window": (Wk.WORKLOADS["decode64k"].scaled(window=0), 3, 3, 800, 128, False, True, False, 1.0),
+    # enough queries that the per-query clusters shrink to the smallest size
+    # that fits (window values then re-gathered instead of held in registers)
+    "bf16_many_queries": (Wk.WORKLOADS["decode64k"], 40, 4, 1200, 128, False, True, False, 1.0),
 }
 
 
