@@ -40,15 +40,6 @@ sys.path.insert(0, ROOT)
 from compressed_sparse_attention_compressor_b200 import workloads as Wk  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = {
-    "index_topk_tc_kernel": "index_tc.cu",
-    "index_score_simt_kernel": "index_topk.cu",
-    "topk_row_kernel": "index_topk.cu",
-    "attn_simt_kernel": "attention.cu",
-    "attn_merge_kernel": "attention.cu",
-    "decode_append_kernel": "compress.cu",
-    "compress_kernel": "compress.cu",
-}
 
 
 def parse():
@@ -110,19 +101,23 @@ def load_peaks():
 
 
 def load_traffic(name):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel's
-    source is unchanged since the capture (else None)."""
-    try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f).get(name)
-        if not rec:
-            return None
-        src = os.path.join(ROOT, "compressed_sparse_attention_compressor_b200", "csrc", KERNEL_SOURCES[name])
-        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != rec["source_sha256_16"]:
-            return None
-        return float(rec["bytes_per_launch"])
-    except Exception:
-        return None
+    """DRAM bytes per launch from the committed ncu summary of a kernel
+    (profiles/<kernel>_<workload>.md), if the kernel's source is unchanged
+    since the capture (else None)."""
+    import glob
+    import re
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{name}_*.md"))):
+        try:
+            text = open(path).read()
+            nbytes = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", text).group(1))
+            src = re.search(r"- source:\s*(\S+)", text).group(1)
+            want = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text).group(1)
+            cur = os.path.join(ROOT, "compressed_sparse_attention_compressor_b200", "csrc", src)
+            if hashlib.sha256(open(cur, "rb").read()).hexdigest()[:16] == want:
+                return float(nbytes)
+        except Exception:
+            continue
+    return None
 
 
 # ---------------------------------------------------------------------------
