@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "pool.cuh"
 
 namespace csa {
 
@@ -18,11 +19,12 @@ csa_status_t launch_decode_append(const csa_params_t* p, int batch, const csa_de
                                   int64_t* q_pos, int32_t* q_req, void* zero, size_t zero_bytes,
                                   cudaStream_t stream);
 bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dtype, int k_dtype);
+bool index_tc_append_supported(const csa_params_t* p, int w_dtype);
 size_t index_tc_control_bytes(int batch);
 size_t index_tc_workspace_bytes(int batch, int64_t cap, int k);
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
-                                  float* out_score, void* ws, cudaStream_t stream);
+                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap = nullptr);
 uint32_t index_tc_take_error();
 uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
@@ -331,14 +333,47 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
   const int max_keys = static_cast<int>((sparse ? p->topk : cc->cap) + p->window);
   void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys));
 
-  if ((st = launch_decode_append(p, batch, cc, tok, pos, n_vis, q_pos, q_req, tc ? index_ws : nullptr,
-                                 tc ? index_tc_control_bytes(batch) : 0, s)) != CSA_OK)
+  // CSA on the tensor-core indexer: the token is appended inside the indexer
+  // (by the CTA that owns each request's last chunk); otherwise by its own kernel
+  const bool fused = tc && index_tc_append_supported(p, tok->w_ik.dtype);
+  if (fused) {
+    const cudaError_t e = cudaMemsetAsync(index_ws, 0, index_tc_control_bytes(batch), s);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    AppendArgs ap;
+    ap.pos = pos;
+    ap.m = p->m;
+    ap.d = p->d;
+    ap.act_dtype = tok->c.dtype;
+    ap.c_t = tok->c.data;
+    ap.z_t = tok->z.data;
+    ap.k_t = tok->k_swa.data;
+    ap.v_t = tok->v_swa.data;
+    ap.open_c = cc->open_c.data;
+    ap.open_z = cc->open_z.data;
+    ap.swa_k = cc->swa_k.data;
+    ap.swa_v = cc->swa_v.data;
+    ap.swa_dtype = cc->swa_k.dtype;
+    ap.swa_cap = p->swa_cap;
+    ap.kv = make_out_spec(&cc->kv, p->d);
+    ap.w_ik = tok->w_ik.data;
+    ap.w_dtype = tok->w_ik.dtype;
+    ap.kidx = make_out_spec(&cc->kidx, p->d_idx);
+    ap.n_vis_out = n_vis;
+    ap.q_pos_out = q_pos;
+    ap.q_req_out = q_req;
+    ap.shrink = 0;
+    if ((st = launch_index_topk_tc(p, batch, &tok->q_idx, tok->w, &cc->kidx, cc->cap, n_vis, idx, nullptr, index_ws,
+                                   s, &ap)) != CSA_OK)
+      return st;
+  } else if ((st = launch_decode_append(p, batch, cc, tok, pos, n_vis, q_pos, q_req, tc ? index_ws : nullptr,
+                                        tc ? index_tc_control_bytes(batch) : 0, s)) != CSA_OK) {
     return st;
-  if (tc) {
+  }
+  if (tc && !fused) {
     if ((st = launch_index_topk_tc(p, batch, &tok->q_idx, tok->w, &cc->kidx, cc->cap, n_vis, idx, nullptr, index_ws,
                                    s)) != CSA_OK)
       return st;
-  } else if (sparse) {
+  } else if (sparse && !tc) {
     const int64_t ld = round_up(cc->cap, 4);
     float* scores = static_cast<float*>(index_ws);
     if ((st = launch_index_score(p, batch, &tok->q_idx, tok->w, &cc->kidx, batch, cc->cap, q_req, n_vis, scores, ld,

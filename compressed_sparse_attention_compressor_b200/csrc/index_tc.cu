@@ -49,6 +49,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "pool.cuh"
 #include "sm100.cuh"
 
 namespace csa {
@@ -72,6 +73,7 @@ constexpr int kEqCache = 8192;                   // boundary entries resolved in
 constexpr int kACache = 2048;                    // entries above the boundary kept in shared memory
 constexpr int kMaxChunks = 148;                  // CTAs of one request (<= SMs)
 constexpr int kSStages = 16;                     // FP8 row-scale ring (one 512-byte tile each)
+constexpr int kAppendShrink = 26;                // tiles the appending CTA's chunk gives up
 constexpr uint32_t kWaitLimit = 1u << 22;        // mbarrier polls
 constexpr uint32_t kSpinLimit = 1u << 22;        // grid-barrier polls (~64 ns apart)
 static_assert(kScoreCol + kMaxChunkTiles <= kTmemCols, "TMEM columns");
@@ -95,7 +97,7 @@ struct Cfg {
   static constexpr int kSmem = oMisc + 256 + 1024;
   // FP8: N = 128 = both E4M3 terms of the split query (rows 0..63 and 64..127 of B)
   static constexpr uint32_t kIdesc = FP8 ? idesc(0, 0, kTileM, 2 * kHeads) : idesc(1, 1, kTileM, kHeads);
-  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 4) <= 512, "mbarrier area");
+  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 5) <= 512, "mbarrier area");
   static_assert(oB % 1024 == 0, "operand alignment");
   static_assert(kSmem <= 232448, "shared memory");
   // phase-2 scratch, inside the (then idle) stage and scale rings
@@ -125,6 +127,8 @@ struct IdxArgs {
   uint32_t* cnt;           // [batch][chunks][2] entries above / at the boundary per chunk
   uint2* st;               // [batch][chunks][k] (index, score bits) above the boundary, beyond kACache
   uint2* eq;               // [batch][chunks][kMaxChunkTiles * 128] (index, score bits) at the boundary
+  int append;              // 1: n = (pos + 1) / m and the last chunk's CTA appends the token
+  AppendArgs ap;
 };
 
 struct Shared {
@@ -352,6 +356,122 @@ __device__ __forceinline__ void block_sum2(uint32_t& a, uint32_t& b, uint32_t* s
   __syncthreads();
 }
 
+// All threads of one CTA: the decode-step append of request r.  wbuf: room
+// for W_IK (d x 128, 16-aligned; the idle stage ring); scratch: d + 256
+// floats; wbar: an initialised mbarrier.  The stores are visible to this
+// CTA's later TMA loads (and to every later kernel) when it returns.
+__device__ void append_block(const AppendArgs& p, int r, int64_t cap, uint8_t* wbuf, float* scratch,
+                             uint64_t* wbar, Shared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = p.d, m = p.m;
+  const int64_t t = p.pos[r];
+  const bool closes = (t + 1) % m == 0;
+  const int wbytes = d * kDI * elem_bytes(p.w_dtype);
+  if (closes && tid == 0) {  // W_IK by bulk copies, in flight while the block is pooled
+    mbar_arrive_expect_tx(wbar, wbytes);
+    for (int off = 0; off < wbytes; off += 32768)
+      bulk_load(wbuf + off, static_cast<const uint8_t*>(p.w_ik) + off, min(32768, wbytes - off), wbar);
+  }
+  const int ea = elem_bytes(p.act_dtype), es = elem_bytes(p.swa_dtype);
+  const int vecs = d / 8;
+  const int slot_m = static_cast<int>(t % m);
+  const int64_t slot_w = t % p.swa_cap;
+  const char* crow = static_cast<const char*>(p.c_t) + static_cast<int64_t>(r) * d * ea;
+  const char* zrow = static_cast<const char*>(p.z_t) + static_cast<int64_t>(r) * d * ea;
+  char* ocb = static_cast<char*>(p.open_c) + static_cast<int64_t>(r) * m * d * ea;
+  char* ozb = static_cast<char*>(p.open_z) + static_cast<int64_t>(r) * m * d * ea;
+  // the token's rows into their slots: SWA key / value, open-block C / Z
+  for (int task = tid; task < 4 * vecs; task += kThreads) {
+    const int row = task / vecs, col = (task % vecs) * 8;
+    float v[8];
+    const char* src = row == 0 ? static_cast<const char*>(p.k_t) + static_cast<int64_t>(r) * d * ea
+                    : row == 1 ? static_cast<const char*>(p.v_t) + static_cast<int64_t>(r) * d * ea
+                    : row == 2 ? crow : zrow;
+    load8(src, p.act_dtype, col, nullptr, 1, v);
+    char* dst = row == 0 ? static_cast<char*>(p.swa_k) + (static_cast<int64_t>(r) * p.swa_cap + slot_w) * d * es
+              : row == 1 ? static_cast<char*>(p.swa_v) + (static_cast<int64_t>(r) * p.swa_cap + slot_w) * d * es
+              : (row == 2 ? ocb : ozb) + static_cast<int64_t>(slot_m) * d * ea;
+    store8(dst, row < 2 ? p.swa_dtype : p.act_dtype, col, v);
+  }
+  if (tid == 0) {
+    p.n_vis_out[r] = static_cast<int32_t>((t + 1) / m);
+    p.q_pos_out[r] = t;
+    p.q_req_out[r] = r;
+  }
+  if (closes) {  // uniform over the CTA
+    const int64_t row = static_cast<int64_t>(r) * cap + (t + 1) / m - 1;
+    float* pooled = scratch;  // [d]
+    float* red = scratch + d;  // [2][128]
+    // every thread of a warp pools 8 channels (FP8: 8 lanes = one 64-channel scale group)
+    const int nvt = (vecs + 31) / 32 * 32;
+    for (int vec = tid; vec < nvt; vec += kThreads) {  // warp-uniform trip count
+      const bool valid = vec < vecs;
+      const int col = valid ? vec * 8 : 0;
+      float v[8];
+      if (valid) {
+        auto rowC = [&](int i) -> const char* { return i == slot_m ? crow : ocb + static_cast<int64_t>(i) * d * ea; };
+        auto rowZ = [&](int i) -> const char* { return i == slot_m ? zrow : ozb + static_cast<int64_t>(i) * d * ea; };
+        pool8(rowC, rowZ, p.act_dtype, m, col, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pooled[col + e] = v[e];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      store_pooled8(p.kv, row, col, v, valid);
+    }
+    // indexer key = pooled . W_IK (fp32 pooled row, before storage rounding):
+    // thread (j, half) sums half of the d channels of output j
+    if (tid == 0 && !mbar_wait(wbar, 0, kWaitLimit)) {
+      atomicOr(&g_index_tc_error, 1u);
+      sh.fail = 1;
+    }
+    __syncthreads();  // pooled row complete; W_IK landed (or the wait gave up)
+    const bool wok = !sh.fail;
+    if (tid < 2 * kDI) {
+      const int j = tid & (kDI - 1), half = tid / kDI;
+      const int c0 = half * (d / 2), c1 = c0 + d / 2;
+      float acc = 0.f;
+      if (wok) {
+        if (p.w_dtype == kBF16) {
+          const uint16_t* w = reinterpret_cast<const uint16_t*>(wbuf) + j;
+          for (int c = c0; c < c1; ++c) acc = fmaf(pooled[c], bf16_bits_to_f32(w[c * kDI]), acc);
+        } else {
+          const float* w = reinterpret_cast<const float*>(wbuf) + j;
+          for (int c = c0; c < c1; ++c) acc = fmaf(pooled[c], w[c * kDI], acc);
+        }
+      }
+      red[half * kDI + j] = acc;
+    }
+    __syncthreads();
+    float key = 0.f;
+    if (tid < kDI) key = red[tid] + red[kDI + tid];
+    if (wok) {
+      if (p.kidx.dtype == kFP8) {
+        float a = tid < kDI ? fabsf(key) : 0.f;
+        a = warp_max(a);
+        if (lane == 0 && warp < kDI / 32) red[2 * kDI + warp] = a;
+        __syncthreads();
+        float amax = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDI / 32; ++w) amax = fmaxf(amax, red[2 * kDI + w]);
+        const float sc = amax > 0.f ? amax / 448.f : 1.f;
+        if (tid < kDI) static_cast<uint8_t*>(p.kidx.data)[row * p.kidx.row_stride + tid] = f32_to_e4m3(key / sc);
+        if (tid == 0) p.kidx.scale[row * p.kidx.scale_stride] = sc;
+      } else if (tid < kDI) {
+        if (p.kidx.dtype == kBF16) static_cast<uint16_t*>(p.kidx.data)[row * p.kidx.row_stride + tid] = f32_to_bf16_bits(key);
+        else static_cast<float*>(p.kidx.data)[row * p.kidx.row_stride + tid] = key;
+      }
+    }
+  }
+  // the generic-proxy stores above, before this CTA's TMA (async-proxy) loads
+  // of the same rows; W_IK's shared memory, before TMA writes it again
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  fence_proxy_async_smem();
+  __threadfence();
+  __syncthreads();
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap,
@@ -370,15 +490,27 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   uint64_t* tempty = tfull + 1;          // ... and have been read back
   uint64_t* qbar = tempty + 1;
   uint64_t* mdone = qbar + 1;
+  uint64_t* abar = mdone + 1;  // W_IK of the in-kernel append
   uint8_t* Bs = smem + C::oB;
   const float* scale_ring = reinterpret_cast<const float*>(smem + C::oScales);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x / a.chunks, c = blockIdx.x % a.chunks;
-  const int64_t n = min(max(static_cast<int64_t>(a.n_visible[r]), int64_t(0)), a.cap);
+  const int64_t n_raw = a.append ? (a.ap.pos[r] + 1) / a.ap.m : static_cast<int64_t>(a.n_visible[r]);
+  const int64_t n = min(max(n_raw, int64_t(0)), a.cap);
   const int tiles_req = static_cast<int>((n + kTileM - 1) / kTileM);
-  const int t0 = static_cast<int>(static_cast<int64_t>(c) * tiles_req / a.chunks);
-  const int t1 = static_cast<int>(static_cast<int64_t>(c + 1) * tiles_req / a.chunks);
+  int t0, t1;
+  if (a.append && a.chunks > 1) {
+    // the last chunk (whose CTA appends the token first) is shorter by `shrink` tiles
+    const int per = (tiles_req + a.chunks - 1) / a.chunks;
+    const int last = min(tiles_req, max(1, per - a.ap.shrink));
+    const int rest = tiles_req - last;
+    t0 = c < a.chunks - 1 ? c * rest / (a.chunks - 1) : rest;
+    t1 = c < a.chunks - 1 ? (c + 1) * rest / (a.chunks - 1) : tiles_req;
+  } else {
+    t0 = static_cast<int>(static_cast<int64_t>(c) * tiles_req / a.chunks);
+    t1 = static_cast<int>(static_cast<int64_t>(c + 1) * tiles_req / a.chunks);
+  }
   const int nt = min(t1 - t0, kMaxChunkTiles);
   const int64_t base = static_cast<int64_t>(t0) * kTileM;  // first key of the chunk
   const int nloc = static_cast<int>(max(int64_t(0), min(n, static_cast<int64_t>(t0 + nt) * kTileM) - base));
@@ -396,10 +528,13 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     mbar_init(tempty, kNAcc * 128);
     mbar_init(qbar, 1);
     mbar_init(mdone, 1);
+    mbar_init(abar, 1);
     sh.fail = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  if (a.append && c == a.chunks - 1)
+    append_block(a.ap, r, a.cap, smem + C::oStages, reinterpret_cast<float*>(smem + C::oHist), abar, sh);
 
   // ================= phase 1: stream the keys, scores into TMEM =================
   if (warp == 0) {
@@ -409,6 +544,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       bulk_load(smem + C::oQ, a.q_idx + static_cast<int64_t>(r) * kHeads * kDI, kHeads * kDI * 2, qbar);
       int issued = 0, sissued = 0;
       const int nst = (nt + C::kTPS - 1) / C::kTPS;
+      const uint64_t l2_stream = l2_policy_evict_first();
       for (int p = 0; p < nst && !sh.fail; ++p) {
         const int s = p % C::kStages;
         if (!mbar_wait(&empty[s], ((p / C::kStages) & 1) ^ 1, kWaitLimit)) {
@@ -420,11 +556,13 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         const int y = static_cast<int>(r * a.cap + static_cast<int64_t>(t0 + t) * kTileM);
         uint8_t* dst = smem + C::oStages + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        // the keys are read once: evict them from L2 first, so that the stream
+        // does not push out the code and the small data of the later phases
         if constexpr (FP8) {
-          tma_load_2d(dst, &kmap, &full[s], 0, y);  // 256 rows: tiles t and t + 1
+          tma_load_2d_hint(dst, &kmap, &full[s], 0, y, l2_stream);  // 256 rows: tiles t and t + 1
         } else {
-          tma_load_2d(dst, &kmap, &full[s], 0, y);
-          tma_load_2d(dst + 16384, &kmap, &full[s], 64, y);
+          tma_load_2d_hint(dst, &kmap, &full[s], 0, y, l2_stream);
+          tma_load_2d_hint(dst + 16384, &kmap, &full[s], 64, y, l2_stream);
         }
         issued = p + 1;
         if constexpr (FP8) {
@@ -970,7 +1108,17 @@ bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dty
   if (static_cast<int64_t>(batch) * cap >= (int64_t(1) << 31)) return false;
   const int ch = index_tc_chunks(batch, cap);
   const int64_t tiles = (cap + kTileM - 1) / kTileM;
-  return ch <= kMaxChunks && (tiles + ch - 1) / ch <= kMaxChunkTiles && p->topk >= 1;
+  // room for the in-kernel append's shorter last chunk
+  const int64_t per = (tiles + ch - 1) / ch + (ch > 1 ? (kAppendShrink + ch - 2) / (ch - 1) + 1 : 0);
+  return ch <= kMaxChunks && per <= kMaxChunkTiles && p->topk >= 1;
+}
+
+// The decode step can append inside the indexer: W_IK (d x 128) fits the
+// idle stage ring and the pooled row the shared scratch.
+bool index_tc_append_supported(const csa_params_t* p, int w_dtype) {
+  const int wb = w_dtype == kBF16 ? 2 : 4;
+  return p->d % 8 == 0 && static_cast<size_t>(p->d) * kDI * wb <= static_cast<size_t>(Cfg<true>::oScales) &&
+         static_cast<size_t>(p->d + 3 * kDI) * 4 <= 2 * kHistBins * 4;
 }
 
 size_t index_tc_control_bytes(int batch) { return static_cast<size_t>(batch) * (2 * kHistBins + 4) * 4; }
@@ -988,7 +1136,7 @@ size_t index_tc_workspace_bytes(int batch, int64_t cap, int k) {
 // must be zero on entry (the caller zeroes them).
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
-                                  float* out_score, void* ws, cudaStream_t stream) {
+                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap) {
   Launcher& L = launcher();
   if (!L.encode) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const bool fp8 = k_idx->dtype == kFP8;
@@ -1029,6 +1177,13 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.k = p->topk;
   a.out_idx = out_idx;
   a.out_score = out_score;
+  a.append = ap != nullptr;
+  if (ap) {
+    a.ap = *ap;
+    a.ap.shrink = kAppendShrink;
+  } else {
+    memset(&a.ap, 0, sizeof(a.ap));
+  }
   char* base = static_cast<char*>(ws);
   size_t off = 0;
   auto take = [&](size_t bytes) {

@@ -21,6 +21,7 @@ DECODE = {
     "tiny_open": Wk.WORKLOADS["tiny"].scaled(context=1022),           # block not closed by this token
     "decode64k": Wk.WORKLOADS["decode64k"].scaled(batch=3, context=4096 + 4 * 37),
     "decode1m": Wk.WORKLOADS["decode1m"].scaled(batch=2, context=8192),
+    "decode1m_open": Wk.WORKLOADS["decode1m"].scaled(batch=2, context=8190),  # appended in the indexer, block open
     "hybrid_csa": Wk.WORKLOADS["hybrid_csa"].scaled(batch=2, context=3000),
     "hybrid_hca": Wk.WORKLOADS["hybrid_hca"].scaled(batch=2, context=128 * 40),
     "hybrid_ratio1": Wk.WORKLOADS["hybrid_ratio1"].scaled(batch=2, context=2500, topk=300),
