@@ -1097,7 +1097,7 @@ int index_tc_chunks(int batch, int64_t cap) {
   const int64_t tiles = (cap + kTileM - 1) / kTileM;
   int ch = sms / (batch > 0 ? batch : 1);
   if (ch > tiles) ch = static_cast<int>(tiles > 0 ? tiles : 1);
-  return ch;
+  return ch > 0 ? ch : 1;  // more requests than SMs: not run by this kernel, sized as one chunk
 }
 
 bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dtype, int k_dtype) {

@@ -1,5 +1,6 @@
 // Block pooling and quantised row stores shared by the compressor, the
-// decode-step append kernel and the indexer's in-kernel append.
+// decode-step append kernel and the indexer's in-kernel append (whose
+// argument block is below).
 //
 // "DeepSeek-V4.1-Flash, illustrated", Equation (1) figure (compression
 // weights Z over a block of projected entries C); tech-report tour, "A
