@@ -143,6 +143,37 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
+// Bounded per-request grid barrier in two halves, so that local work can
+// run between the arrival and the wait.  request_arrive: the CTA's earlier
+// writes, then one arrival.  request_wait: until `target` arrivals; false on
+// a timeout.
+__device__ void request_arrive(uint32_t* ctr) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+  }
+}
+
+__device__ bool request_wait(uint32_t* ctr, uint32_t target, Shared& sh) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    uint32_t it = 0;
+    while (ld_acquire_gpu(ctr) < target) {
+      if (++it > kSpinLimit) {
+        atomicOr(&g_index_tc_error, 1u);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+    sh.bcast[7] = ok;
+  }
+  __syncthreads();
+  return sh.bcast[7] != 0;
+}
+
 // Bounded per-request grid barrier; returns false on timeout.
 __device__ bool request_barrier(uint32_t* ctr, uint32_t target, Shared& sh) {
   __syncthreads();
@@ -516,6 +547,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   const int nloc = static_cast<int>(max(int64_t(0), min(n, static_cast<int64_t>(t0 + nt) * kTileM) - base));
 
   if (tid == 0) {
+    prefetch_tensormap(&kmap);
+    if constexpr (FP8) prefetch_tensormap(&smap);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);  // the MMA commit
@@ -815,24 +848,27 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     };
 
     // scores TMEM -> shared memory in index order: warps 2..9, two per lane quarter
-    if (warp >= 2) {
-      const int q = warp & 3, half = (warp - 2) >> 2;
-      const uint32_t qaddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kScoreCol;
-      for (int tb = half * 32; tb < nt; tb += 64) {
-        uint32_t v[32];
-        tmem_ld32(qaddr + tb, v);
-        tmem_wait_ld();
+    auto copy_scores = [&]() {
+      if (warp >= 2) {
+        const int q = warp & 3, half = (warp - 2) >> 2;
+        const uint32_t qaddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kScoreCol;
+        for (int tb = half * 32; tb < nt; tb += 64) {
+          uint32_t v[32];
+          tmem_ld32(qaddr + tb, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (tb + u < nt) sc[(tb + u) * kTileM + q * 32 + lane] = __uint_as_float(v[u]);
+          for (int u = 0; u < 32; ++u)
+            if (tb + u < nt) sc[(tb + u) * kTileM + q * 32 + lane] = __uint_as_float(v[u]);
+        }
       }
-    }
-    __syncthreads();
+    };
     // every thread owns a contiguous, 4-aligned segment of the chunk's entries
     const int seg = ((nloc + kThreads - 1) / kThreads + 3) & ~3;
     const int i0 = min(nloc, tid * seg), i1 = min(nloc, i0 + seg);
 
     if (n <= k) {
+      copy_scores();
+      __syncthreads();
       for (int i = tid; i < nloc; i += kThreads) {
         oi[base + i] = static_cast<int32_t>(base + i);
         if (os) os[base + i] = sc[i];
@@ -853,7 +889,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         const uint32_t v = gh_g[i] + gh_g[kHistBins + i];
         if (v) atomicAdd(&gh1[i], v);
       }
-      bool alive = request_barrier(&bar[0], a.chunks, sh);
+      // arrive, copy the scores while the request's slower CTAs finish, wait
+      request_arrive(&bar[0]);
+      copy_scores();
+      bool alive = request_wait(&bar[0], a.chunks, sh);
       uint32_t shift = 20, prefix = 0;
       if (alive) {
         load_hist(hist, gh1);
