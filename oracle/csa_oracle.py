@@ -246,6 +246,59 @@ def boundary_gap(scores: np.ndarray, k: int) -> float:
 
 
 # ===========================================================================
+# hierarchical sparse indexer: the candidate pool and re-indexing inside it
+# ===========================================================================
+def block_scores(scores: np.ndarray, block: int) -> np.ndarray:
+    """Score of each block of ``block`` consecutive entries: the maximum of its
+    entries' index scores; a partial last block takes the maximum over the
+    entries it has.  Tech-report tour, chapter "Compressed Sparse Attention
+    2", section "The Hierarchical Sparse Indexer" (block score = max of its
+    positions)."""
+    s = np.asarray(scores, np.float64)
+    n = s.shape[0]
+    nb = (n + block - 1) // block
+    out = np.empty(nb, np.float64)
+    for b in range(nb):
+        out[b] = s[b * block: min(n, (b + 1) * block)].max()
+    return out
+
+
+def candidate_pool(scores: np.ndarray, block: int, pool_blocks: int) -> np.ndarray:
+    """The candidate pool the first Full layer builds for one query: the
+    ``pool_blocks`` best blocks of ``block`` entries (block score descending,
+    lower block first on exact ties), as block ids in ascending order, padded
+    with -1 when fewer blocks exist.  Same section as block_scores (2,048
+    blocks of 8 positions, a pool of 16,384 candidates)."""
+    bs = block_scores(scores, block)
+    chosen = topk(bs, pool_blocks)
+    chosen = np.sort(chosen[chosen >= 0])
+    out = np.full(pool_blocks, -1, np.int64)
+    out[: chosen.shape[0]] = chosen
+    return out
+
+
+def pool_entries(pool: np.ndarray, block: int, n_vis: int) -> np.ndarray:
+    """Visible entry ids of a pool, ascending."""
+    ids = [b * block + i for b in np.asarray(pool) if b >= 0 for i in range(block) if b * block + i < n_vis]
+    return np.asarray(ids, np.int64)
+
+
+def reindex_topk(q_idx: np.ndarray, w: np.ndarray, keys: np.ndarray, pool: np.ndarray, block: int, k: int):
+    """A Reindex layer's selection: the lightning-indexer scores of the pool's
+    entries only (its own query, the shared keys), top k of them (score
+    descending, lower entry first on exact ties), as entry ids padded with
+    -1.  Tech-report tour, chapter "Compressed Sparse Attention 2", sections
+    "Full, Reindex, and Reuse" (Reindex rescores the candidate pool) and "The
+    Hierarchical Sparse Indexer" (later indexers search only the pool).
+    keys [n_vis][d_idx] are the visible keys; returns (ids, scores of the pool)."""
+    ent = pool_entries(pool, block, keys.shape[0])
+    s = index_scores(q_idx, w, keys[ent]) if ent.shape[0] else np.zeros(0)
+    sel = topk(s, k)
+    ids = np.where(sel >= 0, ent[np.maximum(sel, 0)] if ent.shape[0] else -1, -1)
+    return ids.astype(np.int64), s
+
+
+# ===========================================================================
 # a4 / a5: sparse (or dense) attention + sliding window + sink, one softmax
 # ===========================================================================
 def window_positions(t: int, W: int, lo: int = 0) -> np.ndarray:

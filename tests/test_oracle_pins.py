@@ -375,3 +375,76 @@ def test_decode_step_ratio1_appends_the_token_row():
     for b in range(2):
         assert np.array_equal(res["new_rows"][b], c_t[b])
         assert np.allclose(res["new_keys"][b], c_t[b] @ O.decode_stored(inp.w_ik), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# hierarchical sparse indexer: candidate pool and re-indexing
+# ---------------------------------------------------------------------------
+def _brute_pool(scores, block, pool_blocks):
+    """Pool by the definition, in plain Python: every block's maximum, blocks
+    ranked by (maximum descending, block id ascending), the first pool_blocks
+    ids in ascending order."""
+    s = [float(x) for x in scores]
+    maxima = []
+    for b in range(0, len(s), block):
+        maxima.append(max(s[b:b + block]))
+    ranked = sorted(range(len(maxima)), key=lambda i: (-maxima[i], i))
+    chosen = sorted(ranked[:pool_blocks])
+    return chosen + [-1] * (pool_blocks - len(chosen))
+
+
+def test_pool_sizes_from_the_page():
+    with open(GOLDEN) as f:
+        g = json.load(f)["candidate_pool"]
+    assert g["pool_blocks"] * g["block"] == g["pool_positions"] == 16384
+    assert round(100.0 * g["pool_positions"] / g["context"], 1) == g["fraction_percent_about"]
+    # a pool built with those sizes holds exactly pool_positions entries
+    s = np.random.default_rng(0).standard_normal(200_000)
+    pool = O.candidate_pool(s, g["block"], g["pool_blocks"])
+    assert O.pool_entries(pool, g["block"], s.shape[0]).shape[0] == g["pool_positions"]
+
+
+def test_block_scores_partial_tail_and_ties():
+    s = np.array([1.0, 5.0, 2.0, 2.0, 7.0, 0.0, 0.0, 0.0, 5.0, 5.0, 1.0, 1.0, 3.0])
+    assert np.array_equal(O.block_scores(s, 4), [5.0, 7.0, 5.0, 3.0])  # last block: entry 12 alone
+    # blocks 0 and 2 tie at 5: the lower block wins the second place
+    assert np.array_equal(O.candidate_pool(s, 4, 2), [0, 1])
+    assert np.array_equal(O.candidate_pool(s, 4, 3), [0, 1, 2])
+    assert np.array_equal(O.candidate_pool(s, 4, 6), [0, 1, 2, 3, -1, -1])
+    assert np.array_equal(O.pool_entries(O.candidate_pool(s, 4, 6), 4, 13), np.arange(13))
+
+
+def test_pool_matches_brute_force():
+    rng = np.random.default_rng(1)
+    for n, block, pb in [(37, 4, 3), (64, 8, 5), (100, 1, 10), (9, 8, 1), (50, 7, 50)]:
+        s = np.round(rng.standard_normal(n), 1)  # coarse values: many exact ties
+        assert list(O.candidate_pool(s, block, pb)) == _brute_pool(s, block, pb), (n, block, pb)
+
+
+def test_pool_of_single_entry_blocks_is_the_top_entries():
+    s = np.random.default_rng(2).standard_normal(500)
+    assert np.array_equal(O.candidate_pool(s, 1, 40), np.sort(O.topk(s, 40)))
+
+
+def test_reindex_over_every_block_is_the_plain_top_k():
+    rng = np.random.default_rng(3)
+    keys = rng.standard_normal((300, 8))
+    q, w = rng.standard_normal((3, 8)), rng.random(3)
+    pool = O.candidate_pool(rng.standard_normal(300), 8, 64)  # 38 blocks <= 64: all of them
+    ids, _ = O.reindex_topk(q, w, keys, pool, 8, 20)
+    assert np.array_equal(ids, O.topk(O.index_scores(q, w, keys), 20))
+
+
+def test_reindex_selects_inside_the_pool_by_brute_force():
+    rng = np.random.default_rng(4)
+    keys = np.round(rng.standard_normal((120, 6)), 1)
+    q, w = rng.standard_normal((2, 6)), np.ones(2)
+    pool = O.candidate_pool(rng.standard_normal(120), 8, 4)
+    ids, _ = O.reindex_topk(q, w, keys, pool, 8, 10)
+    members = [b * 8 + i for b in pool if b >= 0 for i in range(8) if b * 8 + i < 120]
+    sc = {j: sum(max(0.0, float(np.dot(q[h], keys[j]))) * w[h] for h in range(2)) for j in members}
+    want = sorted(members, key=lambda j: (-sc[j], j))[:10]
+    assert sorted(ids.tolist()) == sorted(want)
+    # fewer pool entries than k: all of them, padded with -1
+    ids2, _ = O.reindex_topk(q, w, keys, pool, 8, 40)
+    assert sorted(ids2[ids2 >= 0].tolist()) == sorted(members) and np.all(ids2[len(members):] == -1)
