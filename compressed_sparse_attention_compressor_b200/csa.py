@@ -25,7 +25,8 @@ STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "C
 
 EXPORTS = ["csa_workspace_size", "csa_compress", "csa_index_topk", "csa_index_score", "csa_topk",
            "csa_sparse_swa_attention", "csa_decode_step", "csa_last_error", "csa_sync_status", "csa_profile_start",
-           "csa_profile_stop", "csa_profile_count", "csa_profile_get", "csa_sparse_swa_attention_noalloc"]
+           "csa_profile_stop", "csa_profile_count", "csa_profile_get", "csa_sparse_swa_attention_noalloc",
+           "csa_index_topk_pool", "csa_index_topk_reindex", "csa_index_pool_workspace_size"]
 
 
 class CsaError(RuntimeError):
@@ -75,6 +76,9 @@ def load() -> ctypes.CDLL:
         "csa_index_topk": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, V, V, V, SZ, V]),
         "csa_index_score": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, V, I64, V]),
         "csa_topk": (I32, [V, I32, I64, V, I32, V, V, V, SZ, V]),
+        "csa_index_topk_pool": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, I32, I32, V, V, V, V, SZ, V]),
+        "csa_index_topk_reindex": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, V, I32, I32, V, V, V, SZ, V]),
+        "csa_index_pool_workspace_size": (SZ, [P(Params), I32, I64, I32, I32]),
         "csa_sparse_swa_attention": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V, SZ, V]),
         "csa_sparse_swa_attention_noalloc": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V]),
         "csa_decode_step": (I32, [P(Params), I32, P(DecodeCaches), P(DecodeToken), V, T, V, V, SZ, V]),
@@ -205,6 +209,35 @@ def csa_topk(scores: torch.Tensor, n_rows: int, ld: int, n_valid: torch.Tensor, 
     _check(load().csa_topk(_ptr(scores), n_rows, ld, _ptr(n_valid), k, _ptr(out_idx), _ptr(out_score),
                            _ptr(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
                            _stream(stream)), "csa_topk")
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def csa_index_pool_workspace_size(p: Params, n_queries: int, max_entries: int, block: int, pool_blocks: int) -> int:
+    return load().csa_index_pool_workspace_size(ctypes.byref(p), n_queries, max_entries, block, pool_blocks)
+
+
+def csa_index_topk_pool(p: Params, n_queries: int, q_idx: DevTensor, w: torch.Tensor, k_idx: DevTensor, batch: int,
+                        cap: int, q_req: torch.Tensor | None, n_visible: torch.Tensor, block: int, pool_blocks: int,
+                        out_pool: torch.Tensor, out_idx: torch.Tensor | None, out_score: torch.Tensor | None,
+                        workspace: torch.Tensor, stream=None):
+    _check(load().csa_index_topk_pool(ctypes.byref(p), n_queries, ctypes.byref(q_idx.c()), _ptr(w),
+                                      ctypes.byref(k_idx.c()), batch, cap, _ptr(q_req), _ptr(n_visible), block,
+                                      pool_blocks, _ptr(out_pool), _ptr(out_idx), _ptr(out_score), _ptr(workspace),
+                                      _nbytes(workspace), _stream(stream)), "csa_index_topk_pool")
+
+
+def csa_index_topk_reindex(p: Params, n_queries: int, q_idx: DevTensor, w: torch.Tensor, k_idx: DevTensor,
+                           batch: int, cap: int, q_req: torch.Tensor | None, n_visible: torch.Tensor,
+                           pool: torch.Tensor, block: int, pool_blocks: int, out_idx: torch.Tensor,
+                           out_score: torch.Tensor | None, workspace: torch.Tensor, stream=None):
+    _check(load().csa_index_topk_reindex(ctypes.byref(p), n_queries, ctypes.byref(q_idx.c()), _ptr(w),
+                                         ctypes.byref(k_idx.c()), batch, cap, _ptr(q_req), _ptr(n_visible),
+                                         _ptr(pool), block, pool_blocks, _ptr(out_idx), _ptr(out_score),
+                                         _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "csa_index_topk_reindex")
 
 
 def csa_sparse_swa_attention(p: Params, n_queries: int, q: DevTensor, kv: DevTensor, batch: int, cap: int,

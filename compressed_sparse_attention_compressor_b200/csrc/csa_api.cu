@@ -30,15 +30,22 @@ uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                                 const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
                                 const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const int32_t* pool = nullptr, int block = 1,
+                                int pool_blocks = 0);
 csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
-                         int32_t* out_idx, float* out_score, cudaStream_t stream);
+                         int32_t* out_idx, float* out_score, cudaStream_t stream, int nv_div = 1, int ordered = 0);
+csa_status_t launch_block_max(const float* scores, int nq, int64_t ld, const int32_t* n_visible, int64_t cap,
+                              int block, float* out, int64_t ld_out, cudaStream_t stream);
+csa_status_t launch_pool_map(const int32_t* pos, const float* pos_score, int nq, int k, const int32_t* pool, int block,
+                             int pool_blocks, int32_t* out_idx, cudaStream_t stream);
 csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
                               int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible, const int32_t* q_req,
                               const csa_tensor_t* swa_k, const csa_tensor_t* swa_v, const int64_t* q_pos,
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
                               void* workspace, int max_keys, cudaStream_t stream);
 size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys);
+
+csa_status_t set_error(csa_status_t st, const char* fmt, ...);
 
 namespace {
 thread_local char g_msg[512] = "";
@@ -98,6 +105,31 @@ size_t index_ws_bytes(int nq, int64_t cap) {
   Carver c(nullptr);
   c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
   return c.off;
+}
+
+// Full layer of the hierarchical indexer: all scores, then the block maxima.
+size_t pool_ws_bytes(int nq, int64_t cap, int block) {
+  Carver c(nullptr);
+  c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
+  c.take<float>(static_cast<size_t>(nq) * round_up((cap + block - 1) / block, 4));
+  return c.off;
+}
+
+// Reindex layer: the pool's scores, the selected pool positions and their scores.
+size_t reindex_ws_bytes(int nq, int block, int pool_blocks, int k) {
+  Carver c(nullptr);
+  c.take<float>(static_cast<size_t>(nq) * round_up(static_cast<int64_t>(block) * pool_blocks, 4));
+  c.take<int32_t>(static_cast<size_t>(nq) * k);
+  c.take<float>(static_cast<size_t>(nq) * k);
+  return c.off;
+}
+
+csa_status_t check_pool_shape(int32_t block, int32_t pool_blocks) {
+  if (block < 1 || block > 128 || (block & (block - 1)) != 0)
+    return set_error(CSA_ERR_INVALID_ARG, "block=%d must be a power of two in [1, 128]", block);
+  if (pool_blocks < 1 || static_cast<int64_t>(block) * pool_blocks > (int64_t(1) << 30))
+    return set_error(CSA_ERR_INVALID_ARG, "bad pool_blocks=%d", pool_blocks);
+  return CSA_OK;
 }
 
 }  // namespace
@@ -242,6 +274,94 @@ csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_
       CSA_OK)
     return st;
   return launch_topk(scores, n_queries, ld, n_visible, cap, p->topk, out_idx, out_score, s);
+}
+
+namespace {
+
+csa_status_t check_index_args(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,
+                              const csa_tensor_t* k_idx, int32_t batch, int64_t cap, const int32_t* n_visible) {
+  csa_status_t st;
+  if ((st = check_params(p, true)) != CSA_OK) return st;
+  if (n_queries < 0 || cap < 0 || batch < 1) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap");
+  if (n_queries == 0) return CSA_OK;
+  if ((st = check_tensor("q_idx", q_idx, p->d_idx, true, true, false, 0)) != CSA_OK) return st;
+  if ((st = check_tensor("k_idx", k_idx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
+  if (w == nullptr || n_visible == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null w / n_visible");
+  return CSA_OK;
+}
+
+}  // namespace
+
+size_t csa_index_pool_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries, int32_t block,
+                                     int32_t pool_blocks) {
+  if (p == nullptr || n_queries < 0 || max_entries < 0 || block < 1 || pool_blocks < 1) return 0;
+  const size_t a = pool_ws_bytes(n_queries, max_entries, block);
+  const size_t b = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk > 0 ? p->topk : 1);
+  return (a > b ? a : b) + 256;
+}
+
+csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,
+                                 const csa_tensor_t* k_idx, int32_t batch, int64_t cap, const int32_t* q_req,
+                                 const int32_t* n_visible, int32_t block, int32_t pool_blocks, int32_t* out_pool,
+                                 int32_t* out_idx, float* out_score, void* workspace, size_t workspace_bytes,
+                                 csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  if ((st = check_index_args(p, n_queries, q_idx, w, k_idx, batch, cap, n_visible)) != CSA_OK) return st;
+  if ((st = check_pool_shape(block, pool_blocks)) != CSA_OK) return st;
+  if (out_idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "out_idx needs topk >= 1");
+  if (n_queries == 0) return CSA_OK;
+  if (out_pool == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null out_pool");
+  const size_t need = pool_ws_bytes(n_queries, cap, block);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  const int64_t ld = round_up(cap, 4);
+  const int64_t nb = (cap + block - 1) / block, ldb = round_up(nb, 4);
+  float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
+  float* bmax = c.take<float>(static_cast<size_t>(n_queries) * ldb);
+  if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s)) !=
+      CSA_OK)
+    return st;
+  if (out_idx != nullptr &&
+      (st = launch_topk(scores, n_queries, ld, n_visible, cap, p->topk, out_idx, out_score, s)) != CSA_OK)
+    return st;
+  if ((st = launch_block_max(scores, n_queries, ld, n_visible, cap, block, bmax, ldb, s)) != CSA_OK) return st;
+  return launch_topk(bmax, n_queries, ldb, n_visible, nb, pool_blocks, out_pool, nullptr, s, block, 1);
+}
+
+csa_status_t csa_index_topk_reindex(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx,
+                                    const float* w, const csa_tensor_t* k_idx, int32_t batch, int64_t cap,
+                                    const int32_t* q_req, const int32_t* n_visible, const int32_t* pool, int32_t block,
+                                    int32_t pool_blocks, int32_t* out_idx, float* out_score, void* workspace,
+                                    size_t workspace_bytes, csa_stream_t stream) {
+  g_msg[0] = 0;
+  csa_status_t st;
+  if ((st = check_index_args(p, n_queries, q_idx, w, k_idx, batch, cap, n_visible)) != CSA_OK) return st;
+  if ((st = check_pool_shape(block, pool_blocks)) != CSA_OK) return st;
+  if (p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "csa_index_topk_reindex needs topk >= 1");
+  if (n_queries == 0) return CSA_OK;
+  if (pool == nullptr || out_idx == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null pool / out_idx");
+  const size_t need = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk);
+  if (workspace == nullptr || workspace_bytes < need)
+    return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carver c(workspace);
+  const int64_t np = static_cast<int64_t>(block) * pool_blocks, ld = round_up(np, 4);
+  float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
+  int32_t* pos = c.take<int32_t>(static_cast<size_t>(n_queries) * p->topk);
+  float* pos_score = c.take<float>(static_cast<size_t>(n_queries) * p->topk);
+  if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, np, s, pool,
+                               block, pool_blocks)) != CSA_OK)
+    return st;
+  if ((st = launch_topk(scores, n_queries, ld, nullptr, np, p->topk, pos, pos_score, s)) != CSA_OK) return st;
+  if (out_score != nullptr) {
+    cudaError_t e = cudaMemcpyAsync(out_score, pos_score, static_cast<size_t>(n_queries) * p->topk * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+  }
+  return launch_pool_map(pos, pos_score, n_queries, p->topk, pool, block, pool_blocks, out_idx, s);
 }
 
 csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q,

@@ -26,17 +26,23 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kScoreThreads = 256;
 
+// pool != nullptr (re-indexing inside a candidate pool): score j of query
+// qi is that of entry pool[qi][j / block] * block + j % block for j <
+// pool_blocks * block, -inf where the pool slot is -1 or the entry is not
+// visible.
 template <int H, int DI>
 __global__ void __launch_bounds__(kScoreThreads)
 index_score_simt_kernel(const void* __restrict__ q_idx, int q_dtype, const float* __restrict__ w,
                         const void* __restrict__ keys, const float* __restrict__ kscale, int k_dtype,
                         int batch, int64_t cap, const int32_t* __restrict__ q_req,
-                        const int32_t* __restrict__ n_visible, float* __restrict__ scores, int64_t ld) {
+                        const int32_t* __restrict__ n_visible, float* __restrict__ scores, int64_t ld,
+                        const int32_t* __restrict__ pool, int block, int pool_blocks) {
   __shared__ __align__(16) float qs[H * DI];
   __shared__ float ws[H];
   const int qi = blockIdx.y;
   const int r = q_req ? q_req[qi] : qi;
-  const int64_t n = (r < 0 || r >= batch) ? 0 : min(max(static_cast<int64_t>(n_visible[qi]), int64_t(0)), cap);
+  const int64_t nvis = (r < 0 || r >= batch) ? 0 : min(max(static_cast<int64_t>(n_visible[qi]), int64_t(0)), cap);
+  const int64_t n = pool ? static_cast<int64_t>(pool_blocks) * block : nvis;
   const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kScoreThreads;
   if (j0 >= n) return;  // uniform over the CTA
   const char* qrow = static_cast<const char*>(q_idx) + static_cast<int64_t>(qi) * H * DI * elem_bytes(q_dtype);
@@ -45,7 +51,16 @@ index_score_simt_kernel(const void* __restrict__ q_idx, int q_dtype, const float
   __syncthreads();
   const int64_t j = j0 + threadIdx.x;
   if (j >= n) return;
-  const int64_t krow = static_cast<int64_t>(r) * cap + j;
+  int64_t e = j;  // the entry scored
+  if (pool) {
+    const int32_t b = pool[static_cast<int64_t>(qi) * pool_blocks + j / block];
+    e = b < 0 ? -1 : static_cast<int64_t>(b) * block + j % block;
+    if (e < 0 || e >= nvis) {
+      scores[static_cast<int64_t>(qi) * ld + j] = -INFINITY;
+      return;
+    }
+  }
+  const int64_t krow = static_cast<int64_t>(r) * cap + e;
   const char* kp = static_cast<const char*>(keys) + krow * DI * elem_bytes(k_dtype);
   const float* sp = (k_dtype == kFP8) ? kscale + krow : nullptr;
   float acc[H];
@@ -128,10 +143,12 @@ __device__ void find_bin(TopkShared& sh, int nb, uint32_t need) {
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
-                int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
+                int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int nv_div, int ordered) {
   __shared__ TopkShared sh;
   const int row = blockIdx.x;
-  const int64_t n = min(max(static_cast<int64_t>(n_valid[row]), int64_t(0)), max_n);
+  // valid columns: ceil(n_valid / nv_div), or max_n without n_valid
+  const int64_t nv = n_valid ? (static_cast<int64_t>(n_valid[row]) + nv_div - 1) / nv_div : max_n;
+  const int64_t n = min(max(nv, int64_t(0)), max_n);
   const float* s = scores + static_cast<int64_t>(row) * ld;
   int32_t* oi = out_idx + static_cast<int64_t>(row) * k;
   float* os = out_score ? out_score + static_cast<int64_t>(row) * k : nullptr;
@@ -189,6 +206,29 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
       tot_gt += a; tot_eq += b;
     }
     const uint32_t lm = (1u << lane) - 1u;
+    if (ordered) {
+      // the selection in ascending index order: entries above T, and the
+      // first take_eq equal to T
+      const bool sel = gt || (eq && base_eq + off_eq + __popc(beq & lm) < take_eq);
+      const uint32_t bsel = __ballot_sync(0xFFFFFFFFu, sel);
+      __syncthreads();
+      if (lane == 0) sh.warp_gt[warp] = __popc(bsel);
+      __syncthreads();
+      uint32_t off_s = 0, tot_s = 0;
+      for (int w2 = 0; w2 < kTopkWarps; ++w2) {
+        if (w2 < warp) off_s += sh.warp_gt[w2];
+        tot_s += sh.warp_gt[w2];
+      }
+      if (sel) {
+        const uint32_t p = base_gt + off_s + __popc(bsel & lm);
+        oi[p] = static_cast<int32_t>(j);
+        if (os) os[p] = v;
+      }
+      base_gt += tot_s;
+      base_eq += tot_eq;
+      __syncthreads();
+      continue;
+    }
     if (gt) {
       const uint32_t p = base_gt + off_gt + __popc(bgt & lm);
       oi[p] = static_cast<int32_t>(j);
@@ -211,12 +251,12 @@ template <int H, int DI>
 csa_status_t launch_score_t(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                             const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
                             const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const int32_t* pool, int block, int pool_blocks) {
   dim3 grid(static_cast<unsigned>((max_entries + kScoreThreads - 1) / kScoreThreads), nq);
   prof_begin(stream);
   index_score_simt_kernel<H, DI><<<grid, kScoreThreads, 0, stream>>>(
       q_idx->data, q_idx->dtype, w, k_idx->data, k_idx->scale, k_idx->dtype, batch, cap, q_req, n_visible, scores,
-      ld);
+      ld, pool, block, pool_blocks);
   return check_launch("index_score_simt_kernel", stream);
 }
 
@@ -225,12 +265,12 @@ csa_status_t launch_score_t(const csa_params_t* p, int nq, const csa_tensor_t* q
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                                 const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
                                 const int32_t* n_visible, float* scores, int64_t ld, int64_t max_entries,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const int32_t* pool, int block, int pool_blocks) {
   if (nq == 0 || max_entries == 0) return CSA_OK;
 #define CSA_SCORE_CASE(H, DI)                                                                                  \
   if (p->h_idx == H && p->d_idx == DI)                                                                         \
     return launch_score_t<H, DI>(p, nq, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, max_entries, \
-                                 stream);
+                                 stream, pool, block, pool_blocks);
   CSA_SCORE_CASE(4, 32)
   CSA_SCORE_CASE(8, 32)
   CSA_SCORE_CASE(16, 64)
@@ -241,11 +281,66 @@ csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_
 }
 
 csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
-                         int32_t* out_idx, float* out_score, cudaStream_t stream) {
+                         int32_t* out_idx, float* out_score, cudaStream_t stream, int nv_div, int ordered) {
   if (n_rows == 0) return CSA_OK;
   prof_begin(stream);
-  topk_row_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score);
+  topk_row_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score, nv_div,
+                                                       ordered);
   return check_launch("topk_row_kernel", stream);
+}
+
+namespace {
+
+// Block maxima of score rows: out[q][b] = max of scores[q][b*block ..
+// min(n, (b+1)*block)) for the n = n_visible[q] valid scores of row q.
+__global__ void block_max_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_visible,
+                                 int64_t cap, int block, float* __restrict__ out, int64_t ld_out) {
+  const int q = blockIdx.y;
+  const int64_t n = min(max(static_cast<int64_t>(n_visible[q]), int64_t(0)), cap);
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b * block >= n) return;
+  const float* s = scores + static_cast<int64_t>(q) * ld + b * block;
+  float m = s[0];
+  for (int i = 1; i < block && b * block + i < n; ++i) m = fmaxf(m, s[i]);
+  out[static_cast<int64_t>(q) * ld_out + b] = m;
+}
+
+// Pool positions -> entry ids: pos -> pool[q][pos / block] * block + pos % block;
+// -1 for padding and for positions whose score is -inf (not a visible entry).
+__global__ void pool_map_kernel(const int32_t* __restrict__ pos, const float* __restrict__ pos_score, int k,
+                                const int32_t* __restrict__ pool, int block, int pool_blocks,
+                                int32_t* __restrict__ out_idx) {
+  const int q = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= k) return;
+  const int32_t p = pos[static_cast<int64_t>(q) * k + i];
+  int32_t e = -1;
+  if (p >= 0 && pos_score[static_cast<int64_t>(q) * k + i] != -INFINITY) {
+    const int32_t b = pool[static_cast<int64_t>(q) * pool_blocks + p / block];
+    if (b >= 0) e = b * block + p % block;
+  }
+  out_idx[static_cast<int64_t>(q) * k + i] = e;
+}
+
+}  // namespace
+
+csa_status_t launch_block_max(const float* scores, int nq, int64_t ld, const int32_t* n_visible, int64_t cap,
+                              int block, float* out, int64_t ld_out, cudaStream_t stream) {
+  if (nq == 0) return CSA_OK;
+  const int64_t nb = (cap + block - 1) / block;
+  dim3 grid(static_cast<unsigned>((nb + 255) / 256), nq);
+  prof_begin(stream);
+  block_max_kernel<<<grid, 256, 0, stream>>>(scores, ld, n_visible, cap, block, out, ld_out);
+  return check_launch("block_max_kernel", stream);
+}
+
+csa_status_t launch_pool_map(const int32_t* pos, const float* pos_score, int nq, int k, const int32_t* pool, int block,
+                             int pool_blocks, int32_t* out_idx, cudaStream_t stream) {
+  if (nq == 0) return CSA_OK;
+  dim3 grid(static_cast<unsigned>((k + 255) / 256), nq);
+  prof_begin(stream);
+  pool_map_kernel<<<grid, 256, 0, stream>>>(pos, pos_score, k, pool, block, pool_blocks, out_idx);
+  return check_launch("pool_map_kernel", stream);
 }
 
 }  // namespace csa

@@ -179,6 +179,64 @@ csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int
                       int32_t k, int32_t* out_idx, float* out_score, void* workspace,
                       size_t workspace_bytes, csa_stream_t stream);
 
+/* Hierarchical sparse indexer, first (Full) layer.  [TOUR] chapter
+ * "Compressed Sparse Attention 2", section "The Hierarchical Sparse Indexer"
+ * (a block's score is the maximum of its positions' scores; the best blocks
+ * form a candidate pool, e.g. 2,048 blocks of 8 positions = 16,384
+ * candidates at 1M context), section "Full, Reindex, and Reuse" (the Full
+ * layer scores everything and builds the pool).
+ * Scores s_j as csa_index_topk.  Block b of query i covers entries
+ * [b*block, (b+1)*block) and scores max s_j over its visible entries; the
+ * last block may be partial.  out_pool[i] receives the min(pool_blocks,
+ * ceil(n_visible[i] / block)) best blocks -- larger block score first,
+ * lower block id first among exactly equal scores -- as block ids in
+ * ASCENDING order, padded with -1.
+ *   block        power of two in [1, 128].
+ *   out_pool     [n_queries][pool_blocks] int32.
+ *   out_idx      optional [n_queries][p->topk] int32 (needs p->topk >= 1):
+ *                the layer's own top-k, exactly as csa_index_topk;
+ *   out_score    optional, with out_idx, as csa_index_topk.
+ *   workspace    csa_index_pool_workspace_size(p, n_queries, cap, block,
+ *                pool_blocks) bytes.
+ * Other arguments, layouts and errors as csa_index_topk.                    */
+csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx,
+                                 const float* w, const csa_tensor_t* k_idx, int32_t batch, int64_t cap,
+                                 const int32_t* q_req, const int32_t* n_visible, int32_t block,
+                                 int32_t pool_blocks, int32_t* out_pool, int32_t* out_idx,
+                                 float* out_score, void* workspace, size_t workspace_bytes,
+                                 csa_stream_t stream);
+
+/* Hierarchical sparse indexer, a Reindex layer.  [TOUR] chapter "Compressed
+ * Sparse Attention 2", sections "Full, Reindex, and Reuse" (a Reindex layer
+ * runs its own indexer query over the candidate pool only) and "The
+ * Hierarchical Sparse Indexer" (later indexers search the pool, not the
+ * whole context).
+ * Pool position j of query i (j < pool_blocks * block) is entry
+ * e = pool[i][j / block] * block + j % block; it is a candidate when
+ * pool[i][j / block] >= 0 and e < n_visible[i].  out_idx[i] receives the
+ * min(topk, candidates) candidates with the largest s_e (computed as in
+ * csa_index_topk, from this call's q_idx and w) as ENTRY ids -- larger
+ * score first in value, the earlier pool position first among exactly equal
+ * scores (the lower entry when the pool is ascending, as csa_index_topk_pool
+ * writes it).  The order inside out_idx[i] is unspecified; unused slots hold
+ * -1 (out_score -inf).
+ *   pool         [n_queries][pool_blocks] int32 block ids (-1 = empty slot).
+ *   out_idx      [n_queries][p->topk] int32; out_score optional fp32.
+ *   workspace    csa_index_pool_workspace_size(...) bytes.
+ * Requires p->topk >= 1.  Other arguments as csa_index_topk_pool.           */
+csa_status_t csa_index_topk_reindex(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx,
+                                    const float* w, const csa_tensor_t* k_idx, int32_t batch, int64_t cap,
+                                    const int32_t* q_req, const int32_t* n_visible, const int32_t* pool,
+                                    int32_t block, int32_t pool_blocks, int32_t* out_idx,
+                                    float* out_score, void* workspace, size_t workspace_bytes,
+                                    csa_stream_t stream);
+
+/* Workspace bytes that csa_index_topk_pool and csa_index_topk_reindex need
+ * for n_queries queries with at most max_entries visible entries (0 for
+ * invalid arguments).                                                       */
+size_t csa_index_pool_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries,
+                                     int32_t block, int32_t pool_blocks);
+
 /* a4 + a5 -- sparse (CSA) or dense (HCA) attention over compressed entries,
  * the sliding window and the sink, in one online softmax.  [ATLAS]
  * "compressed KV", "Sliding-window attention", "MLA"; [TOUR] "The indexer

@@ -101,3 +101,31 @@ def test_workspace_size_grows_with_problem(lib):
     # many queries (chunked prefill: more queries than SMs)
     p.topk = 512
     assert csa.csa_workspace_size(p, 4096, 33792) >= 4096 * 33792 * 4
+
+
+def test_pool_entry_points_reject_bad_arguments(lib):
+    p = csa.params(4, 512, 128, 64, 64, 64, 128, 128)
+    q, k = _t(), _t()
+    ws = csa.csa_index_pool_workspace_size(p, 4, 262144, 8, 2048)
+    # the Full layer keeps every score and every block maximum
+    assert ws >= 4 * 262144 * 4 + 4 * (262144 // 8) * 4
+    for block in (0, 3, 256):
+        st = lib.csa_index_topk_pool(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                     block, 64, 16, None, None, 16, 1 << 30, None)
+        assert st == 1 and b"block" in lib.csa_last_error()
+    st = lib.csa_index_topk_pool(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                 8, 0, 16, None, None, 16, 1 << 30, None)
+    assert st == 1 and b"pool_blocks" in lib.csa_last_error()
+    st = lib.csa_index_topk_pool(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                 8, 64, 16, None, None, 16, 64, None)
+    assert st == 3 and b"workspace" in lib.csa_last_error()
+    st = lib.csa_index_topk_reindex(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                    None, 8, 64, 16, None, 16, 1 << 30, None)
+    assert st == 1 and b"pool" in lib.csa_last_error()
+    st = lib.csa_index_topk_reindex(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                    16, 8, 64, 16, None, 16, 64, None)
+    assert st == 3 and b"workspace" in lib.csa_last_error()
+    p.topk = 0
+    st = lib.csa_index_topk_reindex(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
+                                    16, 8, 64, 16, None, 16, 1 << 30, None)
+    assert st == 1 and b"topk" in lib.csa_last_error()
