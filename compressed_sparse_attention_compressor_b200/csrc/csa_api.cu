@@ -24,7 +24,8 @@ size_t index_tc_control_bytes(int batch);
 size_t index_tc_workspace_bytes(int batch, int64_t cap, int k);
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
-                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap = nullptr);
+                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap = nullptr,
+                                  float* bmax = nullptr, int64_t ldb = 0, int block = 1);
 uint32_t index_tc_take_error();
 uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
@@ -107,12 +108,23 @@ size_t index_ws_bytes(int nq, int64_t cap) {
   return c.off;
 }
 
-// Full layer of the hierarchical indexer: all scores, then the block maxima.
-size_t pool_ws_bytes(int nq, int64_t cap, int block) {
+// Full layer of the hierarchical indexer: the block maxima, then either all
+// scores (CUDA-core scoring) or the fused indexer's workspace and a top-k
+// scratch for a caller that wants the pool alone.
+size_t pool_ws_bytes(const csa_params_t* p, int nq, int64_t cap, int block) {
   Carver c(nullptr);
-  c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
   c.take<float>(static_cast<size_t>(nq) * round_up((cap + block - 1) / block, 4));
-  return c.off;
+  const size_t head = c.off;
+  c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
+  size_t need = c.off;
+  if (p->topk >= 1 && p->h_idx > 0 && p->d_idx > 0) {
+    Carver t(nullptr);
+    t.off = head;
+    t.take<int32_t>(static_cast<size_t>(nq) * p->topk);
+    t.take<char>(index_tc_workspace_bytes(nq, cap, p->topk));
+    if (t.off > need) need = t.off;
+  }
+  return need;
 }
 
 // Reindex layer: the pool's scores, the selected pool positions and their scores.
@@ -295,7 +307,7 @@ csa_status_t check_index_args(const csa_params_t* p, int32_t n_queries, const cs
 size_t csa_index_pool_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries, int32_t block,
                                      int32_t pool_blocks) {
   if (p == nullptr || n_queries < 0 || max_entries < 0 || block < 1 || pool_blocks < 1) return 0;
-  const size_t a = pool_ws_bytes(n_queries, max_entries, block);
+  const size_t a = pool_ws_bytes(p, n_queries, max_entries, block);
   const size_t b = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk > 0 ? p->topk : 1);
   return (a > b ? a : b) + 256;
 }
@@ -312,15 +324,27 @@ csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const
   if (out_idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "out_idx needs topk >= 1");
   if (n_queries == 0) return CSA_OK;
   if (out_pool == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null out_pool");
-  const size_t need = pool_ws_bytes(n_queries, cap, block);
+  const size_t need = pool_ws_bytes(p, n_queries, cap, block);
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Carver c(workspace);
   const int64_t ld = round_up(cap, 4);
   const int64_t nb = (cap + block - 1) / block, ldb = round_up(nb, 4);
-  float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
   float* bmax = c.take<float>(static_cast<size_t>(n_queries) * ldb);
+  if (q_req == nullptr && n_queries == batch && p->topk >= 1 &&
+      index_tc_supported(p, batch, cap, q_idx->dtype, k_idx->dtype)) {
+    // the fused tensor-core indexer writes its top-k and the block maxima
+    int32_t* idx = c.take<int32_t>(static_cast<size_t>(n_queries) * p->topk);
+    void* tws = c.take<char>(index_tc_workspace_bytes(batch, cap, p->topk));
+    cudaError_t e = cudaMemsetAsync(tws, 0, index_tc_control_bytes(batch), s);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    if ((st = launch_index_topk_tc(p, batch, q_idx, w, k_idx, cap, n_visible, out_idx ? out_idx : idx, out_score,
+                                   tws, s, nullptr, bmax, ldb, block)) != CSA_OK)
+      return st;
+    return launch_topk(bmax, n_queries, ldb, n_visible, nb, pool_blocks, out_pool, nullptr, s, block, 1);
+  }
+  float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
   if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s)) !=
       CSA_OK)
     return st;

@@ -129,6 +129,9 @@ struct IdxArgs {
   uint2* eq;               // [batch][chunks][kMaxChunkTiles * 128] (index, score bits) at the boundary
   int append;              // 1: n = (pos + 1) / m and the last chunk's CTA appends the token
   AppendArgs ap;
+  float* bmax;             // optional [batch][ldb]: max score of each block of `block` entries
+  int64_t ldb;
+  int block;               // power of two <= kTileM, so no block straddles two chunks
 };
 
 struct Shared {
@@ -862,12 +865,25 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         }
       }
     };
+    // block maxima of the chunk (the chunk starts on a tile, so on a block)
+    auto write_block_max = [&]() {
+      __syncthreads();
+      const int bs = a.block, nb = (nloc + bs - 1) / bs;
+      float* bm = a.bmax + static_cast<int64_t>(r) * a.ldb + base / bs;
+      for (int b = tid; b < nb; b += kThreads) {
+        const int e0 = b * bs, e1 = min(nloc, e0 + bs);
+        float m = sc[e0];
+        for (int e = e0 + 1; e < e1; ++e) m = fmaxf(m, sc[e]);
+        bm[b] = m;
+      }
+    };
     // every thread owns a contiguous, 4-aligned segment of the chunk's entries
     const int seg = ((nloc + kThreads - 1) / kThreads + 3) & ~3;
     const int i0 = min(nloc, tid * seg), i1 = min(nloc, i0 + seg);
 
     if (n <= k) {
       copy_scores();
+      if (a.bmax) write_block_max();
       __syncthreads();
       for (int i = tid; i < nloc; i += kThreads) {
         oi[base + i] = static_cast<int32_t>(base + i);
@@ -892,6 +908,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       // arrive, copy the scores while the request's slower CTAs finish, wait
       request_arrive(&bar[0]);
       copy_scores();
+      if (a.bmax) write_block_max();
       bool alive = request_wait(&bar[0], a.chunks, sh);
       uint32_t shift = 20, prefix = 0;
       if (alive) {
@@ -1175,7 +1192,8 @@ size_t index_tc_workspace_bytes(int batch, int64_t cap, int k) {
 // must be zero on entry (the caller zeroes them).
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
-                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap) {
+                                  float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap,
+                                  float* bmax, int64_t ldb, int block) {
   Launcher& L = launcher();
   if (!L.encode) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const bool fp8 = k_idx->dtype == kFP8;
@@ -1217,6 +1235,9 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.out_idx = out_idx;
   a.out_score = out_score;
   a.append = ap != nullptr;
+  a.bmax = bmax;
+  a.ldb = ldb;
+  a.block = block;
   if (ap) {
     a.ap = *ap;
     a.ap.shrink = kAppendShrink;

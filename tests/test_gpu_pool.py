@@ -97,18 +97,24 @@ EXACT = {
     "f32_b1": (Wk.WORKLOADS["tiny"].scaled(topk=40), 2, 2, 700, 1, 64),
     "bf16_b8": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 3, 3, 6000 + 3, 8, 96),
     "bf16_b128": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 2, 2, 9000, 128, 7),
+    "bf16_b32_many_chunks": (Wk.WORKLOADS["decode64k"].scaled(topk=256), 2, 2, 150000, 32, 300),
 }
 
 
+@pytest.mark.parametrize("per_request", [False, True])
 @pytest.mark.parametrize("name", list(EXACT))
-def test_pool_and_reindex_exact(name, cuda_lib):
+def test_pool_and_reindex_exact(name, per_request, cuda_lib):
+    """per_request: one query per request without q_req, the form that the
+    fused tensor-core indexer takes for bf16 / FP8 keys of 64 x 128."""
     wl, nq, B, cap, block, pool_blocks = EXACT[name]
+    if per_request and nq != B:
+        pytest.skip("needs one query per request")
     seed = 4200 + len(name)
     kidx, q_idx, w = integer_inputs(seed, wl, nq, B, cap, dup_blocks=(7, 11, 40), block=block)
     q_req = (np.arange(nq) % B).astype(np.int32)
     # full cache, a partial last block, fewer blocks than the pool holds
     n_vis = np.array([cap, cap - block // 2 - 1, min(cap, block * pool_blocks // 2 + 3)][:nq], np.int32)
-    gp, gi = gpu_pool(wl, q_idx, w, kidx, B, cap, q_req, n_vis, block, pool_blocks)
+    gp, gi = gpu_pool(wl, q_idx, w, kidx, B, cap, None if per_request else q_req, n_vis, block, pool_blocks)
     qd = O.decode_stored(q_idx)
     pools = []
     for i in range(nq):
