@@ -20,6 +20,14 @@ collective on the data path): weak scaling, max-over-ranks device time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle as the reference arm
+  python bench.py --path hier ...        # the hierarchical sparse indexer (hier1m)
+
+``--path hier`` times one Reindex layer of a decoder group at 1M tokens
+(ratio 1, FP8 indexer keys, top 512): the lightning indexer over the
+16,384-position candidate pool that the group's Full layer built (2,048
+blocks of 8), its top-512, and the pool-position -> entry mapping.  The Full
+layer (full scan + block maxima + pool) and a full scan with the Reindex
+layer's query are timed beside it.
 """
 from __future__ import annotations
 
@@ -50,6 +58,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode1m", choices=[k for k, v in Wk.WORKLOADS.items() if not v.is_prefill])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="step", choices=["step", "hier"])
     return ap.parse_args()
 
 
@@ -336,6 +345,144 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+def run_hier(args, rank, world, local_rank):
+    """The hierarchical sparse indexer: one Reindex layer over the Full
+    layer's candidate pool, on hier1m."""
+    import torch
+
+    from compressed_sparse_attention_compressor_b200 import csa
+    from compressed_sparse_attention_compressor_b200.csa import DevTensor
+
+    torch.cuda.set_device(local_rank)
+    base = Wk.WORKLOADS["hier1m"]
+    wl = base.scaled(seed=base.seed + 100 * rank)
+    block, pool_blocks = Wk.HIER_POOL
+    B, cap, s = wl.batch, wl.context // wl.m, wl.seed
+    sI = 1.0 / np.sqrt(wl.d_idx)
+    up = DevTensor.from_stored
+    kidx_st = Wk.store(Wk.normal(s, "kidx", (B, cap, wl.d_idx), sI), wl.idx_dtype, wl.idx_group)
+    qf_st = Wk.store(Wk.normal(s, "q_idx", (B, wl.h_idx, wl.d_idx), sI), wl.act_dtype)
+    qr_st = Wk.store(Wk.normal(s, "q_idx_reindex", (B, wl.h_idx, wl.d_idx), sI), wl.act_dtype)
+    wf_np, wr_np = Wk.uniform(s, "w", (B, wl.h_idx)), Wk.uniform(s, "w_reindex", (B, wl.h_idx))
+    kidx, q_full, q_re = up(kidx_st), up(qf_st), up(qr_st)
+    w_full, w_re = torch.from_numpy(wf_np).cuda(), torch.from_numpy(wr_np).cuda()
+    n_vis = torch.full((B,), cap, dtype=torch.int32, device="cuda")
+    p = csa.params(wl.m, wl.d, wl.d_idx, wl.h_q, wl.h_idx, wl.topk, wl.window, max(wl.window, 1), 1.0)
+    ws = csa.workspace(max(csa.csa_index_pool_workspace_size(p, B, cap, block, pool_blocks),
+                           csa.csa_workspace_size(p, B, cap)))
+    pool = torch.empty((B, pool_blocks), dtype=torch.int32, device="cuda")
+    idx_full = torch.empty((B, wl.topk), dtype=torch.int32, device="cuda")
+    idx_re = torch.empty((B, wl.topk), dtype=torch.int32, device="cuda")
+    idx_scan = torch.empty((B, wl.topk), dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    evict = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush.zero_()
+        evict.sum()
+        torch.cuda._sleep(200_000)
+
+    def full():
+        csa.csa_index_topk_pool(p, B, q_full, w_full, kidx, B, cap, None, n_vis, block, pool_blocks, pool, idx_full,
+                                None, ws, stream)
+
+    def reindex():
+        csa.csa_index_topk_reindex(p, B, q_re, w_re, kidx, B, cap, None, n_vis, pool, block, pool_blocks, idx_re,
+                                   None, ws, stream)
+
+    def scan():
+        csa.csa_index_topk(p, B, q_re, w_re, kidx, B, cap, None, n_vis, idx_scan, None, ws, stream)
+
+    def timed(fn, K):
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            flush_l2()
+            e0[i].record(stream)
+            fn()
+            e1[i].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in zip(e0, e1)]
+
+    full()
+    for _ in range(args.warmup):
+        for fn in (full, reindex, scan):
+            flush_l2()
+            fn()
+    torch.cuda.synchronize()
+    K = args.steps
+    with ClockSampler(local_rank) as clk:
+        re_ms = timed(reindex, K)
+    full_ms = timed(full, K)
+    scan_ms = timed(scan, K)
+    ms = float(sum(re_ms)) / K
+
+    csa.csa_profile_start(64 * K)
+    for _ in range(K):
+        flush_l2()
+        reindex()
+    torch.cuda.synchronize()
+    csa.csa_profile_stop()
+    per = {}
+    for name, t in csa.csa_profile_records():
+        c = per.setdefault(name, [0, 0.0])
+        c[0] += 1
+        c[1] += t
+    dom = max(per, key=lambda n: per[n][1])
+    dom_ms = per[dom][1] / per[dom][0]
+    P = block * pool_blocks
+    # the dominant launch: the pool scores on the CUDA cores (fp32 FMA issue bound)
+    flops = 2.0 * B * P * wl.h_idx * wl.d_idx
+    alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    achieved = flops / (dom_ms * 1e-3) / 1e12
+    res = {
+        "metric": "Reindex-layer selections/s (top-512 over a 16,384-candidate pool, 1M tokens)",
+        "value": B / (ms * 1e-3),
+        "unit": "queries/s",
+        "n_gpus": 1,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8",
+        "data": "synthetic (seeded Gaussian indexer keys and queries)",
+        "config": {"workload": wl.name, "batch": B, "context": wl.context, "m": wl.m, "entries": cap,
+                   "block": block, "pool_blocks": pool_blocks, "candidates": P, "topk": wl.topk,
+                   "indexer": f"{wl.h_idx}x{wl.d_idx}", "idx_dtype": wl.idx_dtype,
+                   "l2": "flushed between timed steps (256 MB write, then 256 MB read)"},
+        "full_layer_ms": float(sum(full_ms)) / K,
+        "full_scan_ms": float(sum(scan_ms)) / K,
+        "reindex_vs_full_scan": (float(sum(scan_ms)) / K) / ms,
+        "roofline": {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                     "frac": achieved / alu_peak, "traffic": None, "algorithmic_flops": flops, "avg_ms": dom_ms,
+                     "peak_source": "fp32 FMA issue: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"},
+        "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
+                    for n, (c, t) in per.items()},
+        "gpu_launches": sum(c for c, _ in per.values()),
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        # the oracle on request 0: its Full layer builds the pool (not timed),
+        # its Reindex layer is the sample
+        from oracle import csa_oracle as O
+
+        keys = O.decode(kidx_st.data[0], kidx_st.dtype, kidx_st.scale[0], kidx_st.group)
+        qf, qr = O.decode_stored(qf_st)[0], O.decode_stored(qr_st)[0]
+        opool = O.candidate_pool(O.index_scores(qf, wf_np[0], keys), block, pool_blocks)
+        n_s, t_s = 0, 0.0
+        while n_s < 3 or t_s < 5.0:
+            t0 = time.perf_counter()
+            O.reindex_topk(qr, wr_np[0], keys, opool, block, wl.topk)
+            t_s += time.perf_counter() - t0
+            n_s += 1
+        res["cpu_baseline"] = {"value": n_s / t_s, "unit": "queries/s", "cores": _threads(), "kind": "oracle",
+                               "sample": f"{n_s} Reindex-layer selections of request 0 ({t_s:.1f} s)"}
+    return res
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
@@ -413,6 +560,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if args.path == "hier":
+        if rank == 0:
+            print(json.dumps(run_hier(args, rank, world, local_rank)), flush=True)
+        return 0
     res = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, t = oracle_sample(args.workload)

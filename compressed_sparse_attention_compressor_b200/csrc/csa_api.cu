@@ -25,7 +25,10 @@ size_t index_tc_workspace_bytes(int batch, int64_t cap, int k);
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
                                   float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap = nullptr,
-                                  float* bmax = nullptr, int64_t ldb = 0, int block = 1);
+                                  float* bmax = nullptr, int64_t ldb = 0, int block = 1,
+                                  const int32_t* pool = nullptr, int pool_blocks = 0, int pblock = 0);
+bool index_tc_pool_supported(const csa_params_t* p, int batch, int64_t cap, int block, int pool_blocks, int q_dtype,
+                             int k_dtype);
 uint32_t index_tc_take_error();
 uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
@@ -308,7 +311,11 @@ size_t csa_index_pool_workspace_size(const csa_params_t* p, int32_t n_queries, i
                                      int32_t pool_blocks) {
   if (p == nullptr || n_queries < 0 || max_entries < 0 || block < 1 || pool_blocks < 1) return 0;
   const size_t a = pool_ws_bytes(p, n_queries, max_entries, block);
-  const size_t b = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk > 0 ? p->topk : 1);
+  size_t b = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk > 0 ? p->topk : 1);
+  if (p->topk >= 1 && p->h_idx > 0 && p->d_idx > 0) {
+    const size_t t = index_tc_workspace_bytes(n_queries, static_cast<int64_t>(block) * pool_blocks, p->topk);
+    if (t > b) b = t;
+  }
   return (a > b ? a : b) + 256;
 }
 
@@ -367,10 +374,21 @@ csa_status_t csa_index_topk_reindex(const csa_params_t* p, int32_t n_queries, co
   if (p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "csa_index_topk_reindex needs topk >= 1");
   if (n_queries == 0) return CSA_OK;
   if (pool == nullptr || out_idx == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null pool / out_idx");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (q_req == nullptr && n_queries == batch &&
+      index_tc_pool_supported(p, batch, cap, block, pool_blocks, q_idx->dtype, k_idx->dtype)) {
+    // one query per request: the fused tensor-core indexer over the pool
+    const size_t need = index_tc_workspace_bytes(batch, static_cast<int64_t>(block) * pool_blocks, p->topk);
+    if (workspace == nullptr || workspace_bytes < need)
+      return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, index_tc_control_bytes(batch), s);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    return launch_index_topk_tc(p, batch, q_idx, w, k_idx, cap, n_visible, out_idx, out_score, workspace, s, nullptr,
+                                nullptr, 0, 1, pool, pool_blocks, block);
+  }
   const size_t need = reindex_ws_bytes(n_queries, block, pool_blocks, p->topk);
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Carver c(workspace);
   const int64_t np = static_cast<int64_t>(block) * pool_blocks, ld = round_up(np, 4);
   float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);

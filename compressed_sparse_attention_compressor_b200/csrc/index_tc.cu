@@ -132,6 +132,12 @@ struct IdxArgs {
   float* bmax;             // optional [batch][ldb]: max score of each block of `block` entries
   int64_t ldb;
   int block;               // power of two <= kTileM, so no block straddles two chunks
+  // candidate-pool mode: position j of request r is entry
+  // pool[r][j / pblock] * pblock + j % pblock; the keys come in pblock-row boxes
+  const int32_t* pool;     // [batch][pool_blocks] ascending block ids, -1 padded (or null)
+  int pool_blocks;
+  int pblock;              // 8 .. 128, a power of two
+  const float* kscale;     // FP8 row scales [batch][cap] (pool mode)
 };
 
 struct Shared {
@@ -140,7 +146,44 @@ struct Shared {
   uint32_t qmax[kThreads / 32];
   float qinv;
   int fail;
+  int red[kThreads / 32];
 };
+
+// Candidate-pool mode: the positions of request r that hold visible
+// entries.  The pool's valid slots (block id >= 0, block start < n_vis) form
+// its leading run when the pool ascends with -1 padding at the end; the run
+// ends at the first other slot, and the positions are the entries of the
+// run's blocks, the last of which may be partial.  Called by every thread.
+__device__ int64_t pool_positions(const IdxArgs& a, int r, Shared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* prow = a.pool + static_cast<int64_t>(r) * a.pool_blocks;
+  const int64_t nv = min(max(static_cast<int64_t>(a.n_visible[r]), int64_t(0)), a.cap);
+  const int bs = a.pblock;
+  int first_bad = a.pool_blocks;
+  for (int q = tid; q < a.pool_blocks; q += kThreads) {
+    const int32_t b = __ldg(prow + q);
+    if (b < 0 || static_cast<int64_t>(b) * bs >= nv) {
+      first_bad = q;
+      break;
+    }
+  }
+  first_bad = static_cast<int>(__reduce_min_sync(0xFFFFFFFFu, static_cast<uint32_t>(first_bad)));
+  if (lane == 0) sh.red[warp] = first_bad;
+  __syncthreads();
+  int end = a.pool_blocks;
+  for (int w2 = 0; w2 < kThreads / 32; ++w2) end = min(end, sh.red[w2]);
+  __syncthreads();
+  uint32_t cnt = 0;
+  for (int q = tid; q < end; q += kThreads)
+    cnt += static_cast<uint32_t>(min(static_cast<int64_t>(bs), nv - static_cast<int64_t>(__ldg(prow + q)) * bs));
+  cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+  if (lane == 0) sh.red[warp] = static_cast<int>(cnt);
+  __syncthreads();
+  int64_t np = 0;
+  for (int w2 = 0; w2 < kThreads / 32; ++w2) np += sh.red[w2];
+  __syncthreads();
+  return np;
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -530,8 +573,15 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x / a.chunks, c = blockIdx.x % a.chunks;
-  const int64_t n_raw = a.append ? (a.ap.pos[r] + 1) / a.ap.m : static_cast<int64_t>(a.n_visible[r]);
-  const int64_t n = min(max(n_raw, int64_t(0)), a.cap);
+  const int64_t n_raw = a.pool ? pool_positions(a, r, sh)
+                               : a.append ? (a.ap.pos[r] + 1) / a.ap.m : static_cast<int64_t>(a.n_visible[r]);
+  const int64_t n = min(max(n_raw, int64_t(0)), a.pool ? static_cast<int64_t>(a.pool_blocks) * a.pblock : a.cap);
+  const int32_t* prow = a.pool ? a.pool + static_cast<int64_t>(r) * a.pool_blocks : nullptr;
+  // pool position -> entry id (identity without a pool)
+  auto entry_of = [&](uint32_t j) -> int32_t {
+    if (!prow) return static_cast<int32_t>(j);
+    return __ldg(prow + j / a.pblock) * a.pblock + static_cast<int32_t>(j % a.pblock);
+  };
   const int tiles_req = static_cast<int>((n + kTileM - 1) / kTileM);
   int t0, t1;
   if (a.append && a.chunks > 1) {
@@ -573,7 +623,75 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     append_block(a.ap, r, a.cap, smem + C::oStages, reinterpret_cast<float*>(smem + C::oHist), abar, sh);
 
   // ================= phase 1: stream the keys, scores into TMEM =================
-  if (warp == 0) {
+  if (warp == 0 && prow) {
+    // candidate-pool mode: per stage, lane l loads the pblock-row box of
+    // slot q0 + l (and, FP8, its row scales); a stage's slots are <= 32
+    if (lane == 0) {
+      mbar_arrive_expect_tx(qbar, kHeads * kDI * 2);
+      bulk_load(smem + C::oQ, a.q_idx + static_cast<int64_t>(r) * kHeads * kDI, kHeads * kDI * 2, qbar);
+    }
+    const int bs = a.pblock, spt = kTileM / bs, sps = C::kTPS * spt;
+    const int nst = (nt + C::kTPS - 1) / C::kTPS;
+    const int64_t end_slot = (n + bs - 1) / bs;  // slots that hold positions
+    const uint64_t l2_stream = l2_policy_evict_first();
+    int issued = 0, sissued = 0;
+    for (int p = 0; p < nst; ++p) {
+      if (__shfl_sync(0xFFFFFFFFu, sh.fail, 0)) break;
+      const int s = p % C::kStages;
+      const int t = p * C::kTPS;
+      const int64_t q0 = static_cast<int64_t>(t0 + t) * kTileM / bs;
+      // slots past the run re-read the first block: those positions are >= n
+      int32_t b = 0;
+      if (lane < sps) b = __ldg(prow + (q0 + lane < end_slot ? q0 + lane : 0));
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty[s], ((p / C::kStages) & 1) ^ 1, kWaitLimit);
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+        if (lane == 0) {
+          atomicOr(&g_index_tc_error, 1u);
+          sh.fail = 1;
+        }
+        break;
+      }
+      uint8_t* dst = smem + C::oStages + s * C::kStageBytes;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+      __syncwarp();
+      if (lane < sps) {
+        const int y = static_cast<int>(r * a.cap + static_cast<int64_t>(b) * bs);
+        tma_load_2d_hint(dst + lane * bs * 128, &kmap, &full[s], 0, y, l2_stream);
+        if constexpr (!FP8) tma_load_2d_hint(dst + 16384 + lane * bs * 128, &kmap, &full[s], 64, y, l2_stream);
+      }
+      issued = p + 1;
+      if constexpr (FP8) {
+        bool sfail = false;
+        for (int j = 0; j < C::kTPS && t + j < nt; ++j) {
+          const int u = t + j, ss = u % kSStages;
+          bool sok = true;
+          if (lane == 0) sok = mbar_wait(&sempty[ss], ((u / kSStages) & 1) ^ 1, kWaitLimit);
+          if (!__shfl_sync(0xFFFFFFFFu, sok, 0)) {
+            if (lane == 0) {
+              atomicOr(&g_index_tc_error, 1u);
+              sh.fail = 1;
+            }
+            sfail = true;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&sfull[ss], kTileM * 4);
+          __syncwarp();
+          if (lane >= j * spt && lane < (j + 1) * spt)
+            bulk_load(smem + C::oScales + ss * kTileM * 4 + (lane - j * spt) * bs * 4,
+                      a.kscale + r * a.cap + static_cast<int64_t>(b) * bs, bs * 4, &sfull[ss]);
+          sissued = u + 1;
+        }
+        if (sfail) break;
+      }
+    }
+    if (lane == 0 && sh.fail) {  // let the copies still in flight land before the CTA winds down
+      for (int p = max(0, issued - C::kStages); p < issued; ++p)
+        mbar_wait(&full[p % C::kStages], (p / C::kStages) & 1, kWaitLimit);
+      for (int u = max(0, sissued - kSStages); u < sissued; ++u)
+        mbar_wait(&sfull[u % kSStages], (u / kSStages) & 1, kWaitLimit);
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // the query first, so that it is not queued behind the key stream
       mbar_arrive_expect_tx(qbar, kHeads * kDI * 2);
@@ -845,7 +963,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     uint2* ecache = reinterpret_cast<uint2*>(p2 + C::pEq);
     auto put = [&](uint32_t pos, uint2 e) {
       if (pos < static_cast<uint32_t>(k)) {
-        oi[pos] = static_cast<int32_t>(e.x);
+        oi[pos] = entry_of(e.x);
         if (os) os[pos] = __uint_as_float(e.y);
       }
     };
@@ -886,7 +1004,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       if (a.bmax) write_block_max();
       __syncthreads();
       for (int i = tid; i < nloc; i += kThreads) {
-        oi[base + i] = static_cast<int32_t>(base + i);
+        oi[base + i] = entry_of(static_cast<uint32_t>(base + i));
         if (os) os[base + i] = sc[i];
       }
       if (c == 0)
@@ -1169,6 +1287,23 @@ bool index_tc_supported(const csa_params_t* p, int batch, int64_t cap, int q_dty
   return ch <= kMaxChunks && per <= kMaxChunkTiles && p->topk >= 1;
 }
 
+// Candidate-pool mode (a Reindex layer): positions are the pool's entries,
+// loaded as `block`-row boxes of whole 1 KB swizzle atoms (block >= 8).
+bool index_tc_pool_supported(const csa_params_t* p, int batch, int64_t cap, int block, int pool_blocks, int q_dtype,
+                             int k_dtype) {
+  if (block < 8 || block > kTileM || (block & (block - 1)) != 0) return false;
+  if (p->h_idx != kHeads || p->d_idx != kDI || q_dtype != kBF16) return false;
+  if (k_dtype != kFP8 && k_dtype != kBF16) return false;
+  // FP8: whole blocks of row scales, so that no block's scales run past the tensor
+  if (k_dtype == kFP8 && cap % block != 0) return false;
+  if (batch < 1 || batch > (launcher().sms > 0 ? launcher().sms : 148)) return false;
+  if (static_cast<int64_t>(batch) * cap >= (int64_t(1) << 31)) return false;
+  const int64_t np = static_cast<int64_t>(block) * pool_blocks;
+  const int ch = index_tc_chunks(batch, np);
+  const int64_t tiles = (np + kTileM - 1) / kTileM;
+  return ch <= kMaxChunks && (tiles + ch - 1) / ch <= kMaxChunkTiles && p->topk >= 1;
+}
+
 // The decode step can append inside the indexer: W_IK (d x 128) fits the
 // idle stage ring and the pooled row the shared scratch.
 bool index_tc_append_supported(const csa_params_t* p, int w_dtype) {
@@ -1193,16 +1328,21 @@ size_t index_tc_workspace_bytes(int batch, int64_t cap, int k) {
 csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_tensor_t* q_idx, const float* w,
                                   const csa_tensor_t* k_idx, int64_t cap, const int32_t* n_visible, int32_t* out_idx,
                                   float* out_score, void* ws, cudaStream_t stream, const AppendArgs* ap,
-                                  float* bmax, int64_t ldb, int block) {
+                                  float* bmax, int64_t ldb, int block, const int32_t* pool,
+                                  int pool_blocks, int pblock) {
   Launcher& L = launcher();
   if (!L.encode) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const bool fp8 = k_idx->dtype == kFP8;
-  const int ch = index_tc_chunks(batch, cap);
+  // pool mode chunks the pool's positions, not the cache
+  const int64_t npos = pool ? static_cast<int64_t>(pool_blocks) * pblock : cap;
+  const int ch = index_tc_chunks(batch, npos);
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDI), static_cast<cuuint64_t>(batch) * cap};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDI) * (fp8 ? 1 : 2)};
-  // FP8: one 256-row box = two key tiles per stage; bf16: two 64-column boxes per tile
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), static_cast<cuuint32_t>(fp8 ? 2 * kTileM : kTileM)};
+  // FP8: one 256-row box = two key tiles per stage; bf16: two 64-column boxes
+  // per tile; pool mode: one box per pool block
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(fp8 ? 128 : 64),
+                             static_cast<cuuint32_t>(pool ? pblock : fp8 ? 2 * kTileM : kTileM)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult cr = L.encode(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                          k_idx->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1238,6 +1378,10 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.bmax = bmax;
   a.ldb = ldb;
   a.block = block;
+  a.pool = pool;
+  a.pool_blocks = pool_blocks;
+  a.pblock = pblock;
+  a.kscale = fp8 ? k_idx->scale : nullptr;
   if (ap) {
     a.ap = *ap;
     a.ap.shrink = kAppendShrink;

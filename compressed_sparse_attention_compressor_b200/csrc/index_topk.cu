@@ -171,9 +171,16 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
     const int sh_ = shifts[pass];
     for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
     __syncthreads();
-    for (int64_t j = tid; j < n; j += kTopkThreads) {
-      const uint32_t key = score_key(s[j]);
-      if ((key & pmask) == prefix) atomicAdd(&sh.hist[(key >> sh_) & (nb - 1)], 1u);
+    // scores crowd into few bins: one atomic per distinct bin and warp
+    for (int64_t j0 = 0; j0 < n; j0 += kTopkThreads) {
+      const int64_t j = j0 + tid;
+      uint32_t bin = 0xFFFFFFFFu;
+      if (j < n) {
+        const uint32_t key = score_key(s[j]);
+        if ((key & pmask) == prefix) bin = (key >> sh_) & (nb - 1);
+      }
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (bin != 0xFFFFFFFFu && __ffs(peers) - 1 == lane) atomicAdd(&sh.hist[bin], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) find_bin(sh, nb, need);
@@ -187,63 +194,43 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
   const uint32_t take_eq = need;    // entries equal to T that are kept
   const uint32_t n_gt = static_cast<uint32_t>(k) - take_eq;
 
-  // index-ordered selection
-  uint32_t base_gt = 0, base_eq = 0;
-  for (int64_t j0 = 0; j0 < n; j0 += kTopkThreads) {
-    const int64_t j = j0 + tid;
-    float v = 0.f;
-    uint32_t key = 0;
-    if (j < n) { v = s[j]; key = score_key(v); }
-    const bool gt = j < n && key > T;
-    const bool eq = j < n && key == T;
-    const uint32_t bgt = __ballot_sync(0xFFFFFFFFu, gt), beq = __ballot_sync(0xFFFFFFFFu, eq);
-    if (lane == 0) { sh.warp_gt[warp] = __popc(bgt); sh.warp_eq[warp] = __popc(beq); }
-    __syncthreads();
-    uint32_t off_gt = 0, off_eq = 0, tot_gt = 0, tot_eq = 0;
-    for (int w2 = 0; w2 < kTopkWarps; ++w2) {
-      const uint32_t a = sh.warp_gt[w2], b = sh.warp_eq[w2];
-      if (w2 < warp) { off_gt += a; off_eq += b; }
-      tot_gt += a; tot_eq += b;
-    }
-    const uint32_t lm = (1u << lane) - 1u;
-    if (ordered) {
-      // the selection in ascending index order: entries above T, and the
-      // first take_eq equal to T
-      const bool sel = gt || (eq && base_eq + off_eq + __popc(beq & lm) < take_eq);
-      const uint32_t bsel = __ballot_sync(0xFFFFFFFFu, sel);
-      __syncthreads();
-      if (lane == 0) sh.warp_gt[warp] = __popc(bsel);
-      __syncthreads();
-      uint32_t off_s = 0, tot_s = 0;
-      for (int w2 = 0; w2 < kTopkWarps; ++w2) {
-        if (w2 < warp) off_s += sh.warp_gt[w2];
-        tot_s += sh.warp_gt[w2];
-      }
-      if (sel) {
-        const uint32_t p = base_gt + off_s + __popc(bsel & lm);
+  // selection: every thread owns a contiguous segment; a block scan of the
+  // per-segment counts gives each entry its output slot
+  const int64_t seg = (n + kTopkThreads - 1) / kTopkThreads;
+  const int64_t a0 = min(n, tid * seg), a1 = min(n, a0 + seg);
+  uint32_t cg = 0, ce = 0;
+  for (int64_t j = a0; j < a1; ++j) {
+    const uint32_t key = score_key(s[j]);
+    cg += key > T;
+    ce += key == T;
+  }
+  uint32_t ig = cg, ie = ce;  // inclusive scans within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t vg = __shfl_up_sync(0xFFFFFFFFu, ig, o), ve = __shfl_up_sync(0xFFFFFFFFu, ie, o);
+    if (lane >= o) { ig += vg; ie += ve; }
+  }
+  if (lane == 31) { sh.warp_gt[warp] = ig; sh.warp_eq[warp] = ie; }
+  __syncthreads();
+  uint32_t og = ig - cg, oe = ie - ce;  // entries above / at T before this segment
+  for (int w2 = 0; w2 < warp; ++w2) { og += sh.warp_gt[w2]; oe += sh.warp_eq[w2]; }
+  for (int64_t j = a0; j < a1; ++j) {
+    const float v = s[j];
+    const uint32_t key = score_key(v);
+    if (key > T) {
+      // ordered: the kept entries before j are og above T and min(oe, take_eq) at T
+      const uint32_t p = ordered ? og + min(oe, take_eq) : og;
+      oi[p] = static_cast<int32_t>(j);
+      if (os) os[p] = v;
+      ++og;
+    } else if (key == T) {
+      if (oe < take_eq) {
+        const uint32_t p = ordered ? og + oe : n_gt + oe;
         oi[p] = static_cast<int32_t>(j);
         if (os) os[p] = v;
       }
-      base_gt += tot_s;
-      base_eq += tot_eq;
-      __syncthreads();
-      continue;
+      ++oe;
     }
-    if (gt) {
-      const uint32_t p = base_gt + off_gt + __popc(bgt & lm);
-      oi[p] = static_cast<int32_t>(j);
-      if (os) os[p] = v;
-    }
-    if (eq) {
-      const uint32_t r = base_eq + off_eq + __popc(beq & lm);
-      if (r < take_eq) {
-        oi[n_gt + r] = static_cast<int32_t>(j);
-        if (os) os[n_gt + r] = v;
-      }
-    }
-    base_gt += tot_gt;
-    base_eq += tot_eq;
-    __syncthreads();
   }
 }
 

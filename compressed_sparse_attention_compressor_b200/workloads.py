@@ -195,7 +195,14 @@ WORKLOADS: dict[str, Workload] = {
                            "normal", seed=1006),
     "hybrid_ratio1": Workload("hybrid_ratio1", 8, 262144, 1, 512, 64, 64, 128, 2048, 128, "bf16", "bf16",
                               "bf16", "normal", seed=1007),
+    # a decoder group of the hierarchical indexer: ratio 1 at 1M tokens, top
+    # 512, a pool of 2,048 blocks of 8 positions
+    "hier1m": Workload("hier1m", 4, 1048576, 1, 512, 64, 64, 128, 512, 128, "fp8", "fp8", "bf16", "normal",
+                       seed=1008),
 }
+
+# candidate pool of the hierarchical indexer: (block, pool_blocks)
+HIER_POOL = (8, 2048)
 
 
 # --------------------------------------------------------------------------

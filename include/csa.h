@@ -213,13 +213,15 @@ csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const
  * whole context).
  * Pool position j of query i (j < pool_blocks * block) is entry
  * e = pool[i][j / block] * block + j % block; it is a candidate when
- * pool[i][j / block] >= 0 and e < n_visible[i].  out_idx[i] receives the
+ * pool[i][j / block] >= 0 and e < n_visible[i].  The pool must be in the
+ * form csa_index_topk_pool writes: block ids ascending, then -1 padding
+ * (for other pools the selection is unspecified, though every index written
+ * is -1 or a visible entry).  out_idx[i] receives the
  * min(topk, candidates) candidates with the largest s_e (computed as in
  * csa_index_topk, from this call's q_idx and w) as ENTRY ids -- larger
  * score first in value, the earlier pool position first among exactly equal
- * scores (the lower entry when the pool is ascending, as csa_index_topk_pool
- * writes it).  The order inside out_idx[i] is unspecified; unused slots hold
- * -1 (out_score -inf).
+ * scores, which is the lower entry.  The order inside out_idx[i] is
+ * unspecified; unused slots hold -1 (out_score -inf).
  *   pool         [n_queries][pool_blocks] int32 block ids (-1 = empty slot).
  *   out_idx      [n_queries][p->topk] int32; out_score optional fp32.
  *   workspace    csa_index_pool_workspace_size(...) bytes.

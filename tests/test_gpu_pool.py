@@ -126,7 +126,7 @@ def test_pool_and_reindex_exact(name, per_request, cuda_lib):
     # a Reindex layer: its own query and weights over the oracle's pool
     _, q2, w2 = integer_inputs(seed + 1, wl, nq, B, cap, (), block)
     pool = np.stack(pools).astype(np.int32)
-    ri, rs = gpu_reindex(wl, q2, w2, kidx, B, cap, q_req, n_vis, pool, block)
+    ri, rs = gpu_reindex(wl, q2, w2, kidx, B, cap, None if per_request else q_req, n_vis, pool, block)
     q2d = O.decode_stored(q2)
     for i in range(nq):
         check_reindex_row(ri[i], rs[i], pool[i], block, keys_of(kidx, q_req[i], n_vis[i]), q2d[i], w2[i], wl.topk,
@@ -137,15 +137,20 @@ def test_pool_and_reindex_exact(name, per_request, cuda_lib):
 # seeded normal inputs in the workloads' precisions
 # ---------------------------------------------------------------------------
 CASES = {
-    "fp8": (Wk.WORKLOADS["decode1m"], 3, 3, 40000 + 5, 8, 512),
+    "fp8": (Wk.WORKLOADS["decode1m"], 3, 3, 40000 + 8, 8, 512),
+    "fp8_ragged_cap": (Wk.WORKLOADS["decode1m"], 3, 3, 40000 + 4, 8, 512),
+    "fp8_b16": (Wk.WORKLOADS["decode1m"], 2, 2, 60000, 16, 300),
     "bf16": (Wk.WORKLOADS["decode64k"], 2, 2, 20000, 8, 256),
     "f32": (Wk.WORKLOADS["tiny"], 2, 1, 3000, 16, 40),
 }
 
 
+@pytest.mark.parametrize("per_request", [False, True])
 @pytest.mark.parametrize("name", list(CASES))
-def test_pool_and_reindex_match_oracle(name, cuda_lib):
+def test_pool_and_reindex_match_oracle(name, per_request, cuda_lib):
     wl, nq, B, cap, block, pool_blocks = CASES[name]
+    if per_request and nq != B:
+        pytest.skip("needs one query per request")
     seed = 4300 + len(name)
     sI = 1 / np.sqrt(wl.d_idx)
     kidx = Wk.store(Wk.normal(seed, "kidx", (B, cap, wl.d_idx), sI), wl.idx_dtype, wl.d_idx)
@@ -153,7 +158,7 @@ def test_pool_and_reindex_match_oracle(name, cuda_lib):
     w = Wk.uniform(seed, "w", (nq, wl.h_idx))
     q_req = (np.arange(nq) % B).astype(np.int32)
     n_vis = np.array([cap, cap - 3, block * pool_blocks // 3 + 1][:nq], np.int32)
-    gp, gi = gpu_pool(wl, q_idx, w, kidx, B, cap, q_req, n_vis, block, pool_blocks)
+    gp, gi = gpu_pool(wl, q_idx, w, kidx, B, cap, None if per_request else q_req, n_vis, block, pool_blocks)
     exact = wl.idx_dtype == "f32"
     qd = O.decode_stored(q_idx)
     swaps = 0
@@ -174,7 +179,7 @@ def test_pool_and_reindex_match_oracle(name, cuda_lib):
         # the last (possibly partial) block is always in the pool
         ch = np.sort(g.choice(nb - 1, size=take - 1, replace=False)) if take > 1 else np.zeros(0, np.int64)
         pool[i, :take] = np.append(ch, nb - 1)
-    ri, rs = gpu_reindex(wl, q2, w2, kidx, B, cap, q_req, n_vis, pool, block)
+    ri, rs = gpu_reindex(wl, q2, w2, kidx, B, cap, None if per_request else q_req, n_vis, pool, block)
     q2d = O.decode_stored(q2)
     for i in range(nq):
         swaps += check_reindex_row(ri[i], rs[i], pool[i], block, keys_of(kidx, q_req[i], n_vis[i]), q2d[i], w2[i],
