@@ -102,6 +102,7 @@ index_score_simt_kernel(const void* __restrict__ q_idx, int q_dtype, const float
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kU = 4;  // 16-byte loads in flight per thread
 
 struct TopkShared {
   uint32_t hist[2048];
@@ -141,6 +142,23 @@ __device__ void find_bin(TopkShared& sh, int nb, uint32_t need) {
   }
 }
 
+// Four consecutive scores of a row (zero past n), as one 16-byte load when
+// the row start allows it: each thread keeps several loads in flight.
+struct Row4 {
+  const float* s;
+  int64_t n;
+  bool vec;
+  __device__ __forceinline__ void load(int64_t j, float (&v)[4]) const {  // j % 4 == 0
+    if (vec && j + 3 < n) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(s + j));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[c] = j + c < n ? __ldg(s + j + c) : 0.f;
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kTopkThreads)
 topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
                 int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int nv_div, int ordered) {
@@ -162,74 +180,140 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
     return;
   }
 
-  // radix select of the k-th largest key
-  uint32_t prefix = 0, pmask = 0, need = static_cast<uint32_t>(k);
-  const int shifts[3] = {21, 10, 0};
-  const int bits[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int nb = 1 << bits[pass];
-    const int sh_ = shifts[pass];
-    for (int i = tid; i < nb; i += kTopkThreads) sh.hist[i] = 0;
+  const Row4 rs4{s, n, (reinterpret_cast<uintptr_t>(s) & 15) == 0};
+  // radix select of the k-th largest key over the keys' own range: the
+  // range [lo, lo + span) is cut into <= 2048 bins of 2^shift keys and
+  // narrowed to the bin holding the k-th key until a bin is one key wide.
+  // Bins that follow the data keep shared-memory atomics on distinct words.
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int64_t j0 = 0; j0 < n; j0 += kU * 4 * kTopkThreads) {
+    float v[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) rs4.load(j0 + 4 * (u * kTopkThreads + tid), v[u]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (j0 + 4 * (u * kTopkThreads + tid) + c < n) {
+          const uint32_t key = score_key(v[u][c]);
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+  }
+  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+  if (lane == 0) { sh.warp_gt[warp] = kmin; sh.warp_eq[warp] = kmax; }
+  __syncthreads();
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int w2 = 0; w2 < kTopkWarps; ++w2) { lo = min(lo, sh.warp_gt[w2]); hi = max(hi, sh.warp_eq[w2]); }
+  __syncthreads();
+  uint64_t span = static_cast<uint64_t>(hi - lo) + 1;
+  uint32_t need = static_cast<uint32_t>(k);
+  int shift = max(0, 64 - __clzll(static_cast<long long>(span - 1)) - 11);
+  for (;;) {
+    for (int i = tid; i < 2048; i += kTopkThreads) sh.hist[i] = 0;
     __syncthreads();
-    // scores crowd into few bins: one atomic per distinct bin and warp
-    for (int64_t j0 = 0; j0 < n; j0 += kTopkThreads) {
-      const int64_t j = j0 + tid;
-      uint32_t bin = 0xFFFFFFFFu;
-      if (j < n) {
-        const uint32_t key = score_key(s[j]);
-        if ((key & pmask) == prefix) bin = (key >> sh_) & (nb - 1);
-      }
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-      if (bin != 0xFFFFFFFFu && __ffs(peers) - 1 == lane) atomicAdd(&sh.hist[bin], __popc(peers));
+    for (int64_t j0 = 0; j0 < n; j0 += kU * 4 * kTopkThreads) {
+      float v[kU][4];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) rs4.load(j0 + 4 * (u * kTopkThreads + tid), v[u]);
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t d = score_key(v[u][c]) - lo;
+          if (j0 + 4 * (u * kTopkThreads + tid) + c < n && static_cast<uint64_t>(d) < span)
+            atomicAdd(&sh.hist[d >> shift], 1u);
+        }
     }
     __syncthreads();
-    if (warp == 0) find_bin(sh, nb, need);
+    if (warp == 0) find_bin(sh, 2048, need);
     __syncthreads();
-    prefix |= sh.sel_bin << sh_;
-    pmask |= static_cast<uint32_t>(nb - 1) << sh_;
+    const uint32_t b = sh.sel_bin;
     need -= sh.above;
+    lo += b << shift;
+    span = min(span - (static_cast<uint64_t>(b) << shift), static_cast<uint64_t>(1) << shift);
     __syncthreads();
+    if (shift == 0) break;
+    shift = max(0, shift - 11);
   }
+  const uint32_t prefix = lo;
   const uint32_t T = prefix;        // exact key of the k-th largest score
   const uint32_t take_eq = need;    // entries equal to T that are kept
   const uint32_t n_gt = static_cast<uint32_t>(k) - take_eq;
 
-  // selection: every thread owns a contiguous segment; a block scan of the
-  // per-segment counts gives each entry its output slot
-  const int64_t seg = (n + kTopkThreads - 1) / kTopkThreads;
-  const int64_t a0 = min(n, tid * seg), a1 = min(n, a0 + seg);
+  // selection: every warp owns a contiguous segment that it walks 128
+  // entries (four per lane) at a time; a scan over the lanes ranks the
+  // entries inside the warp and one scan of the per-warp counts gives every
+  // entry its output slot
+  const int64_t segw = ((n + kTopkWarps - 1) / kTopkWarps + 127) & ~int64_t(127);
+  const int64_t a0 = min(n, warp * segw), a1 = min(n, a0 + segw);
   uint32_t cg = 0, ce = 0;
-  for (int64_t j = a0; j < a1; ++j) {
-    const uint32_t key = score_key(s[j]);
-    cg += key > T;
-    ce += key == T;
-  }
-  uint32_t ig = cg, ie = ce;  // inclusive scans within the warp
+  for (int64_t j1 = a0; j1 < a1; j1 += kU * 128) {
+    float v[kU][4];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t vg = __shfl_up_sync(0xFFFFFFFFu, ig, o), ve = __shfl_up_sync(0xFFFFFFFFu, ie, o);
-    if (lane >= o) { ig += vg; ie += ve; }
-  }
-  if (lane == 31) { sh.warp_gt[warp] = ig; sh.warp_eq[warp] = ie; }
-  __syncthreads();
-  uint32_t og = ig - cg, oe = ie - ce;  // entries above / at T before this segment
-  for (int w2 = 0; w2 < warp; ++w2) { og += sh.warp_gt[w2]; oe += sh.warp_eq[w2]; }
-  for (int64_t j = a0; j < a1; ++j) {
-    const float v = s[j];
-    const uint32_t key = score_key(v);
-    if (key > T) {
-      // ordered: the kept entries before j are og above T and min(oe, take_eq) at T
-      const uint32_t p = ordered ? og + min(oe, take_eq) : og;
-      oi[p] = static_cast<int32_t>(j);
-      if (os) os[p] = v;
-      ++og;
-    } else if (key == T) {
-      if (oe < take_eq) {
-        const uint32_t p = ordered ? og + oe : n_gt + oe;
-        oi[p] = static_cast<int32_t>(j);
-        if (os) os[p] = v;
+    for (int u = 0; u < kU; ++u) rs4.load(j1 + u * 128 + 4 * lane, v[u]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const bool ok = j1 + u * 128 + 4 * lane + c < a1;
+        const uint32_t key = score_key(v[u][c]);
+        cg += ok && key > T;
+        ce += ok && key == T;
       }
-      ++oe;
+  }
+  cg = __reduce_add_sync(0xFFFFFFFFu, cg);
+  ce = __reduce_add_sync(0xFFFFFFFFu, ce);
+  if (lane == 0) { sh.warp_gt[warp] = cg; sh.warp_eq[warp] = ce; }
+  __syncthreads();
+  uint32_t og = 0, oe = 0;  // entries above / at T before the current step
+  for (int w2 = 0; w2 < warp; ++w2) { og += sh.warp_gt[w2]; oe += sh.warp_eq[w2]; }
+  for (int64_t j1 = a0; j1 < a1; j1 += kU * 128) {
+    float vv[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) rs4.load(j1 + u * 128 + 4 * lane, vv[u]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t j0 = j1 + u * 128;
+      if (j0 >= a1) break;
+      const float* v = vv[u];
+      uint32_t key[4], lg = 0, le = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const bool ok = j0 + 4 * lane + c < a1;
+        key[c] = score_key(v[c]);
+        lg += ok && key[c] > T;
+        le += ok && key[c] == T;
+      }
+      uint32_t ig = lg, ie = le;  // inclusive scans over the lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t vg = __shfl_up_sync(0xFFFFFFFFu, ig, o), ve = __shfl_up_sync(0xFFFFFFFFu, ie, o);
+        if (lane >= o) { ig += vg; ie += ve; }
+      }
+      uint32_t g = og + ig - lg, e = oe + ie - le;  // before this lane's first entry
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int64_t j = j0 + 4 * lane + c;
+        if (j >= a1) break;
+        if (key[c] > T) {
+          // ordered: the kept entries before j are g above T and min(e, take_eq) at T
+          const uint32_t p = ordered ? g + min(e, take_eq) : g;
+          oi[p] = static_cast<int32_t>(j);
+          if (os) os[p] = v[c];
+          ++g;
+        } else if (key[c] == T) {
+          if (e < take_eq) {
+            const uint32_t p = ordered ? g + e : n_gt + e;
+            oi[p] = static_cast<int32_t>(j);
+            if (os) os[p] = v[c];
+          }
+          ++e;
+        }
+      }
+      og += __shfl_sync(0xFFFFFFFFu, ig, 31);
+      oe += __shfl_sync(0xFFFFFFFFu, ie, 31);
     }
   }
 }

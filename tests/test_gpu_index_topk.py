@@ -11,14 +11,16 @@ from tests._harness import check_selection, gpu_index_topk, i32
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("k,n_cols", [(1, 10), (64, 1000), (512, 20000), (1024, 100000), (7, 5)])
-def test_topk_alone_is_bit_exact_with_ties(k, n_cols, cuda_lib):
+@pytest.mark.parametrize("k,n_cols,pad", [(1, 10, 5), (64, 1000, 5), (512, 20000, 5), (1024, 100000, 5), (7, 5, 5),
+                                         (1024, 100000, 4), (2048, 131072, 0), (33, 5003, 1)])
+def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, cuda_lib):
     """Same fp32 scores on both sides: selection must match exactly,
-    including planted exact ties, -0 vs +0, and rows with n_valid <= k."""
+    including planted exact ties, -0 vs +0, and rows with n_valid <= k.
+    pad: row stride - n_cols (a multiple of 4 gives 16-byte aligned rows)."""
     rows = 6
     s = Wk.make_scores(3000 + k, rows, n_cols)
     n_valid = np.array([n_cols, n_cols - 1, min(n_cols, k), min(n_cols, k + 1), 0, max(n_cols // 3, 1)], np.int32)
-    ld = n_cols + 5
+    ld = n_cols + pad
     buf = np.zeros((rows, ld), np.float32)
     buf[:, :n_cols] = s
     scores = torch.from_numpy(buf).cuda()
