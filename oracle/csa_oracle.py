@@ -96,8 +96,69 @@ def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
     return E4M3_VALUES[np.asarray(codes, dtype=np.uint8)]
 
 
+# ---------------------------------------------------------------------------
+# MXFP4 main KV.  Tech-report tour, chapter "Engram, DSpark, FP4", section
+# "FP4 main KV cache": elements are FP4 E2M1, one E4M3 scale per 16 channels,
+# no second-level (global) scale, so the largest storable magnitude is
+# 448 * 6 = 2688; values are dequantised before attention.
+# ---------------------------------------------------------------------------
+def _e2m1_table() -> np.ndarray:
+    """Value of every E2M1 code (OCP FP4), from the format definition.
+
+    Layout s ee m, exponent bias 1.  e == 0: subnormal m/2.  Otherwise
+    (1 + m/2) * 2^(e-1).  No infinities or NaN.
+    """
+    t = np.empty(16, np.float64)
+    for code in range(16):
+        sgn = -1.0 if code & 0x8 else 1.0
+        e, m = (code >> 1) & 0x3, code & 0x1
+        t[code] = sgn * (m / 2.0 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1))
+    return t
+
+
+E2M1_VALUES = _e2m1_table()
+E2M1_MAX = 6.0
+MXFP4_GROUP = 16
+
+
+def e2m1_round(y: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest E2M1 value, ties to the even code,
+    saturating at +-6.  Returns codes 0..15 (sign in bit 3; a negative value
+    that rounds to zero keeps its sign bit)."""
+    y = np.asarray(y, np.float64)
+    mags = E2M1_VALUES[:8]                       # codes 0..7, ascending
+    a = np.minimum(np.abs(y), E2M1_MAX)
+    hi = np.minimum(np.searchsorted(mags, a, side="left"), 7)
+    lo = np.maximum(hi - 1, 0)
+    d_hi, d_lo = mags[hi] - a, a - mags[lo]
+    code = np.where((d_lo < d_hi) | ((d_lo == d_hi) & (lo % 2 == 0)), lo, hi)
+    code = np.where(a == mags[hi], hi, code)
+    return (code | np.where(np.signbit(y), 8, 0)).astype(np.uint8)
+
+
+def quantize_mxfp4(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 storage of fp64 values (last axis a multiple of 32).
+
+    Reading of the section cited above: per 16 channels, the scale is the
+    E4M3 value nearest max|x| / 6 (round to nearest even, saturating at 448),
+    so that the largest magnitude lands on the largest E2M1 value; each
+    element is the E2M1 value nearest x / scale (saturating at 6); a zero
+    scale stores zero codes.  Returns (packed codes [.., d/2] uint8, element
+    2i in the low nibble of byte i; E4M3 scale codes [.., d/16] uint8)."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    g = x.reshape(x.shape[:-1] + (d // MXFP4_GROUP, MXFP4_GROUP))
+    sc_code = e4m3_round(np.abs(g).max(axis=-1) / E2M1_MAX)
+    sc = e4m3_to_f64(sc_code)
+    safe = np.where(sc > 0, sc, 1.0)
+    codes = np.where(sc[..., None] > 0, e2m1_round(g / safe[..., None]), 0).astype(np.uint8).reshape(x.shape)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return packed, sc_code
+
+
 def decode(data: np.ndarray, dtype: str, scale: np.ndarray | None = None, group: int = 0) -> np.ndarray:
-    """Exact fp64 value of a stored tensor (codes times group scale for FP8)."""
+    """Exact fp64 value of a stored tensor (codes times group scale for FP8
+    and MXFP4)."""
     if dtype == "f32":
         return np.asarray(data, dtype=np.float32).astype(np.float64)
     if dtype == "bf16":
@@ -106,6 +167,11 @@ def decode(data: np.ndarray, dtype: str, scale: np.ndarray | None = None, group:
         v = e4m3_to_f64(data)
         sc = np.repeat(np.asarray(scale, np.float64), group, axis=-1)
         return v * sc
+    if dtype == "mxfp4":
+        b = np.asarray(data, np.uint8)
+        codes = np.stack([b & 0xF, b >> 4], axis=-1).reshape(b.shape[:-1] + (2 * b.shape[-1],))
+        sc = np.repeat(e4m3_to_f64(scale), MXFP4_GROUP, axis=-1)
+        return E2M1_VALUES[codes] * sc
     raise ValueError(dtype)
 
 
@@ -151,6 +217,9 @@ def round_to_storage(x: np.ndarray, dtype: str, group: int = 0) -> np.ndarray:
     if dtype == "fp8":
         codes, scale = quantize_groups(x, group)
         return decode(codes, "fp8", scale, group)
+    if dtype == "mxfp4":
+        codes, scale = quantize_mxfp4(x)
+        return decode(codes, "mxfp4", scale, MXFP4_GROUP)
     raise ValueError(dtype)
 
 

@@ -448,3 +448,74 @@ def test_reindex_selects_inside_the_pool_by_brute_force():
     # fewer pool entries than k: all of them, padded with -1
     ids2, _ = O.reindex_topk(q, w, keys, pool, 8, 40)
     assert sorted(ids2[ids2 >= 0].tolist()) == sorted(members) and np.all(ids2[len(members):] == -1)
+
+
+# ---------------------------------------------------------------- MXFP4 main KV
+def test_e2m1_values_embed_in_the_torch_pinned_e4m3_table():
+    """E2M1 (1 sign, 2 exponent, 1 mantissa bit) is the set of E4M3 values in
+    [0, 6] with at most two significant bits and a multiple of 0.5: a
+    derivation from torch's E4M3 cast, independent of the oracle's formula."""
+    e4 = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+    def two_significant_bits(n):  # n > 0: its odd part has at most two bits
+        return (n // (n & -n)).bit_length() <= 2
+
+    cand = sorted({float(v) for v in e4 if np.isfinite(v) and 0 <= v <= 6 and 2 * v == int(2 * v)
+                   and (v == 0 or two_significant_bits(int(2 * v)))})
+    assert np.array_equal(O.E2M1_VALUES[:8], np.array(cand))
+    assert np.array_equal(O.E2M1_VALUES[8:], -O.E2M1_VALUES[:8])
+
+
+def test_mxfp4_ceiling_from_the_page():
+    f = _facts()["mxfp4"]
+    assert O.E2M1_MAX == f["e2m1_max"] and O.E4M3_MAX == f["e4m3_max"] and O.MXFP4_GROUP == f["group"]
+    top = np.abs(np.outer(O.E2M1_VALUES, O.e4m3_to_f64(np.arange(0x7F)))).max()
+    assert top == f["ceiling"] == f["e4m3_max"] * f["e2m1_max"]
+    # a group at the ceiling is stored exactly; beyond it, it saturates there
+    x = np.zeros((1, 32))
+    x[0, 3], x[0, 20] = 2688.0, -1e6
+    c, s = O.quantize_mxfp4(x)
+    y = O.decode(c, "mxfp4", s, 16)
+    assert y[0, 3] == 2688.0 and y[0, 20] == -2688.0
+    # the largest magnitude seen in training sits > 100x below the ceiling
+    assert f["ceiling"] / f["largest_observed_about"] > 100
+
+
+def test_e2m1_round_is_nearest_with_ties_to_even_by_brute_force():
+    mags = O.E2M1_VALUES[:8]
+    g = np.random.default_rng(11)
+    mids = (mags[1:] + mags[:-1]) / 2
+    x = np.concatenate([g.uniform(-8, 8, 4000), mids, -mids, mags, -mags, [0.0, 6.5, -100.0]])
+    got = O.E2M1_VALUES[O.e2m1_round(x)]
+    for xi, gi in zip(x, got):
+        a = min(abs(xi), 6.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        code = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert abs(gi) == mags[code] and (gi == 0 or np.sign(gi) == np.sign(xi))
+
+
+def test_mxfp4_round_trip_error_bound_and_layout():
+    g = np.random.default_rng(12)
+    # values on the grid of a group whose largest code is 6: stored exactly
+    s = O.e4m3_to_f64(g.integers(0x20, 0x60, size=(50, 4)))
+    codes = g.integers(0, 16, size=(50, 4, 16))
+    codes[:, :, 5] = 7
+    x = (O.E2M1_VALUES[codes] * s[..., None]).reshape(50, 64)
+    c, sc = O.quantize_mxfp4(x)
+    assert np.array_equal(O.decode(c, "mxfp4", sc, 16), x)
+    # Gaussian rows: the error of an element is at most its group's scale
+    y = g.standard_normal((40, 512)) * np.exp(g.uniform(-3, 3, (40, 1)))
+    c, sc = O.quantize_mxfp4(y)
+    err = np.abs(O.decode(c, "mxfp4", sc, 16) - y)
+    assert np.all(err <= np.repeat(O.e4m3_to_f64(sc), 16, axis=-1) * (1 + 1e-12))
+    # element 2i in the low nibble of byte i; the sign in bit 3 of a nibble
+    b = np.array([[0x72, 0x0F] + [0] * 14], np.uint8)
+    v = O.decode(b, "mxfp4", np.array([[0x38, 0x38]], np.uint8), 16)
+    assert v[0, :4].tolist() == [1.0, 6.0, -6.0, 0.0]
+    # a 512-channel row: 256 code bytes + 32 scale bytes = 288, vs 544 for FP8
+    # with an fp32 scale per 64 ("nearly halves")
+    assert 512 // 2 + 512 // 16 == 288 and 288 / (512 + 4 * 8) < 0.55
+    # an all-zero group keeps a zero scale and zero codes
+    c, sc = O.quantize_mxfp4(np.zeros((1, 32)))
+    assert np.all(c == 0) and np.all(sc == 0)
