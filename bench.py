@@ -74,6 +74,8 @@ def key_row_bytes(wl):
 
 
 def kv_row_bytes(wl):
+    if wl.kv_dtype == "mxfp4":
+        return wl.d // 2 + wl.d // 16  # two E2M1 codes per byte, one E4M3 scale byte per 16
     return wl.d * _eb(wl.kv_dtype) + (4 * wl.d // wl.kv_group if wl.kv_dtype == "fp8" else 0)
 
 
@@ -322,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8" if wl.kv_dtype == "fp8" else wl.act_dtype,
+        "dtype": wl.kv_dtype if wl.kv_dtype in ("fp8", "mxfp4") else wl.act_dtype,
         "data": "synthetic (seeded Gaussian caches and queries)",
         "config": {
             "workload": wl.name, "batch_per_gpu": B, "context": wl.context, "m": wl.m,

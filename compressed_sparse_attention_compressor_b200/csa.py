@@ -18,8 +18,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcsa.so")
 
-CSA_F32, CSA_BF16, CSA_FP8_E4M3 = 0, 1, 2
-_DTYPES = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8": CSA_FP8_E4M3}
+CSA_F32, CSA_BF16, CSA_FP8_E4M3, CSA_MXFP4_E2M1 = 0, 1, 2, 3
+_DTYPES = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8": CSA_FP8_E4M3, "mxfp4": CSA_MXFP4_E2M1}
 STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CAPACITY",
           4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_CUDA"}
 
@@ -102,8 +102,9 @@ def load() -> ctypes.CDLL:
 @dataclass
 class DevTensor:
     """A device tensor in storage format: ``data`` (float32 / int16 bf16 bits /
-    uint8 E4M3 codes) plus, for 'fp8', fp32 ``scale`` with one value per
-    ``group`` consecutive elements of a row."""
+    uint8 E4M3 codes / uint8 pairs of E2M1 codes) plus, for 'fp8', fp32
+    ``scale`` with one value per ``group`` consecutive elements of a row, for
+    'mxfp4', uint8 E4M3 scale codes, one per 16 elements."""
 
     data: torch.Tensor
     dtype: str
@@ -112,10 +113,14 @@ class DevTensor:
 
     def c(self) -> Tensor:
         return Tensor(self.data.data_ptr(), self.scale.data_ptr() if self.scale is not None else None,
-                      _DTYPES[self.dtype], self.group if self.dtype == "fp8" else 0)
+                      _DTYPES[self.dtype], self.group if self.dtype in ("fp8", "mxfp4") else 0)
 
     @staticmethod
     def empty(shape, dtype: str, device="cuda", group: int = 0) -> "DevTensor":
+        if dtype == "mxfp4":
+            lead = tuple(shape[:-1])
+            return DevTensor(torch.zeros(lead + (shape[-1] // 2,), dtype=torch.uint8, device=device), "mxfp4",
+                             torch.zeros(lead + (shape[-1] // 16,), dtype=torch.uint8, device=device), 16)
         tdt = {"f32": torch.float32, "bf16": torch.int16, "fp8": torch.uint8}[dtype]
         data = torch.zeros(tuple(shape), dtype=tdt, device=device)
         scale = None

@@ -45,7 +45,7 @@ struct AttnCfg {
 
 struct AttnArgs {
   const void* q; int q_dtype;
-  const void* kv; const float* kv_scale; int kv_dtype; int kv_group; int batch; int64_t cap;
+  const void* kv; const void* kv_scale; int kv_dtype; int kv_group; int batch; int64_t cap;
   const int32_t* idx; int topk;           // idx == nullptr: dense over n_visible
   const int32_t* n_visible; const int32_t* q_req;
   const void* swa_k; const void* swa_v; int swa_dtype; int swa_cap; int window;
@@ -103,7 +103,7 @@ attn_simt_kernel(AttnArgs a) {
   const int hh = tid / TPH;          // head owned in the accumulate phase
   const int c4 = tid % TPH;          // first float4 column owned
 
-  const int kveb = elem_bytes(a.kv_dtype), sweb = elem_bytes(a.swa_dtype);
+  const int sweb = elem_bytes(a.swa_dtype);
   const int64_t kv_row0 = live ? static_cast<int64_t>(r) * a.cap : 0;
   const int64_t sw_row0 = live ? static_cast<int64_t>(r) * a.swa_cap : 0;
 
@@ -131,8 +131,12 @@ attn_simt_kernel(AttnArgs a) {
       float x[8], y[8];
       if (e >= 0) {
         const int64_t gr = kv_row0 + e;
-        load8(static_cast<const char*>(a.kv) + gr * D * kveb, a.kv_dtype, col,
-              a.kv_scale ? a.kv_scale + gr * (D / a.kv_group) : nullptr, a.kv_group, x);
+        // FP8: fp32 scales; MXFP4: E4M3 scale bytes
+        const void* srow = a.kv_scale == nullptr ? nullptr
+                           : a.kv_dtype == kMXFP4
+                               ? static_cast<const void*>(static_cast<const uint8_t*>(a.kv_scale) + gr * (D / 16))
+                               : static_cast<const void*>(static_cast<const float*>(a.kv_scale) + gr * (D / a.kv_group));
+        load8(static_cast<const char*>(a.kv) + row_bytes(a.kv_dtype, gr * D), a.kv_dtype, col, srow, a.kv_group, x);
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = x[i];
       } else if (e <= -2) {
@@ -411,7 +415,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
   AttnArgs a;
   a.q = q->data; a.q_dtype = q->dtype;
   a.kv = kv->data; a.kv_scale = kv->scale; a.kv_dtype = kv->dtype;
-  a.kv_group = kv->dtype == kFP8 ? kv->scale_group : 1; a.batch = batch; a.cap = cap;
+  a.kv_group = (kv->dtype == kFP8 || kv->dtype == kMXFP4) ? kv->scale_group : 1; a.batch = batch; a.cap = cap;
   a.idx = idx; a.topk = p->topk;
   a.n_visible = n_visible; a.q_req = q_req;
   a.swa_k = swa_k ? swa_k->data : nullptr; a.swa_v = swa_v ? swa_v->data : nullptr;

@@ -51,7 +51,7 @@ constexpr int kSmem = oMisc + 64 + 1024;
 __device__ uint32_t g_attn_tc_error = 0;
 
 struct AttnTcArgs {
-  const void* kv; const float* kv_scale; int kv_fp8; int batch; int64_t cap;
+  const void* kv; const void* kv_scale; int kv_fmt; int batch; int64_t cap;
   const int32_t* idx; int topk;   // idx == nullptr: dense over n_visible
   const int32_t* n_visible; const int32_t* q_req;
   const uint16_t* swa_k; const uint16_t* swa_v; int swa_cap; int window;
@@ -153,7 +153,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   Src src;
   src.kv = a.kv;
   src.kv_scale = a.kv_scale;
-  src.kv_fp8 = a.kv_fp8;
+  src.kv_fmt = a.kv_fmt;
   src.swa_k = a.swa_k;
   src.swa_v = a.swa_v;
   src.kv_row0 = kv_row0;
@@ -301,7 +301,7 @@ int attn_cluster_min(int sel_max, int window) {
 
 bool attn_tc_supported(const csa_params_t* p, int q_dtype, int kv_dtype, int swa_dtype, bool has_window) {
   if (p->h_q != kH || p->d != kD || q_dtype != kBF16) return false;
-  if (kv_dtype != kBF16 && !(kv_dtype == kFP8)) return false;
+  if (kv_dtype != kBF16 && kv_dtype != kFP8 && kv_dtype != kMXFP4) return false;
   if (has_window && swa_dtype != kBF16) return false;
   return true;
 }
@@ -333,7 +333,7 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
   AttnTcArgs a;
   a.kv = kv->data;
   a.kv_scale = kv->scale;
-  a.kv_fp8 = kv->dtype == kFP8;
+  a.kv_fmt = kv->dtype == kFP8 ? kKvFP8 : kv->dtype == kMXFP4 ? kKvMX4 : kKvBF16;
   a.batch = batch;
   a.cap = cap;
   a.idx = idx;

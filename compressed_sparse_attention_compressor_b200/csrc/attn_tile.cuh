@@ -1,6 +1,6 @@
 // One attention tile on the tensor cores: the 64 query heads (d = 512) of
 // one query over up to 128 keys -- selected compressed entries (K = V = the
-// latent, FP8 dequantised to bf16) and sliding-window positions (separate K
+// latent, FP8 or MXFP4 dequantised to bf16) and sliding-window positions (separate K
 // and V) -- with the unnormalised result left in TMEM and the per-head
 // softmax statistics in shared memory.  Used by the stand-alone attention
 // kernels and by the decode step's fused indexer.
@@ -61,12 +61,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return static_cast<uint32_t>(f32_to_bf16_bits(a)) | (static_cast<uint32_t>(f32_to_bf16_bits(b)) << 16);
 }
 
+// Storage of the compressed rows.
+constexpr int kKvBF16 = 0;
+constexpr int kKvFP8 = 1;   // E4M3 codes, one fp32 scale per 64 elements
+constexpr int kKvMX4 = 2;   // E2M1 codes (two per byte), one E4M3 scale byte per 16 elements
+
 // Where the tile's rows come from: entry codes e >= 0 name compressed row
 // kv_row0 + e, e <= -2 window slot sw_row0 + (-2 - e), e = -1 nothing.
 struct Src {
   const void* kv;
-  const float* kv_scale;  // FP8: one scale per 64 elements
-  int kv_fp8;
+  const void* kv_scale;
+  int kv_fmt;             // kKvBF16 / kKvFP8 / kKvMX4
   const uint16_t* swa_k;
   const uint16_t* swa_v;
   int64_t kv_row0;
@@ -74,46 +79,84 @@ struct Src {
   float tau;
 };
 
+// One 16-byte chunk of a quantised compressed row with its scale(s): FP8, 16
+// codes and their fp32 scale; MXFP4, 32 codes and the two scale bytes of
+// their 16-element groups.
+struct QChunk {
+  uint4 u;
+  uint32_t s;
+};
+
+__device__ __forceinline__ int q_chunks_per_row(int fmt) { return fmt == kKvMX4 ? kD / 32 : kD / 16; }
+
+__device__ __forceinline__ QChunk load_qchunk(const Src& a, int64_t gr, int c) {
+  QChunk q;
+  if (a.kv_fmt == kKvMX4) {
+    q.u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * (kD / 2)) + c);
+    q.s = __ldg(reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(a.kv_scale) + gr * (kD / 16)) + c);
+  } else {
+    q.u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * kD) + c);
+    q.s = __float_as_uint(__ldg(static_cast<const float*>(a.kv_scale) + gr * (kD / 64) + (c >> 2)));
+  }
+  return q;
+}
+
+// Dequantises chunk c of a row into tile row r as bf16 (exact for MXFP4: an
+// E2M1 value times an E4M3 scale has at most 5 significant bits).
+__device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QChunk& q, int fmt) {
+  const uint32_t w[4] = {q.u.x, q.u.y, q.u.z, q.u.w};
+  if (fmt == kKvMX4) {
+    const float s0 = e4m3_to_f32(static_cast<uint8_t>(q.s & 0xFF)), s1 = e4m3_to_f32(static_cast<uint8_t>(q.s >> 8));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // word i: elements 8i .. 8i+7, nibble k = element 8i + k
+      const float sc = i < 2 ? s0 : s1;
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        o[k] = pack_bf16(e2m1_to_f32(w[i] >> (8 * k)) * sc, e2m1_to_f32(w[i] >> (8 * k + 4)) * sc);
+      put_chunk(tile, r, c * 32 + i * 8, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  } else {
+    const float sc = __uint_as_float(q.s);
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFF));
+      const float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
+      o[2 * i] = pack_bf16(lo.x * sc, lo.y * sc);
+      o[2 * i + 1] = pack_bf16(hi.x * sc, hi.y * sc);
+    }
+    put_chunk(tile, r, c * 16, make_uint4(o[0], o[1], o[2], o[3]));
+    put_chunk(tile, r, c * 16 + 8, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
 // All threads: rows of the tile from their sources.  which = 0: keys
 // (compressed entries and window keys); which = 1: only the window rows,
 // from the value ring (compressed rows are their own values).  Loads are
 // issued in batches of 8 per thread before any of them is used.
 __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int which) {
   constexpr int B = 8;
-  if (a.kv_fp8 && which == 0) {
-    // FP8 entries: 32 tasks of 16 codes per row
-    for (int t0 = static_cast<int>(threadIdx.x); t0 < kTK * 32; t0 += kNT * B) {
-      uint4 u[B];
-      float sc[B];
+  if (a.kv_fmt != kKvBF16 && which == 0) {
+    // quantised entries: tpr tasks of one 16-byte chunk per row
+    const int tpr = q_chunks_per_row(a.kv_fmt);
+    for (int t0 = static_cast<int>(threadIdx.x); t0 < kTK * tpr; t0 += kNT * B) {
+      QChunk q[B];
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const int task = t0 + b * kNT;
-        const int r = task >> 5, c16 = task & 31;
-        const int32_t e = task < kTK * 32 ? ent[r] : -1;
-        u[b] = make_uint4(0, 0, 0, 0);
-        sc[b] = 0.f;
-        if (e >= 0) {
-          const int64_t gr = a.kv_row0 + e;
-          u[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * kD) + c16);
-          sc[b] = __ldg(a.kv_scale + gr * (kD / 64) + (c16 >> 2));
-        }
+        const int r = task / tpr, c = task % tpr;
+        const int32_t e = task < kTK * tpr ? ent[r] : -1;
+        q[b].u = make_uint4(0, 0, 0, 0);
+        q[b].s = 0u;
+        if (e >= 0) q[b] = load_qchunk(a, a.kv_row0 + e, c);
       }
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const int task = t0 + b * kNT;
-        const int r = task >> 5, c16 = task & 31;
-        if (task >= kTK * 32 || ent[r] < 0) continue;
-        const uint32_t w[4] = {u[b].x, u[b].y, u[b].z, u[b].w};
-        uint32_t o[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFF));
-          const float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
-          o[2 * i] = pack_bf16(lo.x * sc[b], lo.y * sc[b]);
-          o[2 * i + 1] = pack_bf16(hi.x * sc[b], hi.y * sc[b]);
-        }
-        put_chunk(tile, r, c16 * 16, make_uint4(o[0], o[1], o[2], o[3]));
-        put_chunk(tile, r, c16 * 16 + 8, make_uint4(o[4], o[5], o[6], o[7]));
+        const int r = task / tpr, c = task % tpr;
+        if (task >= kTK * tpr || ent[r] < 0) continue;
+        put_qchunk(tile, r, c, q[b], a.kv_fmt);
       }
     }
   }
@@ -129,7 +172,7 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
       v[b] = make_uint4(0, 0, 0, 0);
       put[b] = task < kTK * 64;
       if (e >= 0) {
-        if (a.kv_fp8 || which == 1) put[b] = false;  // FP8 rows done above; compressed rows keep their keys
+        if (a.kv_fmt != kKvBF16 || which == 1) put[b] = false;  // quantised rows done above; compressed rows keep their keys
         else v[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + (a.kv_row0 + e) * kD) + c8);
       } else if (e <= -2) {
         const uint16_t* src = (which == 0 ? a.swa_k : a.swa_v) + (a.sw_row0 + (-2 - e)) * kD;
@@ -160,7 +203,7 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
 // [nsr + nwr, nk16) are zeroed (the PV product reads them with weight 0).
 __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, int nsr, int nwr, int nk16,
                                uint4 (&vw)[4]) {
-  const int per_sel = a.kv_fp8 ? 32 : 64;  // 16-byte chunks per selected row
+  const int per_sel = a.kv_fmt == kKvBF16 ? 64 : q_chunks_per_row(a.kv_fmt);  // 16-byte chunks per selected row
   const int T1 = nsr * per_sel, T = T1 + nwr * 64;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
@@ -173,29 +216,26 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
   }
   constexpr int B = 16;
   for (int t0 = static_cast<int>(threadIdx.x); t0 < T; t0 += kNT * B) {
-    uint4 u[B];
-    float sc[B];
+    QChunk q[B];
 #pragma unroll
     for (int b = 0; b < B; ++b) {
       const int task = t0 + b * kNT;
-      u[b] = make_uint4(0, 0, 0, 0);
-      sc[b] = 0.f;
+      q[b].u = make_uint4(0, 0, 0, 0);
+      q[b].s = 0u;
       if (task < T1) {
         const int r = task / per_sel, c = task % per_sel;
         const int32_t e = ent[r];
         if (e >= 0) {
           const int64_t gr = a.kv_row0 + e;
-          if (a.kv_fp8) {
-            u[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * kD) + c);
-            sc[b] = __ldg(a.kv_scale + gr * (kD / 64) + (c >> 2));
-          } else {
-            u[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + gr * kD) + c);
-          }
+          if (a.kv_fmt != kKvBF16)
+            q[b] = load_qchunk(a, gr, c);
+          else
+            q[b].u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + gr * kD) + c);
         }
       } else if (task < T) {
         const int w = task - T1;
         const int32_t e = ent[nsr + (w >> 6)];
-        if (e <= -2) u[b] = __ldg(reinterpret_cast<const uint4*>(a.swa_k + (a.sw_row0 + (-2 - e)) * kD) + (w & 63));
+        if (e <= -2) q[b].u = __ldg(reinterpret_cast<const uint4*>(a.swa_k + (a.sw_row0 + (-2 - e)) * kD) + (w & 63));
       }
     }
 #pragma unroll
@@ -203,26 +243,13 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
       const int task = t0 + b * kNT;
       if (task < T1) {
         const int r = task / per_sel, c = task % per_sel;
-        if (a.kv_fp8) {
-          const uint32_t w[4] = {u[b].x, u[b].y, u[b].z, u[b].w};
-          uint32_t o[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFF));
-            const float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
-            const __nv_bfloat162 bl = __floats2bfloat162_rn(lo.x * sc[b], lo.y * sc[b]);
-            const __nv_bfloat162 bh = __floats2bfloat162_rn(hi.x * sc[b], hi.y * sc[b]);
-            o[2 * i] = *reinterpret_cast<const uint32_t*>(&bl);
-            o[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&bh);
-          }
-          put_chunk(tile, r, c * 16, make_uint4(o[0], o[1], o[2], o[3]));
-          put_chunk(tile, r, c * 16 + 8, make_uint4(o[4], o[5], o[6], o[7]));
-        } else {
-          put_chunk(tile, r, c * 8, u[b]);
-        }
+        if (a.kv_fmt != kKvBF16)
+          put_qchunk(tile, r, c, q[b], a.kv_fmt);
+        else
+          put_chunk(tile, r, c * 8, q[b].u);
       } else if (task < T) {
         const int w = task - T1;
-        put_chunk(tile, nsr + (w >> 6), (w & 63) * 8, u[b]);
+        put_chunk(tile, nsr + (w >> 6), (w & 63) * 8, q[b].u);
       }
     }
   }

@@ -1,5 +1,6 @@
 // Device-side helpers shared by the kernels of the library: storage-format
-// loads/stores (fp32, bf16, FP8 E4M3 with fp32 group scales), the ordered
+// loads/stores (fp32, bf16, FP8 E4M3 with fp32 group scales, MXFP4: E2M1
+// with E4M3 scales per 16 elements), the ordered
 // 32-bit key of an fp32 score, and host-side error plumbing.
 #pragma once
 
@@ -15,6 +16,7 @@ namespace csa {
 constexpr int kF32 = CSA_F32;
 constexpr int kBF16 = CSA_BF16;
 constexpr int kFP8 = CSA_FP8_E4M3;
+constexpr int kMXFP4 = CSA_MXFP4_E2M1;
 
 // --------------------------------------------------------------------------
 // scalar conversions
@@ -42,6 +44,24 @@ __device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
 }
 
+// OCP E2M1: sign in bit 3, two exponent bits (bias 1), one mantissa bit;
+// exponent 0 is subnormal (0 or 0.5).  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
+  const uint32_t m = code & 7u;
+  const uint32_t mag = m >= 2u ? (((m >> 1) + 126u) << 23) | ((m & 1u) << 22) : (m ? 0x3F000000u : 0u);
+  return __uint_as_float(mag | ((code & 8u) << 28));
+}
+
+// Round to the nearest E2M1 value, a tie to the even code, saturating at 6:
+// the decision points are the midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5
+// (a midpoint itself goes to the neighbour with the even code).
+__device__ __forceinline__ uint32_t f32_to_e2m1(float x) {
+  const float a = fabsf(x);
+  const uint32_t m = a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
+                   : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.f ? 6u : 7u;
+  return m | ((__float_as_uint(x) >> 28) & 8u);
+}
+
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
   __nv_bfloat16 b = __float2bfloat16_rn(x);
   return *reinterpret_cast<uint16_t*>(&b);
@@ -51,9 +71,10 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
 // 8-element vector loads (16 B of bf16, 32 B of fp32, 8 B of fp8)
 // --------------------------------------------------------------------------
 // Loads elements [col, col+8) of a row into v (fp32).  For FP8, `scale`
-// points at the row's group scales and `group` is the group length
-// (a multiple of 8, so the 8 elements share one scale).
-__device__ __forceinline__ void load8(const void* row, int dtype, int col, const float* scale, int group,
+// points at the row's fp32 group scales and `group` is the group length
+// (a multiple of 8, so the 8 elements share one scale); for MXFP4 at the
+// row's E4M3 scale bytes (group 16), with `row` at the row's first code byte.
+__device__ __forceinline__ void load8(const void* row, int dtype, int col, const void* scale, int group,
                                       float v[8]) {
   if (dtype == kF32) {
     const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(row) + col);
@@ -68,9 +89,14 @@ __device__ __forceinline__ void load8(const void* row, int dtype, int col, const
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
+  } else if (dtype == kMXFP4) {
+    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(row) + col / 2));
+    const float s = e4m3_to_f32(__ldg(static_cast<const uint8_t*>(scale) + col / 16));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = e2m1_to_f32(u >> (4 * e)) * s;
   } else {
     uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(row) + col));
-    float s = __ldg(scale + col / group);
+    float s = __ldg(static_cast<const float*>(scale) + col / group);
     uint32_t w[2] = {u.x, u.y};
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -98,14 +124,24 @@ __device__ __forceinline__ void store8(void* row, int dtype, int col, const floa
   }
 }
 
-__device__ __forceinline__ float load1(const void* row, int dtype, int col, const float* scale, int group) {
+__device__ __forceinline__ float load1(const void* row, int dtype, int col, const void* scale, int group) {
   if (dtype == kF32) return __ldg(static_cast<const float*>(row) + col);
   if (dtype == kBF16) return bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(row) + col));
-  return e4m3_to_f32(__ldg(static_cast<const uint8_t*>(row) + col)) * __ldg(scale + col / group);
+  if (dtype == kMXFP4)
+    return e2m1_to_f32(__ldg(static_cast<const uint8_t*>(row) + col / 2) >> (4 * (col & 1))) *
+           e4m3_to_f32(__ldg(static_cast<const uint8_t*>(scale) + col / 16));
+  return e4m3_to_f32(__ldg(static_cast<const uint8_t*>(row) + col)) *
+         __ldg(static_cast<const float*>(scale) + col / group);
 }
 
+// Bytes per element (MXFP4: see row_bytes).
 __host__ __device__ __forceinline__ int elem_bytes(int dtype) {
   return dtype == kF32 ? 4 : (dtype == kBF16 ? 2 : 1);
+}
+
+// Bytes of `n` elements of a row (MXFP4: two elements per byte).
+__host__ __device__ __forceinline__ int64_t row_bytes(int dtype, int64_t n) {
+  return dtype == kMXFP4 ? n / 2 : n * elem_bytes(dtype);
 }
 
 // --------------------------------------------------------------------------

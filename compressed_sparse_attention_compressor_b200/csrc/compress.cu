@@ -56,7 +56,7 @@ __device__ __forceinline__ void project_row(const float* pooled, int d, const vo
 #pragma unroll
     for (int k = 0; k < 8; ++k)
       if (k < per) dst[lane + 32 * k] = f32_to_e4m3(acc[k] / s);
-    if (lane == 0) ko.scale[row * ko.scale_stride] = s;
+    if (lane == 0) static_cast<float*>(ko.scale)[row * ko.scale_stride] = s;
   } else if (ko.dtype == kBF16) {
     uint16_t* dst = static_cast<uint16_t*>(ko.data) + row * ko.row_stride;
 #pragma unroll
@@ -130,7 +130,7 @@ __device__ __forceinline__ void store_key_row(const float* kv, int d_idx, const 
     const float s = amax > 0.f ? amax / 448.f : 1.f;
     uint8_t* dst = static_cast<uint8_t*>(ko.data) + row * ko.row_stride;
     for (int i = lane; i < d_idx; i += 32) dst[i] = f32_to_e4m3(kv[i] / s);
-    if (lane == 0) ko.scale[row * ko.scale_stride] = s;
+    if (lane == 0) static_cast<float*>(ko.scale)[row * ko.scale_stride] = s;
   } else if (ko.dtype == kBF16) {
     uint16_t* dst = static_cast<uint16_t*>(ko.data) + row * ko.row_stride;
     for (int i = lane; i < d_idx; i += 32) dst[i] = f32_to_bf16_bits(kv[i]);
@@ -495,7 +495,7 @@ decode_append_cluster_kernel(const int64_t* __restrict__ pos, int m, int d, int 
         for (int w = 0; w < 8; ++w) amax = fmaxf(amax, amax_w[w]);
         const float s = amax > 0.f ? amax / 448.f : 1.f;
         if (tid < d_idx) static_cast<uint8_t*>(kidx.data)[row * kidx.row_stride + tid] = f32_to_e4m3(key / s);
-        if (tid == 0) kidx.scale[row * kidx.scale_stride] = s;
+        if (tid == 0) static_cast<float*>(kidx.scale)[row * kidx.scale_stride] = s;
       } else if (tid < d_idx) {
         if (kidx.dtype == kBF16) static_cast<uint16_t*>(kidx.data)[row * kidx.row_stride + tid] = f32_to_bf16_bits(key);
         else static_cast<float*>(kidx.data)[row * kidx.row_stride + tid] = key;

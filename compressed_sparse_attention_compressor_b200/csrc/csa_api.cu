@@ -72,16 +72,23 @@ int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// allow_mx4: MXFP4 main-KV rows (scale_group 16, E4M3 scale bytes).
 csa_status_t check_tensor(const char* name, const csa_tensor_t* t, int row_elems, bool allow_f32, bool allow_bf16,
-                          bool allow_fp8, int fp8_group) {
+                          bool allow_fp8, int fp8_group, bool allow_mx4 = false) {
   if (t == nullptr || t->data == nullptr) return set_error(CSA_ERR_INVALID_ARG, "%s: null tensor", name);
   const int dt = t->dtype;
   if ((dt == kF32 && !allow_f32) || (dt == kBF16 && !allow_bf16) || (dt == kFP8 && !allow_fp8) ||
-      (dt != kF32 && dt != kBF16 && dt != kFP8))
+      (dt == kMXFP4 && !allow_mx4) || (dt != kF32 && dt != kBF16 && dt != kFP8 && dt != kMXFP4))
     return set_error(CSA_ERR_INVALID_ARG, "%s: dtype %d not accepted here", name, dt);
   if (!aligned16(t->data)) return set_error(CSA_ERR_INVALID_ARG, "%s: data not 16-byte aligned", name);
-  if ((static_cast<int64_t>(row_elems) * elem_bytes(dt)) % 16 != 0)
+  if (row_bytes(dt, row_elems) % 16 != 0 || (dt == kMXFP4 && row_elems % 32 != 0))
     return set_error(CSA_ERR_INVALID_ARG, "%s: rows of %d elements are not a multiple of 16 bytes", name, row_elems);
+  if (dt == kMXFP4) {
+    if (t->scale == nullptr || !aligned16(t->scale))
+      return set_error(CSA_ERR_INVALID_ARG, "%s: MXFP4 tensor without 16-byte aligned scales", name);
+    if (t->scale_group != 16)
+      return set_error(CSA_ERR_INVALID_ARG, "%s: MXFP4 scale_group must be 16 (got %d)", name, t->scale_group);
+  }
   if (dt == kFP8) {
     if (t->scale == nullptr) return set_error(CSA_ERR_INVALID_ARG, "%s: FP8 tensor without scales", name);
     if (fp8_group > 0 && t->scale_group != fp8_group)
@@ -230,7 +237,7 @@ csa_status_t csa_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int32_t 
   if ((st = check_tensor("C", C, d, true, true, false, 0)) != CSA_OK) return st;
   if ((st = check_tensor("Z", Z, d, true, true, false, 0)) != CSA_OK) return st;
   if (Z->dtype != C->dtype) return set_error(CSA_ERR_INVALID_ARG, "C and Z dtypes differ");
-  if ((st = check_tensor("out", out, d, true, true, true, 64)) != CSA_OK) return st;
+  if ((st = check_tensor("out", out, d, true, true, true, 64, true)) != CSA_OK) return st;
   if (w_ik != nullptr) {
     if (d_idx < 32 || d_idx > 256 || d_idx % 32 != 0)
       return set_error(CSA_ERR_UNSUPPORTED, "d_idx=%d: projection needs a multiple of 32 in [32, 256]", d_idx);
@@ -418,7 +425,7 @@ csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, 
   if (n_queries < 0 || cap < 0 || batch < 1) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap");
   if (n_queries == 0) return CSA_OK;
   if ((st = check_tensor("q", q, p->d, true, true, false, 0)) != CSA_OK) return st;
-  if ((st = check_tensor("kv", kv, p->d, true, true, true, 64)) != CSA_OK) return st;
+  if ((st = check_tensor("kv", kv, p->d, true, true, true, 64, true)) != CSA_OK) return st;
   if ((st = check_tensor("out", out, p->d, true, true, false, 0)) != CSA_OK) return st;
   if (p->window > 0) {
     if ((st = check_tensor("swa_k", swa_k, p->d, true, true, false, 0)) != CSA_OK) return st;
@@ -451,7 +458,7 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
   if (sparse && !project) return set_error(CSA_ERR_INVALID_ARG, "a sparse (topk >= 1) step needs w_ik");
   if (project && (p->d_idx < 32 || p->d_idx > 256 || p->d_idx % 32 != 0))
     return set_error(CSA_ERR_UNSUPPORTED, "d_idx=%d: projection needs a multiple of 32 in [32, 256]", p->d_idx);
-  if ((st = check_tensor("kv", &cc->kv, p->d, true, true, true, 64)) != CSA_OK) return st;
+  if ((st = check_tensor("kv", &cc->kv, p->d, true, true, true, 64, true)) != CSA_OK) return st;
   if (project && (st = check_tensor("kidx", &cc->kidx, p->d_idx, true, true, true, p->d_idx)) != CSA_OK) return st;
   if ((st = check_tensor("swa_k", &cc->swa_k, p->d, true, true, false, 0)) != CSA_OK) return st;
   if ((st = check_tensor("swa_v", &cc->swa_v, p->d, true, true, false, 0)) != CSA_OK) return st;

@@ -534,7 +534,7 @@ __device__ void append_block(const AppendArgs& p, int r, int64_t cap, uint8_t* w
         for (int w = 0; w < kDI / 32; ++w) amax = fmaxf(amax, red[2 * kDI + w]);
         const float sc = amax > 0.f ? amax / 448.f : 1.f;
         if (tid < kDI) static_cast<uint8_t*>(p.kidx.data)[row * p.kidx.row_stride + tid] = f32_to_e4m3(key / sc);
-        if (tid == 0) p.kidx.scale[row * p.kidx.scale_stride] = sc;
+        if (tid == 0) static_cast<float*>(p.kidx.scale)[row * p.kidx.scale_stride] = sc;
       } else if (tid < kDI) {
         if (p.kidx.dtype == kBF16) static_cast<uint16_t*>(p.kidx.data)[row * p.kidx.row_stride + tid] = f32_to_bf16_bits(key);
         else static_cast<float*>(p.kidx.data)[row * p.kidx.row_stride + tid] = key;
@@ -1381,7 +1381,7 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.pool = pool;
   a.pool_blocks = pool_blocks;
   a.pblock = pblock;
-  a.kscale = fp8 ? k_idx->scale : nullptr;
+  a.kscale = fp8 ? static_cast<const float*>(k_idx->scale) : nullptr;
   if (ap) {
     a.ap = *ap;
     a.ap.shrink = kAppendShrink;

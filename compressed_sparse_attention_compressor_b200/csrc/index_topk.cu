@@ -326,7 +326,8 @@ csa_status_t launch_score_t(const csa_params_t* p, int nq, const csa_tensor_t* q
   dim3 grid(static_cast<unsigned>((max_entries + kScoreThreads - 1) / kScoreThreads), nq);
   prof_begin(stream);
   index_score_simt_kernel<H, DI><<<grid, kScoreThreads, 0, stream>>>(
-      q_idx->data, q_idx->dtype, w, k_idx->data, k_idx->scale, k_idx->dtype, batch, cap, q_req, n_visible, scores,
+      q_idx->data, q_idx->dtype, w, k_idx->data, static_cast<const float*>(k_idx->scale), k_idx->dtype, batch, cap,
+      q_req, n_visible, scores,
       ld, pool, block, pool_blocks);
   return check_launch("index_score_simt_kernel", stream);
 }

@@ -11,11 +11,12 @@
 
 namespace csa {
 
-// Destination of pooled rows: fp32 / bf16, or FP8 E4M3 codes with one fp32
-// scale per `group` elements (scale = max|x| / 448, 1 for an all-zero group).
+// Destination of pooled rows: fp32 / bf16, FP8 E4M3 codes with one fp32
+// scale per `group` elements (scale = max|x| / 448, 1 for an all-zero
+// group), or MXFP4 E2M1 codes with one E4M3 scale per 16 elements.
 struct OutSpec {
   void* data;
-  float* scale;
+  void* scale;
   int dtype;
   int group;
   int64_t row_stride;    // elements between rows
@@ -64,11 +65,34 @@ __device__ __forceinline__ void pool8(RowC rowC, RowZ rowZ, int in_dtype, int m,
   for (int e = 0; e < 8; ++e) out[e] = out[e] / den[e];
 }
 
-// Stores 8 pooled channels of one row.  For FP8 every lane of the warp must
-// call this (the 8 lanes of a 64-channel group exchange maxima); `valid`
-// masks the store.
+// Stores 8 pooled channels of one row.  For FP8 and MXFP4 every lane of the
+// warp must call this (the 8 lanes of a 64-channel FP8 group, or the 2 lanes
+// of a 16-channel MXFP4 group, exchange maxima); `valid` masks the store.
+//
+// MXFP4 (tech-report tour, chapter "Engram, DSpark, FP4", section "FP4 main
+// KV cache"): the group's scale is the E4M3 value nearest max|x| / 6 (so
+// that max|x| lands on the largest E2M1 magnitude), each element the E2M1
+// value nearest x / scale, saturating at 6; an all-zero scale stores zeros.
 __device__ __forceinline__ void store_pooled8(const OutSpec& o, int64_t row, int col, const float v[8],
                                               bool valid) {
+  if (o.dtype == kMXFP4) {
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));  // lanes 2g, 2g+1: one 16-channel group
+    if (!valid) return;
+    const uint8_t sc = f32_to_e4m3(amax / 6.f);
+    const float s = e4m3_to_f32(sc);
+    uint32_t w = 0u;
+    if (s > 0.f) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w |= f32_to_e2m1(v[e] / s) << (4 * e);
+    }
+    uint8_t* dst = static_cast<uint8_t*>(o.data) + (row * o.row_stride + col) / 2;
+    *reinterpret_cast<uint32_t*>(dst) = w;
+    if ((col % 16) == 0) static_cast<uint8_t*>(o.scale)[row * o.scale_stride + col / 16] = sc;
+    return;
+  }
   if (o.dtype != kFP8) {
     if (valid) store8(static_cast<char*>(o.data) + row * o.row_stride * elem_bytes(o.dtype), o.dtype, col, v);
     return;
@@ -87,7 +111,7 @@ __device__ __forceinline__ void store_pooled8(const OutSpec& o, int64_t row, int
   for (int e = 0; e < 8; ++e) w[e / 4] |= static_cast<uint32_t>(f32_to_e4m3(v[e] / s)) << (8 * (e % 4));
   uint8_t* dst = static_cast<uint8_t*>(o.data) + row * o.row_stride + col;
   *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-  if ((col % o.group) == 0) o.scale[row * o.scale_stride + col / o.group] = s;
+  if ((col % o.group) == 0) static_cast<float*>(o.scale)[row * o.scale_stride + col / o.group] = s;
 }
 
 inline OutSpec make_out_spec(const csa_tensor_t* t, int row_elems) {
@@ -95,9 +119,10 @@ inline OutSpec make_out_spec(const csa_tensor_t* t, int row_elems) {
   o.data = t ? t->data : nullptr;
   o.scale = t ? t->scale : nullptr;
   o.dtype = t ? t->dtype : kF32;
-  o.group = (t && t->dtype == kFP8) ? t->scale_group : 1;
+  const bool scaled = t && (t->dtype == kFP8 || t->dtype == kMXFP4);
+  o.group = scaled ? t->scale_group : 1;
   o.row_stride = row_elems;
-  o.scale_stride = (t && t->dtype == kFP8) ? row_elems / t->scale_group : 0;
+  o.scale_stride = scaled ? row_elems / t->scale_group : 0;
   return o;
 }
 

@@ -103,7 +103,11 @@ def store(x: np.ndarray, dtype: str, group: int = 0) -> Stored:
 
 
 def empty_stored(shape, dtype: str, group: int = 0) -> Stored:
-    """A zero-filled tensor in storage format ``dtype`` (scales of 1.0)."""
+    """A zero-filled tensor in storage format ``dtype`` (scales of 1.0; MXFP4:
+    zero codes and zero scale bytes)."""
+    if dtype == "mxfp4":
+        return Stored(np.zeros(tuple(shape[:-1]) + (shape[-1] // 2,), np.uint8), "mxfp4",
+                      np.zeros(tuple(shape[:-1]) + (shape[-1] // 16,), np.uint8), 16)
     if dtype == "f32":
         return Stored(np.zeros(shape, np.float32), "f32")
     if dtype == "bf16":
@@ -125,6 +129,18 @@ def rng(seed: int, tag: str) -> np.random.Generator:
 def normal(seed: int, tag: str, shape, std: float = 1.0) -> np.ndarray:
     g = rng(seed, tag)
     return g.standard_normal(size=shape, dtype=np.float32) * np.float32(std)
+
+
+def random_mxfp4(seed: int, tag: str, shape) -> Stored:
+    """An MXFP4 tensor drawn directly in storage form (no rounding): every
+    E2M1 code uniform over its 16 values, every E4M3 scale byte uniform over
+    0x28 .. 0x2F (0.25 .. 0.46875), so that a group's largest magnitude (6 x
+    scale, 1.5 .. 2.8) and the rms (about 1) are those of N(0, 1) entries.
+    ``shape`` is the logical [.., d] shape."""
+    g = rng(seed, tag)
+    data = g.integers(0, 256, size=tuple(shape[:-1]) + (shape[-1] // 2,), dtype=np.uint8)
+    scale = g.integers(0x28, 0x30, size=tuple(shape[:-1]) + (shape[-1] // 16,), dtype=np.uint8)
+    return Stored(data, "mxfp4", scale, 16)
 
 
 def uniform(seed: int, tag: str, shape) -> np.ndarray:
@@ -199,6 +215,9 @@ WORKLOADS: dict[str, Workload] = {
     # 512, a pool of 2,048 blocks of 8 positions
     "hier1m": Workload("hier1m", 4, 1048576, 1, 512, 64, 64, 128, 512, 128, "fp8", "fp8", "bf16", "normal",
                        seed=1008),
+    # decode1m with the main KV in MXFP4 (E2M1 + one E4M3 scale per 16)
+    "decode1m_fp4": Workload("decode1m_fp4", 4, 1048576, 4, 512, 64, 64, 128, 1024, 128, "mxfp4", "fp8", "bf16",
+                             "normal", kv_group=16, seed=1009),
 }
 
 # candidate pool of the hierarchical indexer: (block, pool_blocks)
@@ -247,6 +266,17 @@ def _sink(wl: Workload) -> np.ndarray:
     return normal(wl.seed, "sink", (wl.h_q,))
 
 
+def _kv_cache(seed: int, wl: Workload, kv: np.ndarray, n_filled: int) -> Stored:
+    """The main-KV cache in storage format: ``kv`` stored, or for MXFP4 rows
+    [0, n_filled) drawn directly in storage form and the rest zero."""
+    if wl.kv_dtype != "mxfp4":
+        return store(kv, wl.kv_dtype, wl.kv_group)
+    st = random_mxfp4(seed, "kv", kv.shape)
+    st.data[:, n_filled:] = 0
+    st.scale[:, n_filled:] = 0
+    return st
+
+
 def make_decode_inputs(wl: Workload) -> DecodeInputs:
     assert not wl.is_prefill
     B, T, m, d = wl.batch, wl.context, wl.m, wl.d
@@ -257,7 +287,9 @@ def make_decode_inputs(wl: Workload) -> DecodeInputs:
     s = wl.seed
     kv_std = 1.0 if wl.kv_dtype == "fp8" else sd
     kv = np.zeros((B, cap, d), np.float32)
-    kv[:, :n_prev] = normal(s, "kv", (B, n_prev, d), kv_std)
+    if wl.kv_dtype != "mxfp4":
+        kv[:, :n_prev] = normal(s, "kv", (B, n_prev, d), kv_std)
+    kv_st = _kv_cache(s, wl, kv, n_prev)
     kidx = np.zeros((B, cap, wl.d_idx), np.float32)
     kidx[:, :n_prev] = normal(s, "kidx", (B, n_prev, wl.d_idx), sI)
     W = wl.window
@@ -268,7 +300,7 @@ def make_decode_inputs(wl: Workload) -> DecodeInputs:
         pos=np.full(B, pos, np.int64),
         n_prev=n_prev,
         cap=cap,
-        kv=store(kv, wl.kv_dtype, wl.kv_group),
+        kv=kv_st,
         kidx=store(kidx, wl.idx_dtype, wl.idx_group),
         swa_k=store(normal(s, "swa_k", (B, swa_cap, d), sd), act),
         swa_v=store(normal(s, "swa_v", (B, swa_cap, d), sd), act),
@@ -390,7 +422,7 @@ def make_prefill_inputs(wl: Workload) -> PipelineInputs:
         C=store(normal(s, "C", (1, L, d), sd), f),
         Z=store(normal(s, "Z", (1, L, d)), f),
         n_cached=n_cached,
-        kv_cached=store(kv, wl.kv_dtype, wl.kv_group),
+        kv_cached=_kv_cache(s, wl, kv, n_cached),
         kidx_cached=store(kidx, wl.idx_dtype, wl.idx_group),
         cap=cap,
         swa_k=store(normal(s, "swa_k", (1, swa_cap, d), sd), f),

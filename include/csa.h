@@ -79,18 +79,29 @@ typedef enum csa_status {
 typedef enum csa_dtype {
   CSA_F32 = 0,
   CSA_BF16 = 1,
-  CSA_FP8_E4M3 = 2          /* OCP E4M3 ('fn': no infinities, 448 max), with
+  CSA_FP8_E4M3 = 2,         /* OCP E4M3 ('fn': no infinities, 448 max), with
                                one fp32 scale per scale_group elements        */
+  CSA_MXFP4_E2M1 = 3        /* OCP E2M1 (values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and
+                               negatives), two per byte -- element 2i in the
+                               low nibble of byte i, the sign in bit 3 of a
+                               nibble -- with one E4M3 scale byte per 16
+                               elements and no further scale: largest value
+                               6 * 448 = 2688.  Main-KV rows only.            */
 } csa_dtype_t;
 
 /* A tensor in storage format.  value = decode(data[i]) * scale[i / scale_group]
- * for CSA_FP8_E4M3 (scale indexed in the same row-major order, one scale per
- * scale_group consecutive elements of a row); scale is ignored otherwise.   */
+ * for CSA_FP8_E4M3 (scale: fp32) and CSA_MXFP4_E2M1 (scale: uint8 E4M3
+ * codes, scale_group 16), scale indexed in the same row-major order, one
+ * scale per scale_group consecutive elements of a row; scale is ignored
+ * otherwise.  CSA_MXFP4_E2M1 rows take d / 2 bytes of codes.  [TOUR] chapter
+ * "Engram, DSpark, FP4", section "FP4 main KV cache" (E2M1 elements, one
+ * E4M3 scale per 16 channels, no second-level scale, dequantised before
+ * attention; SWA KV stays 8-bit).                                          */
 typedef struct csa_tensor {
   void* data;
-  float* scale;
+  void* scale;
   int32_t dtype;        /* csa_dtype_t */
-  int32_t scale_group;  /* FP8 only: elements per scale; must divide the row */
+  int32_t scale_group;  /* FP8 / MXFP4: elements per scale; must divide the row */
 } csa_tensor_t;
 
 /* Problem shape shared by the calls. */

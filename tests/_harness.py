@@ -4,7 +4,7 @@ tolerances.
 
 Tolerances (the acceptance bar of the path):
 * attention outputs and lse, max-abs error against the fp64 oracle:
-  1e-4 for fp32 workloads, 2e-2 for bf16 / FP8 workloads;
+  1e-4 for fp32 workloads, 2e-2 for bf16 / FP8 / MXFP4 workloads;
 * selected index sets: fp32 workloads bit-exact (a differing set is only
   accepted, with a warning, when the oracle's own k-th / (k+1)-th score gap
   is below the fp32 error bound of a score); bf16 / FP8 workloads may differ
@@ -14,7 +14,9 @@ Tolerances (the acceptance bar of the path):
 * compressor outputs: fp32 1e-5 * (1 + |x|); bf16 half an ulp (2^-9 |x|)
   plus 1e-6; FP8 scales to 1e-6 relative and codes within one step of the
   oracle's round-to-nearest-even code (a step only where the oracle value sits
-  within 1e-5 relative of a rounding midpoint).
+  within 1e-5 relative of a rounding midpoint); MXFP4 scale bytes equal the
+  oracle's E4M3 rounding of max|x| / 6 and codes the oracle's E2M1 rounding
+  of x / scale, a neighbour only at a rounding midpoint.
 """
 from __future__ import annotations
 
@@ -28,7 +30,7 @@ from compressed_sparse_attention_compressor_b200 import workloads as Wk
 from compressed_sparse_attention_compressor_b200.csa import DevTensor
 from oracle import csa_oracle as O
 
-ATT_TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8": 2e-2}
+ATT_TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8": 2e-2, "mxfp4": 2e-2}
 BOUNDARY_GAP = 1e-3
 
 
@@ -54,6 +56,8 @@ def to_f64(t: DevTensor) -> np.ndarray:
         return t.data.double().cpu().numpy()
     if t.dtype == "bf16":
         return t.data.view(torch.bfloat16).double().cpu().numpy()
+    if t.dtype == "mxfp4":  # no torch cast for E2M1: the pinned oracle decoder
+        return O.decode(t.data.cpu().numpy(), "mxfp4", t.scale.cpu().numpy(), 16)
     v = t.data.view(torch.float8_e4m3fn).double()
     sc = t.scale.double().repeat_interleave(t.group, dim=-1)
     return (v * sc).cpu().numpy()
@@ -168,6 +172,8 @@ def check_rows(gpu_vals: np.ndarray, ref: np.ndarray, dtype: str, group: int = 0
         # round to nearest: at most half an ulp, 2^-8 |x| (x just above a power of 2)
         assert np.all(np.abs(gpu_vals - ref) <= 2.0 ** -8 * np.abs(ref) * (1 + 1e-5) + 1e-7), \
             f"bf16 rows differ by {np.abs(gpu_vals - ref).max():g}"
+    elif dtype == "mxfp4":
+        check_mxfp4_rows(ref, gpu_codes, gpu_scale)
     else:
         codes, scale = O.quantize_groups(ref, group)
         # the kernel's group maximum is an fp32 pooled value: a few fp32 ulps
@@ -186,3 +192,37 @@ def check_rows(gpu_vals: np.ndarray, ref: np.ndarray, dtype: str, group: int = 0
                 "FP8 code is not a neighbour of the value"
             mid = (a + b) / 2
             assert np.all(np.abs(x - mid) <= 1e-5 * np.abs(x) + 1e-9), "FP8 code differs away from a rounding midpoint"
+
+
+def _neighbours_at_midpoint(x, a, b, what):
+    """Codes a != b (as values) are acceptable only as the two neighbours of
+    x with x at their midpoint, up to the fp32 error of the kernel's input."""
+    assert np.all(np.minimum(a, b) <= x + 1e-9) and np.all(x <= np.maximum(a, b) + 1e-9), \
+        f"{what} code is not a neighbour of the value"
+    assert np.all(np.abs(x - (a + b) / 2) <= 1e-5 * np.abs(x) + 1e-9), f"{what} code differs away from a midpoint"
+
+
+def check_mxfp4_rows(ref, gpu_codes, gpu_scale):
+    """MXFP4 rows: the GPU's E4M3 group scales equal the oracle's rounding of
+    max|x| / 6 (a neighbour only at an E4M3 midpoint), and every element the
+    oracle's E2M1 rounding of x / (the GPU's scale) (a neighbour only at an
+    E2M1 midpoint).  ref: the oracle's fp64 rows [n][d]; gpu_codes [n][d/2],
+    gpu_scale [n][d/16] (uint8)."""
+    ref = np.asarray(ref, np.float64)
+    g = ref.reshape(ref.shape[:-1] + (-1, 16))
+    want = O.e4m3_to_f64(O.e4m3_round(np.abs(g).max(axis=-1) / O.E2M1_MAX))
+    got = O.e4m3_to_f64(gpu_scale)
+    off = got != want
+    if off.any():
+        _neighbours_at_midpoint((np.abs(g).max(axis=-1) / O.E2M1_MAX)[off], got[off], want[off], "MXFP4 scale")
+    b = np.asarray(gpu_codes, np.uint8)
+    codes = np.stack([b & 0xF, b >> 4], axis=-1).reshape(ref.shape)
+    gv = O.E2M1_VALUES[codes]
+    sc = np.repeat(got, 16, axis=-1)
+    zero = sc == 0
+    assert np.all(gv[zero] == 0), "a zero scale must store zero codes"
+    x = np.where(zero, 0.0, ref / np.where(zero, 1.0, sc))
+    ov = O.E2M1_VALUES[O.e2m1_round(x)]
+    off = (gv != ov) & ~zero
+    if off.any():
+        _neighbours_at_midpoint(np.clip(x[off], -O.E2M1_MAX, O.E2M1_MAX), gv[off], ov[off], "E2M1")

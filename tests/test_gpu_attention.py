@@ -25,6 +25,13 @@ CASES = {
     # enough queries that the per-query clusters shrink to the smallest size
     # that fits (window values then re-gathered instead of held in registers)
     "bf16_many_queries": (Wk.WORKLOADS["decode64k"], 40, 4, 1200, 128, False, True, False, 1.0),
+    # MXFP4 main KV (E2M1 + an E4M3 scale per 16 channels), dequantised to bf16 / fp32
+    "mxfp4_csa": (Wk.WORKLOADS["decode1m_fp4"], 3, 3, 4000, 128, False, True, False, 1.0),
+    "mxfp4_hca": (Wk.WORKLOADS["hybrid_hca"].scaled(kv_dtype="mxfp4", kv_group=16), 3, 2, 700, 128, True, True,
+                  False, 1.0),
+    "mxfp4_many_queries": (Wk.WORKLOADS["decode1m_fp4"], 40, 4, 1200, 128, False, True, False, 1.0),
+    "tiny_mxfp4": (Wk.WORKLOADS["tiny"].scaled(kv_dtype="mxfp4", kv_group=16), 3, 2, 1024, 128, False, True, False,
+                   1.0),
 }
 
 
@@ -35,7 +42,10 @@ def test_attention_matches_oracle(name, cuda_lib):
     d = wl.d
     sd = 1 / np.sqrt(d)
     kv_std = 1.0 if wl.kv_dtype == "fp8" else sd
-    kv = Wk.store(Wk.normal(seed, "kv", (B, cap, d), kv_std), wl.kv_dtype, 64)
+    if wl.kv_dtype == "mxfp4":
+        kv = Wk.random_mxfp4(seed, "kv", (B, cap, d))
+    else:
+        kv = Wk.store(Wk.normal(seed, "kv", (B, cap, d), kv_std), wl.kv_dtype, 64)
     act = wl.act_dtype
     swa_k = Wk.store(Wk.normal(seed, "sk", (B, swa_cap, d), sd), act)
     swa_v = Wk.store(Wk.normal(seed, "sv", (B, swa_cap, d), sd), act)

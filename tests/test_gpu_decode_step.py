@@ -26,11 +26,19 @@ DECODE = {
     "hybrid_hca": Wk.WORKLOADS["hybrid_hca"].scaled(batch=2, context=128 * 40),
     "hybrid_ratio1": Wk.WORKLOADS["hybrid_ratio1"].scaled(batch=2, context=2500, topk=300),
     "short_context": Wk.WORKLOADS["decode64k"].scaled(batch=2, context=60),  # fewer entries than top-k, window > T
+    "decode1m_fp4": Wk.WORKLOADS["decode1m_fp4"].scaled(batch=2, context=8192),
+    "decode1m_fp4_open": Wk.WORKLOADS["decode1m_fp4"].scaled(batch=2, context=8190),
+    "decode1m_fp4_simt_index": Wk.WORKLOADS["decode1m_fp4"].scaled(batch=3, context=4096, idx_dtype="bf16",
+                                                                   h_idx=32),
+    "tiny_fp4": Wk.WORKLOADS["tiny"].scaled(context=1024, kv_dtype="mxfp4", kv_group=16),
 }
 
 
 def _dtype_tol(wl):
-    return "f32" if wl.act_dtype == "f32" else wl.kv_dtype
+    # MXFP4 rows: an element of a freshly pooled row at an E2M1 rounding
+    # midpoint may take either neighbour (a full step), so even fp32
+    # workloads get the quantised tolerance
+    return "f32" if wl.act_dtype == "f32" and wl.kv_dtype != "mxfp4" else wl.kv_dtype
 
 
 @pytest.mark.parametrize("name", list(DECODE))
@@ -47,9 +55,9 @@ def test_decode_step_matches_oracle(name, cuda_lib):
         j = (t + 1) // wl.m - 1
         kv = to_f64(g.kv)
         for b in range(wl.batch):
-            fp8 = wl.kv_dtype == "fp8"
-            sc = g.kv.scale[b, j:j + 1].cpu().numpy() if fp8 else None
-            codes = g.kv.data[b, j:j + 1].cpu().numpy() if fp8 else None
+            quant = wl.kv_dtype in ("fp8", "mxfp4")
+            sc = g.kv.scale[b, j:j + 1].cpu().numpy() if quant else None
+            codes = g.kv.data[b, j:j + 1].cpu().numpy() if quant else None
             check_rows(kv[b, j:j + 1], ref["new_rows"][b][None], wl.kv_dtype, 64, sc, codes)
             if not wl.dense:
                 ki = to_f64(g.kidx)
@@ -93,6 +101,19 @@ def test_prefill_pipeline_scaled(cuda_lib):
     _run_pipeline(inp, exact=False)
 
 
+@pytest.mark.parametrize("name", ["tiny", "prefill"])
+def test_pipeline_with_mxfp4_main_kv(name, cuda_lib):
+    """The main KV stored as MXFP4 (E2M1 codes, an E4M3 scale per 16
+    channels): the compressor quantises its pooled rows, the attention
+    dequantises the cached and the new rows."""
+    if name == "tiny":
+        inp = Wk.make_tiny_pipeline_inputs(Wk.WORKLOADS["tiny"].scaled(kv_dtype="mxfp4", kv_group=16))
+        _run_pipeline(inp, exact=True)
+    else:
+        wl = Wk.WORKLOADS["prefill"].scaled(context=2048, chunk=256, kv_dtype="mxfp4", kv_group=16)
+        _run_pipeline(Wk.make_prefill_inputs(wl), exact=False)
+
+
 def _run_pipeline(inp, exact, queries=None):
     wl = inp.wl
     m, d = wl.m, wl.d
@@ -124,7 +145,7 @@ def _run_pipeline(inp, exact, queries=None):
     ref = O.pipeline(inp, qs)
     # compressor output rows and keys
     kvh, kih = to_f64(kv), to_f64(kidx)
-    f8, k8 = wl.kv_dtype == "fp8", wl.idx_dtype == "fp8"
+    f8, k8 = wl.kv_dtype in ("fp8", "mxfp4"), wl.idx_dtype == "fp8"
     check_rows(kvh[0, n0:n0 + n_new], ref["rows"], wl.kv_dtype, 64,
                kv.scale[0, n0:n0 + n_new].cpu().numpy() if f8 else None,
                kv.data[0, n0:n0 + n_new].cpu().numpy() if f8 else None)
@@ -136,5 +157,5 @@ def _run_pipeline(inp, exact, queries=None):
     swaps = 0
     for n, i in enumerate(qs):
         swaps += check_selection(gi[i], ref["scores"][n], wl.topk, exact, gs[i])
-    check_attention(got[qs], got_lse[qs], ref["out"], ref["lse"], "f32" if wl.act_dtype == "f32" else wl.kv_dtype)
+    check_attention(got[qs], got_lse[qs], ref["out"], ref["lse"], _dtype_tol(wl))
     return swaps
