@@ -136,7 +136,8 @@ attn_simt_kernel(AttnArgs a) {
                            : a.kv_dtype == kMXFP4
                                ? static_cast<const void*>(static_cast<const uint8_t*>(a.kv_scale) + gr * (D / 16))
                                : static_cast<const void*>(static_cast<const float*>(a.kv_scale) + gr * (D / a.kv_group));
-        load8(static_cast<const char*>(a.kv) + row_bytes(a.kv_dtype, gr * D), a.kv_dtype, col, srow, a.kv_group, x);
+        load8_kv(static_cast<const char*>(a.kv) + row_bytes(a.kv_dtype, gr * D), a.kv_dtype, col, srow, a.kv_group,
+                 x);
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = x[i];
       } else if (e <= -2) {

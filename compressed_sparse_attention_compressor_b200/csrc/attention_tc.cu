@@ -67,7 +67,9 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-template <bool CLUSTER>
+// FMT: storage of the compressed rows (kKvBF16 / kKvFP8 / kKvMX4); each
+// format gets its own instantiation, so a launch carries only its own gather.
+template <bool CLUSTER, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -153,7 +155,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   Src src;
   src.kv = a.kv;
   src.kv_scale = a.kv_scale;
-  src.kv_fmt = a.kv_fmt;
   src.swa_k = a.swa_k;
   src.swa_v = a.swa_v;
   src.kv_row0 = kv_row0;
@@ -162,7 +163,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   tc_fence_before();
   __syncthreads();  // s_flags[0]
   tc_fence_after();
-  attend_tile(smem, src, CLUSTER, nsr, nwr, s_flags[0] != 0, qbar, sbar, obar, dS, dO, 1, &s_flags[1],
+  attend_tile<FMT>(smem, src, CLUSTER, nsr, nwr, s_flags[0] != 0, qbar, sbar, obar, dS, dO, 1, &s_flags[1],
               &g_attn_tc_error);
   if (!CLUSTER && tid < kH) {
     pp[tid * (kD + 2)] = ml[2 * tid];
@@ -271,8 +272,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
 
 struct TcLauncher {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  bool attr[2] = {false, false};
-  int cluster_ok[17] = {0};  // per cluster size: 0 unknown, else co-resident clusters (-1: none)
+  bool attr[3][2] = {};        // per format, split / cluster kernel
+  int cluster_ok[3][17] = {};  // per format and cluster size: 0 unknown, else co-resident clusters (-1: none)
 };
 
 TcLauncher& tc_launcher() {
@@ -312,6 +313,74 @@ size_t attn_tc_workspace_bytes(int nq, int max_keys) {
 
 csa_status_t launch_attn_merge(const float* part, int nq, int n_splits, int hq, int d, const float* sink, void* out,
                                int out_dtype, float* lse, cudaStream_t stream);
+
+template <int FMT>
+csa_status_t launch_attn_fmt(TcLauncher& L, const csa_params_t* p, int nq, int max_keys, const CUtensorMap& qmap,
+                             const AttnTcArgs& a, const float* sink, const csa_tensor_t* out, float* lse,
+                             cudaStream_t stream) {
+  for (int c = 0; c < 2; ++c)
+    if (!L.attr[FMT][c]) {
+      void* fn = c ? reinterpret_cast<void*>(attn_tc_kernel<true, FMT>) : reinterpret_cast<void*>(attn_tc_kernel<false, FMT>);
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+      if (e == cudaSuccess && c) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      L.attr[FMT][c] = true;
+    }
+  // One cluster per query when its keys fit 16 CTAs of one tile each: the
+  // largest size (least work per CTA) whose nq clusters are co-resident.
+  const int rmin = attn_cluster_min(max_keys - p->window, p->window);
+  int R = 0;
+  for (int r = 16; rmin > 0 && r >= rmin && R == 0; --r) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(r, nq);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = r;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (L.cluster_ok[FMT][r] == 0) {
+      int ncl = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveClusters(&ncl, attn_tc_kernel<true, FMT>, &cfg);
+      L.cluster_ok[FMT][r] = (e == cudaSuccess && ncl >= 1) ? ncl : -1;
+      cudaGetLastError();
+    }
+    if (L.cluster_ok[FMT][r] >= nq || (r == rmin && L.cluster_ok[FMT][r] > 0)) R = r;
+  }
+  if (R > 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(R, nq);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = R;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+      prof_begin(stream);
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true, FMT>, qmap, a);
+      if (e != cudaSuccess) {
+        check_launch("attn_tc_cluster_kernel", stream);
+        return set_error(CSA_ERR_CUDA, "attn_tc_kernel (cluster) launch: %s", cudaGetErrorString(e));
+      }
+      return check_launch("attn_tc_cluster_kernel", stream);
+    }
+  }
+  prof_begin(stream);
+  attn_tc_kernel<false, FMT><<<dim3(a.splits, nq), kThreads, kSmem, stream>>>(qmap, a);
+  csa_status_t st = check_launch("attn_tc_kernel", stream);
+  if (st != CSA_OK) return st;
+  return launch_attn_merge(a.part, nq, a.splits, kH, kD, sink, out->data, out->dtype, lse, stream);
+}
+
 
 csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
                                  int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
@@ -353,67 +422,9 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
   a.out = out->data;
   a.out_dtype = out->dtype;
   a.lse = lse;
-  for (int c = 0; c < 2; ++c)
-    if (!L.attr[c]) {
-      void* fn = c ? reinterpret_cast<void*>(attn_tc_kernel<true>) : reinterpret_cast<void*>(attn_tc_kernel<false>);
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-      if (e == cudaSuccess && c) e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      L.attr[c] = true;
-    }
-  // One cluster per query when its keys fit 16 CTAs of one tile each: the
-  // largest size (least work per CTA) whose nq clusters are co-resident.
-  const int rmin = attn_cluster_min(max_keys - p->window, p->window);
-  int R = 0;
-  for (int r = 16; rmin > 0 && r >= rmin && R == 0; --r) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(r, nq);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = r;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (L.cluster_ok[r] == 0) {
-      int ncl = 0;
-      const cudaError_t e = cudaOccupancyMaxActiveClusters(&ncl, attn_tc_kernel<true>, &cfg);
-      L.cluster_ok[r] = (e == cudaSuccess && ncl >= 1) ? ncl : -1;
-      cudaGetLastError();
-    }
-    if (L.cluster_ok[r] >= nq || (r == rmin && L.cluster_ok[r] > 0)) R = r;
-  }
-  if (R > 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(R, nq);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = R;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    {
-      prof_begin(stream);
-      const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, qmap, a);
-      if (e != cudaSuccess) {
-        check_launch("attn_tc_cluster_kernel", stream);
-        return set_error(CSA_ERR_CUDA, "attn_tc_kernel (cluster) launch: %s", cudaGetErrorString(e));
-      }
-      return check_launch("attn_tc_cluster_kernel", stream);
-    }
-  }
-  prof_begin(stream);
-  attn_tc_kernel<false><<<dim3(a.splits, nq), kThreads, kSmem, stream>>>(qmap, a);
-  csa_status_t st = check_launch("attn_tc_kernel", stream);
-  if (st != CSA_OK) return st;
-  return launch_attn_merge(a.part, nq, a.splits, kH, kD, sink, out->data, out->dtype, lse, stream);
+  if (a.kv_fmt == kKvMX4) return launch_attn_fmt<kKvMX4>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
+  if (a.kv_fmt == kKvFP8) return launch_attn_fmt<kKvFP8>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
+  return launch_attn_fmt<kKvBF16>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
 }
 
 uint32_t attn_tc_take_error() {

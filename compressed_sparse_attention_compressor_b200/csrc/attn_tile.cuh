@@ -57,8 +57,11 @@ __device__ __forceinline__ void put_chunk(uint8_t* tile, int r, int e, uint4 v) 
   *reinterpret_cast<uint4*>(tile + blk * (kTK * 128) + sw128_offset(r, ch)) = v;
 }
 
+// Two floats -> two bf16 (round to nearest even), a in the low half: one
+// packed conversion.
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  return static_cast<uint32_t>(f32_to_bf16_bits(a)) | (static_cast<uint32_t>(f32_to_bf16_bits(b)) << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Storage of the compressed rows.
@@ -70,8 +73,7 @@ constexpr int kKvMX4 = 2;   // E2M1 codes (two per byte), one E4M3 scale byte pe
 // kv_row0 + e, e <= -2 window slot sw_row0 + (-2 - e), e = -1 nothing.
 struct Src {
   const void* kv;
-  const void* kv_scale;
-  int kv_fmt;             // kKvBF16 / kKvFP8 / kKvMX4
+  const void* kv_scale;   // FP8: fp32 scales; MXFP4: E4M3 scale bytes
   const uint16_t* swa_k;
   const uint16_t* swa_v;
   int64_t kv_row0;
@@ -87,11 +89,14 @@ struct QChunk {
   uint32_t s;
 };
 
-__device__ __forceinline__ int q_chunks_per_row(int fmt) { return fmt == kKvMX4 ? kD / 32 : kD / 16; }
+// 16-byte chunks of one compressed row: bf16 64, FP8 32, MXFP4 16.
+template <int FMT>
+constexpr int chunks_per_row() { return FMT == kKvBF16 ? kD / 8 : FMT == kKvFP8 ? kD / 16 : kD / 32; }
 
+template <int FMT>
 __device__ __forceinline__ QChunk load_qchunk(const Src& a, int64_t gr, int c) {
   QChunk q;
-  if (a.kv_fmt == kKvMX4) {
+  if constexpr (FMT == kKvMX4) {
     q.u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.kv) + gr * (kD / 2)) + c);
     q.s = __ldg(reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(a.kv_scale) + gr * (kD / 16)) + c);
   } else {
@@ -103,9 +108,10 @@ __device__ __forceinline__ QChunk load_qchunk(const Src& a, int64_t gr, int c) {
 
 // Dequantises chunk c of a row into tile row r as bf16 (exact for MXFP4: an
 // E2M1 value times an E4M3 scale has at most 5 significant bits).
-__device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QChunk& q, int fmt) {
+template <int FMT>
+__device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QChunk& q) {
   const uint32_t w[4] = {q.u.x, q.u.y, q.u.z, q.u.w};
-  if (fmt == kKvMX4) {
+  if constexpr (FMT == kKvMX4) {
     const float s0 = e4m3_to_f32(static_cast<uint8_t>(q.s & 0xFF)), s1 = e4m3_to_f32(static_cast<uint8_t>(q.s >> 8));
 #pragma unroll
     for (int i = 0; i < 4; ++i) {  // word i: elements 8i .. 8i+7, nibble k = element 8i + k
@@ -135,11 +141,12 @@ __device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QC
 // (compressed entries and window keys); which = 1: only the window rows,
 // from the value ring (compressed rows are their own values).  Loads are
 // issued in batches of 8 per thread before any of them is used.
+template <int FMT>
 __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int which) {
   constexpr int B = 8;
-  if (a.kv_fmt != kKvBF16 && which == 0) {
+  if (FMT != kKvBF16 && which == 0) {
     // quantised entries: tpr tasks of one 16-byte chunk per row
-    const int tpr = q_chunks_per_row(a.kv_fmt);
+    constexpr int tpr = chunks_per_row<FMT>();
     for (int t0 = static_cast<int>(threadIdx.x); t0 < kTK * tpr; t0 += kNT * B) {
       QChunk q[B];
 #pragma unroll
@@ -149,14 +156,14 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
         const int32_t e = task < kTK * tpr ? ent[r] : -1;
         q[b].u = make_uint4(0, 0, 0, 0);
         q[b].s = 0u;
-        if (e >= 0) q[b] = load_qchunk(a, a.kv_row0 + e, c);
+        if (e >= 0) q[b] = load_qchunk<FMT>(a, a.kv_row0 + e, c);
       }
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const int task = t0 + b * kNT;
         const int r = task / tpr, c = task % tpr;
         if (task >= kTK * tpr || ent[r] < 0) continue;
-        put_qchunk(tile, r, c, q[b], a.kv_fmt);
+        put_qchunk<FMT>(tile, r, c, q[b]);
       }
     }
   }
@@ -172,7 +179,7 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
       v[b] = make_uint4(0, 0, 0, 0);
       put[b] = task < kTK * 64;
       if (e >= 0) {
-        if (a.kv_fmt != kKvBF16 || which == 1) put[b] = false;  // quantised rows done above; compressed rows keep their keys
+        if (FMT != kKvBF16 || which == 1) put[b] = false;  // quantised rows done above; compressed rows keep their keys
         else v[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + (a.kv_row0 + e) * kD) + c8);
       } else if (e <= -2) {
         const uint16_t* src = (which == 0 ? a.swa_k : a.swa_v) + (a.sw_row0 + (-2 - e)) * kD;
@@ -201,9 +208,10 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
 // used; the window rows' values go to vw[] (registers) in the same batch
 // (nwr <= 16), to replace the keys once the logits are out.  Rows
 // [nsr + nwr, nk16) are zeroed (the PV product reads them with weight 0).
+template <int FMT>
 __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, int nsr, int nwr, int nk16,
                                uint4 (&vw)[4]) {
-  const int per_sel = a.kv_fmt == kKvBF16 ? 64 : q_chunks_per_row(a.kv_fmt);  // 16-byte chunks per selected row
+  constexpr int per_sel = chunks_per_row<FMT>();  // 16-byte chunks per selected row
   const int T1 = nsr * per_sel, T = T1 + nwr * 64;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
@@ -227,8 +235,8 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
         const int32_t e = ent[r];
         if (e >= 0) {
           const int64_t gr = a.kv_row0 + e;
-          if (a.kv_fmt != kKvBF16)
-            q[b] = load_qchunk(a, gr, c);
+          if constexpr (FMT != kKvBF16)
+            q[b] = load_qchunk<FMT>(a, gr, c);
           else
             q[b].u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + gr * kD) + c);
         }
@@ -243,8 +251,8 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
       const int task = t0 + b * kNT;
       if (task < T1) {
         const int r = task / per_sel, c = task % per_sel;
-        if (a.kv_fmt != kKvBF16)
-          put_qchunk(tile, r, c, q[b], a.kv_fmt);
+        if constexpr (FMT != kKvBF16)
+          put_qchunk<FMT>(tile, r, c, q[b]);
         else
           put_chunk(tile, r, c * 8, q[b].u);
       } else if (task < T) {
@@ -269,6 +277,7 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
 // ml = (max, sum) per head at oML and O^T in TMEM columns dO .. dO + 255
 // (unnormalised, lanes = dims mod 128); on a bounded-wait timeout *fail = 1
 // and bit 0 of *err is set.
+template <int FMT>
 __device__ void attend_tile(uint8_t* smem, const Src& s, bool contiguous, int nsr, int nwr, bool any_window,
                             uint64_t* qbar, uint64_t* sbar, uint64_t* obar, uint32_t dS, uint32_t dO, int bar,
                             int* fail, uint32_t* err) {
@@ -281,8 +290,8 @@ __device__ void attend_tile(uint8_t* smem, const Src& s, bool contiguous, int ns
   const int nk16 = contiguous ? ((nsr + nwr + 15) & ~15) : kTK;  // keys the PV product covers
   const bool vregs = contiguous && nwr <= 16;                       // window values held in registers
   uint4 vw[4];
-  if (vregs) gather_cluster(Kt, ent, s, nsr, nwr, nk16, vw);
-  else gather_rows(Kt, ent, s, 0);
+  if (vregs) gather_cluster<FMT>(Kt, ent, s, nsr, nwr, nk16, vw);
+  else gather_rows<FMT>(Kt, ent, s, 0);
   fence_proxy_async_smem();
   tc_fence_before();
   named_barrier(bar, kNT);
@@ -335,7 +344,7 @@ __device__ void attend_tile(uint8_t* smem, const Src& s, bool contiguous, int ns
       if (task < nwr * 64) put_chunk(Kt, nsr + (task >> 6), (task & 63) * 8, vw[b]);
     }
   } else if (any_window) {
-    gather_rows(Kt, ent, s, 1);
+    gather_rows<FMT>(Kt, ent, s, 1);
   }
   // softmax statistics and P^T: four threads per head, 32 keys each
   {

@@ -72,8 +72,7 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
 // --------------------------------------------------------------------------
 // Loads elements [col, col+8) of a row into v (fp32).  For FP8, `scale`
 // points at the row's fp32 group scales and `group` is the group length
-// (a multiple of 8, so the 8 elements share one scale); for MXFP4 at the
-// row's E4M3 scale bytes (group 16), with `row` at the row's first code byte.
+// (a multiple of 8, so the 8 elements share one scale).  (MXFP4 rows: load8_kv.)
 __device__ __forceinline__ void load8(const void* row, int dtype, int col, const void* scale, int group,
                                       float v[8]) {
   if (dtype == kF32) {
@@ -89,11 +88,6 @@ __device__ __forceinline__ void load8(const void* row, int dtype, int col, const
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
-  } else if (dtype == kMXFP4) {
-    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(row) + col / 2));
-    const float s = e4m3_to_f32(__ldg(static_cast<const uint8_t*>(scale) + col / 16));
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = e2m1_to_f32(u >> (4 * e)) * s;
   } else {
     uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(row) + col));
     float s = __ldg(static_cast<const float*>(scale) + col / group);
@@ -105,6 +99,21 @@ __device__ __forceinline__ void load8(const void* row, int dtype, int col, const
       v[4 * i + 0] = lo.x * s; v[4 * i + 1] = lo.y * s;
       v[4 * i + 2] = hi.x * s; v[4 * i + 3] = hi.y * s;
     }
+  }
+}
+
+// load8 for compressed main-KV rows, which may also be MXFP4: `row` at the
+// row's first code byte, `scale` at its E4M3 scale bytes (group 16).  Kept
+// apart from load8 so that the activation loads carry no MXFP4 code.
+__device__ __forceinline__ void load8_kv(const void* row, int dtype, int col, const void* scale, int group,
+                                         float v[8]) {
+  if (dtype == kMXFP4) {
+    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(row) + col / 2));
+    const float s = e4m3_to_f32(__ldg(static_cast<const uint8_t*>(scale) + col / 16));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = e2m1_to_f32(u >> (4 * e)) * s;
+  } else {
+    load8(row, dtype, col, scale, group, v);
   }
 }
 
@@ -127,9 +136,6 @@ __device__ __forceinline__ void store8(void* row, int dtype, int col, const floa
 __device__ __forceinline__ float load1(const void* row, int dtype, int col, const void* scale, int group) {
   if (dtype == kF32) return __ldg(static_cast<const float*>(row) + col);
   if (dtype == kBF16) return bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(row) + col));
-  if (dtype == kMXFP4)
-    return e2m1_to_f32(__ldg(static_cast<const uint8_t*>(row) + col / 2) >> (4 * (col & 1))) *
-           e4m3_to_f32(__ldg(static_cast<const uint8_t*>(scale) + col / 16));
   return e4m3_to_f32(__ldg(static_cast<const uint8_t*>(row) + col)) *
          __ldg(static_cast<const float*>(scale) + col / group);
 }

@@ -437,6 +437,7 @@ __device__ __forceinline__ void block_sum2(uint32_t& a, uint32_t& b, uint32_t* s
 // for W_IK (d x 128, 16-aligned; the idle stage ring); scratch: d + 256
 // floats; wbar: an initialised mbarrier.  The stores are visible to this
 // CTA's later TMA loads (and to every later kernel) when it returns.
+template <bool KV_MX4>
 __device__ void append_block(const AppendArgs& p, int r, int64_t cap, uint8_t* wbuf, float* scratch,
                              uint64_t* wbar, Shared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -495,7 +496,7 @@ __device__ void append_block(const AppendArgs& p, int r, int64_t cap, uint8_t* w
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] = 0.f;
       }
-      store_pooled8(p.kv, row, col, v, valid);
+      store_pooled8<KV_MX4>(p.kv, row, col, v, valid);
     }
     // indexer key = pooled . W_IK (fp32 pooled row, before storage rounding):
     // thread (j, half) sums half of the d channels of output j
@@ -549,11 +550,22 @@ __device__ void append_block(const AppendArgs& p, int r, int64_t cap, uint8_t* w
   __syncthreads();
 }
 
-template <bool FP8>
+// Launch modes.  Each is its own instantiation, so that a launch carries
+// only its own code: every CTA fetches the kernel's instructions cold.
+constexpr int kModePlain = 0;      // top-k of the visible entries
+constexpr int kModeBmax = 1;       // ... and the block maxima (a.bmax)
+constexpr int kModePool = 2;       // top-k inside a candidate pool (a.pool)
+constexpr int kModeAppend = 3;     // decode step: append the token first (a.ap), main KV not MXFP4
+constexpr int kModeAppendMx4 = 4;  // ... main KV in MXFP4
+constexpr int kModes = 5;
+
+template <bool FP8, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap smap,
                      IdxArgs a) {
   using C = Cfg<FP8>;
+  constexpr bool POOL = MODE == kModePool, BMAX = MODE == kModeBmax;
+  constexpr bool APPEND = MODE == kModeAppend || MODE == kModeAppendMx4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   Shared& sh = *reinterpret_cast<Shared*>(smem + C::oMisc);
@@ -573,18 +585,21 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.x / a.chunks, c = blockIdx.x % a.chunks;
-  const int64_t n_raw = a.pool ? pool_positions(a, r, sh)
-                               : a.append ? (a.ap.pos[r] + 1) / a.ap.m : static_cast<int64_t>(a.n_visible[r]);
-  const int64_t n = min(max(n_raw, int64_t(0)), a.pool ? static_cast<int64_t>(a.pool_blocks) * a.pblock : a.cap);
-  const int32_t* prow = a.pool ? a.pool + static_cast<int64_t>(r) * a.pool_blocks : nullptr;
+  int64_t n_raw;
+  if constexpr (POOL)
+    n_raw = pool_positions(a, r, sh);
+  else
+    n_raw = APPEND ? (a.ap.pos[r] + 1) / a.ap.m : static_cast<int64_t>(a.n_visible[r]);
+  const int64_t n = min(max(n_raw, int64_t(0)), POOL ? static_cast<int64_t>(a.pool_blocks) * a.pblock : a.cap);
+  const int32_t* prow = POOL ? a.pool + static_cast<int64_t>(r) * a.pool_blocks : nullptr;
   // pool position -> entry id (identity without a pool)
   auto entry_of = [&](uint32_t j) -> int32_t {
-    if (!prow) return static_cast<int32_t>(j);
+    if constexpr (!POOL) return static_cast<int32_t>(j);
     return __ldg(prow + j / a.pblock) * a.pblock + static_cast<int32_t>(j % a.pblock);
   };
   const int tiles_req = static_cast<int>((n + kTileM - 1) / kTileM);
   int t0, t1;
-  if (a.append && a.chunks > 1) {
+  if (APPEND && a.chunks > 1) {
     // the last chunk (whose CTA appends the token first) is shorter by `shrink` tiles
     const int per = (tiles_req + a.chunks - 1) / a.chunks;
     const int last = min(tiles_req, max(1, per - a.ap.shrink));
@@ -619,11 +634,13 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     fence_barrier_init();
   }
   __syncthreads();
-  if (a.append && c == a.chunks - 1)
-    append_block(a.ap, r, a.cap, smem + C::oStages, reinterpret_cast<float*>(smem + C::oHist), abar, sh);
+  if constexpr (APPEND)
+    if (c == a.chunks - 1)
+      append_block<MODE == kModeAppendMx4>(a.ap, r, a.cap, smem + C::oStages,
+                                           reinterpret_cast<float*>(smem + C::oHist), abar, sh);
 
   // ================= phase 1: stream the keys, scores into TMEM =================
-  if (warp == 0 && prow) {
+  if (POOL && warp == 0) {
     // candidate-pool mode: per stage, lane l loads the pblock-row box of
     // slot q0 + l (and, FP8, its row scales); a stage's slots are <= 32
     if (lane == 0) {
@@ -1001,7 +1018,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
 
     if (n <= k) {
       copy_scores();
-      if (a.bmax) write_block_max();
+      if constexpr (BMAX) write_block_max();
       __syncthreads();
       for (int i = tid; i < nloc; i += kThreads) {
         oi[base + i] = entry_of(static_cast<uint32_t>(base + i));
@@ -1026,7 +1043,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       // arrive, copy the scores while the request's slower CTAs finish, wait
       request_arrive(&bar[0]);
       copy_scores();
-      if (a.bmax) write_block_max();
+      if constexpr (BMAX) write_block_max();
       bool alive = request_wait(&bar[0], a.chunks, sh);
       uint32_t shift = 20, prefix = 0;
       if (alive) {
@@ -1244,7 +1261,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
 struct Launcher {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   int sms = 0;
-  bool attr_set[2] = {false, false};
+  bool attr_set[2][kModes] = {};  // per key format and launch mode
 };
 
 Launcher& launcher() {
@@ -1403,11 +1420,20 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.eq = reinterpret_cast<uint2*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 8));
 
   const int smem = fp8 ? Cfg<true>::kSmem : Cfg<false>::kSmem;
-  void* fn = fp8 ? reinterpret_cast<void*>(index_topk_tc_kernel<true>) : reinterpret_cast<void*>(index_topk_tc_kernel<false>);
-  if (!L.attr_set[fp8 ? 1 : 0]) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int mode = pool ? kModePool : bmax ? kModeBmax
+                   : ap ? (ap->kv.dtype == kMXFP4 ? kModeAppendMx4 : kModeAppend) : kModePlain;
+  using Kern = void (*)(CUtensorMap, CUtensorMap, IdxArgs);
+  const Kern kerns[2][kModes] = {
+      {index_topk_tc_kernel<false, 0>, index_topk_tc_kernel<false, 1>, index_topk_tc_kernel<false, 2>,
+       index_topk_tc_kernel<false, 3>, index_topk_tc_kernel<false, 4>},
+      {index_topk_tc_kernel<true, 0>, index_topk_tc_kernel<true, 1>, index_topk_tc_kernel<true, 2>,
+       index_topk_tc_kernel<true, 3>, index_topk_tc_kernel<true, 4>}};
+  const Kern fn = kerns[fp8 ? 1 : 0][mode];
+  if (!L.attr_set[fp8 ? 1 : 0][mode]) {
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
     if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    L.attr_set[fp8 ? 1 : 0] = true;
+    L.attr_set[fp8 ? 1 : 0][mode] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch * ch);
@@ -1420,8 +1446,7 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   prof_begin(stream);
-  cudaError_t e = fp8 ? cudaLaunchKernelEx(&cfg, index_topk_tc_kernel<true>, map, smap, a)
-                      : cudaLaunchKernelEx(&cfg, index_topk_tc_kernel<false>, map, smap, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, map, smap, a);
   if (e != cudaSuccess) {
     check_launch("index_topk_tc_kernel", stream);
     return set_error(CSA_ERR_CUDA, "index_topk_tc_kernel launch: %s", cudaGetErrorString(e));

@@ -73,9 +73,11 @@ __device__ __forceinline__ void pool8(RowC rowC, RowZ rowZ, int in_dtype, int m,
 // KV cache"): the group's scale is the E4M3 value nearest max|x| / 6 (so
 // that max|x| lands on the largest E2M1 magnitude), each element the E2M1
 // value nearest x / scale, saturating at 6; an all-zero scale stores zeros.
+// MX4 = false leaves the MXFP4 branch out (callers that never store MXFP4).
+template <bool MX4 = true>
 __device__ __forceinline__ void store_pooled8(const OutSpec& o, int64_t row, int col, const float v[8],
                                               bool valid) {
-  if (o.dtype == kMXFP4) {
+  if (MX4 && o.dtype == kMXFP4) {
     float amax = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
