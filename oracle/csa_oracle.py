@@ -367,6 +367,47 @@ def reindex_topk(q_idx: np.ndarray, w: np.ndarray, keys: np.ndarray, pool: np.nd
     return ids.astype(np.int64), s
 
 
+def csa2_group_selections(modes, layer_q_idx, layer_w, keys, block: int, pool_blocks: int, k: int):
+    """The index selection every layer of one CSA2 layer group attends over,
+    for one query.  Tech-report tour, chapter "Compressed Sparse Attention
+    2": section "Full, Reindex, and Reuse" (modes table: Full computes fresh
+    Top-K indices; Reindex keeps the shared main KV and indexer K and
+    rescores the candidate pool with its own indexer query; Reuse takes the
+    latest selection and runs no indexer) and section "The Hierarchical Sparse
+    Indexer" (the first Full layer of the group builds the candidate pool
+    that later indexers search).
+
+    modes: "full" / "reindex" / "reuse" per layer, the first "full" or
+    "reindex"; layer_q_idx[l] [h_idx][d_idx] and layer_w[l] [h_idx] are that
+    layer's indexer query and weights (unused for Reuse); keys [n_vis][d_idx]
+    the group's shared visible indexer keys.  Returns (selections, pool):
+    selections[l] the entry ids (-1 padded) layer l attends over; pool the
+    block ids the first Full layer kept (None if the group has no Full
+    layer, which then needs no Reindex layer either).
+
+    Reading: a Reindex layer before the group's first Full layer has no pool
+    to rescore, so the first indexing layer must be Full or the group must
+    have no Reindex layer."""
+    sel, pool, latest = [], None, None
+    for l, mode in enumerate(modes):
+        if mode == "full":
+            s = index_scores(layer_q_idx[l], layer_w[l], keys)
+            latest = topk(s, k)
+            if pool is None:
+                pool = candidate_pool(s, block, pool_blocks)
+        elif mode == "reindex":
+            if pool is None:
+                raise ValueError("a Reindex layer needs a preceding Full layer's pool")
+            latest, _ = reindex_topk(layer_q_idx[l], layer_w[l], keys, pool, block, k)
+        elif mode == "reuse":
+            if latest is None:
+                raise ValueError("a Reuse layer needs a preceding Full or Reindex layer")
+        else:
+            raise ValueError(mode)
+        sel.append(np.asarray(latest, np.int64).copy())
+    return sel, pool
+
+
 # ===========================================================================
 # a4 / a5: sparse (or dense) attention + sliding window + sink, one softmax
 # ===========================================================================

@@ -18,6 +18,7 @@ FULL = {
     "hybrid_csa": [0, 5],
     "hybrid_hca": [0, 7],
     "hybrid_ratio1": [3],
+    "decode1m_fp4": [1, 2],
 }
 
 

@@ -519,3 +519,45 @@ def test_mxfp4_round_trip_error_bound_and_layout():
     # an all-zero group keeps a zero scale and zero codes
     c, sc = O.quantize_mxfp4(np.zeros((1, 32)))
     assert np.all(c == 0) and np.all(sc == 0)
+
+
+# ---------------------------------------------------------------- CSA2 layer modes
+def _group_inputs(seed, n=300, H=3, D=8, layers=6):
+    g = np.random.default_rng(seed)
+    keys = g.standard_normal((n, D))
+    qs = g.standard_normal((layers, H, D))
+    ws = g.uniform(0, 1, (layers, H))
+    return keys, qs, ws
+
+
+def test_csa2_reuse_layers_repeat_the_latest_selection():
+    keys, qs, ws = _group_inputs(31)
+    modes = ["full", "reuse", "reuse", "reindex", "reuse", "reuse"]
+    sel, pool = O.csa2_group_selections(modes, qs, ws, keys, 8, 10, 16)
+    assert np.array_equal(sel[1], sel[0]) and np.array_equal(sel[2], sel[0])
+    assert np.array_equal(sel[4], sel[3]) and np.array_equal(sel[5], sel[3])
+    # the Full layer is the plain top-k of its own query; the pool is its blocks
+    assert np.array_equal(sel[0], O.topk(O.index_scores(qs[0], ws[0], keys), 16))
+    assert np.array_equal(pool, O.candidate_pool(O.index_scores(qs[0], ws[0], keys), 8, 10))
+    # the Reindex layer's picks lie inside the pool
+    inside = set(O.pool_entries(pool, 8, keys.shape[0]).tolist())
+    assert set(sel[3][sel[3] >= 0].tolist()) <= inside
+
+
+def test_csa2_reindex_over_a_pool_of_every_block_equals_a_full_layer():
+    keys, qs, ws = _group_inputs(32, n=203)
+    nb = (203 + 7) // 8
+    sel, _ = O.csa2_group_selections(["full", "reindex"], qs, ws, keys, 8, nb, 20)
+    full, _ = O.csa2_group_selections(["full", "full"], qs, ws, keys, 8, nb, 20)
+    assert np.array_equal(np.sort(sel[1]), np.sort(full[1]))
+
+
+def test_csa2_pool_comes_from_the_first_full_layer_only():
+    keys, qs, ws = _group_inputs(33)
+    sel, pool = O.csa2_group_selections(["full", "full", "reindex"], qs, ws, keys, 8, 6, 12)
+    assert np.array_equal(pool, O.candidate_pool(O.index_scores(qs[0], ws[0], keys), 8, 6))
+    assert not np.array_equal(pool, O.candidate_pool(O.index_scores(qs[1], ws[1], keys), 8, 6))
+    with pytest.raises(ValueError):
+        O.csa2_group_selections(["reindex"], qs, ws, keys, 8, 6, 12)
+    with pytest.raises(ValueError):
+        O.csa2_group_selections(["reuse"], qs, ws, keys, 8, 6, 12)
