@@ -46,7 +46,8 @@ constexpr int kTmemCols = 512;
 // shared-memory layout: the attention tile (attn_tile.cuh), then this kernel's
 constexpr int oBars = kTileSmem;
 constexpr int oMisc = oBars + 64;
-constexpr int kSmem = oMisc + 64 + 1024;
+constexpr int oLut = oMisc + 64;  // MXFP4 code-byte table, 256 x bf16x2
+constexpr int kSmem = oLut + 1024 + 1024;
 
 __device__ uint32_t g_attn_tc_error = 0;
 
@@ -143,6 +144,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     ent[tid] = e;
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + oLut));
   __syncthreads();
   if (tid == 0) {
     mbar_arrive_expect_tx(qbar, kH * kD * 2);
@@ -155,6 +157,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   Src src;
   src.kv = a.kv;
   src.kv_scale = a.kv_scale;
+  src.lut = reinterpret_cast<const uint32_t*>(smem + oLut);
   src.swa_k = a.swa_k;
   src.swa_v = a.swa_v;
   src.kv_row0 = kv_row0;

@@ -74,6 +74,7 @@ constexpr int kKvMX4 = 2;   // E2M1 codes (two per byte), one E4M3 scale byte pe
 struct Src {
   const void* kv;
   const void* kv_scale;   // FP8: fp32 scales; MXFP4: E4M3 scale bytes
+  const uint32_t* lut;    // MXFP4: shared-memory table, code byte -> its two E2M1 values as bf16x2
   const uint16_t* swa_k;
   const uint16_t* swa_v;
   int64_t kv_row0;
@@ -106,20 +107,32 @@ __device__ __forceinline__ QChunk load_qchunk(const Src& a, int64_t gr, int c) {
   return q;
 }
 
-// Dequantises chunk c of a row into tile row r as bf16 (exact for MXFP4: an
-// E2M1 value times an E4M3 scale has at most 5 significant bits).
+// The MXFP4 table: byte b -> bf16x2 (E2M1 value of its low nibble, of its
+// high nibble).  All threads of the block; visible after the next barrier.
+__device__ __forceinline__ void fill_mx4_lut(uint32_t* lut) {
+  for (int b = static_cast<int>(threadIdx.x); b < 256; b += static_cast<int>(blockDim.x))
+    lut[b] = pack_bf16(e2m1_to_f32(static_cast<uint32_t>(b) & 0xFu), e2m1_to_f32(static_cast<uint32_t>(b) >> 4));
+}
+
+// Dequantises chunk c of a row into tile row r as bf16.  MXFP4: a table
+// lookup per code byte and one bf16x2 multiply by the group scale, exact (an
+// E2M1 value times an E4M3 scale has at most 5 significant bits, and both
+// factors are exact in bf16).
 template <int FMT>
-__device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QChunk& q) {
+__device__ __forceinline__ void put_qchunk(uint8_t* tile, int r, int c, const QChunk& q, const uint32_t* lut) {
   const uint32_t w[4] = {q.u.x, q.u.y, q.u.z, q.u.w};
   if constexpr (FMT == kKvMX4) {
-    const float s0 = e4m3_to_f32(static_cast<uint8_t>(q.s & 0xFF)), s1 = e4m3_to_f32(static_cast<uint8_t>(q.s >> 8));
+    const __nv_bfloat162 s0 = __float2bfloat162_rn(e4m3_to_f32(static_cast<uint8_t>(q.s & 0xFF)));
+    const __nv_bfloat162 s1 = __float2bfloat162_rn(e4m3_to_f32(static_cast<uint8_t>(q.s >> 8)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // word i: elements 8i .. 8i+7, nibble k = element 8i + k
-      const float sc = i < 2 ? s0 : s1;
+    for (int i = 0; i < 4; ++i) {  // word i: elements 8i .. 8i+7 (byte k: elements 8i+2k, 8i+2k+1)
       uint32_t o[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        o[k] = pack_bf16(e2m1_to_f32(w[i] >> (8 * k)) * sc, e2m1_to_f32(w[i] >> (8 * k + 4)) * sc);
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t two = lut[(w[i] >> (8 * k)) & 0xFFu];
+        const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&two), i < 2 ? s0 : s1);
+        o[k] = *reinterpret_cast<const uint32_t*>(&v);
+      }
       put_chunk(tile, r, c * 32 + i * 8, make_uint4(o[0], o[1], o[2], o[3]));
     }
   } else {
@@ -163,7 +176,7 @@ __device__ void gather_rows(uint8_t* tile, const int32_t* ent, const Src& a, int
         const int task = t0 + b * kNT;
         const int r = task / tpr, c = task % tpr;
         if (task >= kTK * tpr || ent[r] < 0) continue;
-        put_qchunk<FMT>(tile, r, c, q[b]);
+        put_qchunk<FMT>(tile, r, c, q[b], a.lut);
       }
     }
   }
@@ -252,7 +265,7 @@ __device__ void gather_cluster(uint8_t* tile, const int32_t* ent, const Src& a, 
       if (task < T1) {
         const int r = task / per_sel, c = task % per_sel;
         if constexpr (FMT != kKvBF16)
-          put_qchunk<FMT>(tile, r, c, q[b]);
+          put_qchunk<FMT>(tile, r, c, q[b], a.lut);
         else
           put_chunk(tile, r, c * 8, q[b].u);
       } else if (task < T) {
