@@ -237,3 +237,36 @@ def test_pool_full_size_decode1m(cuda_lib):
     for i in range(B):
         check_reindex_row(ri[i], rs[i], pool[i], block, keys_of(kidx, i, n_vis[i]), q2d[i], w2[i], wl.topk,
                           exact=False)
+
+
+@pytest.mark.parametrize("per_request", [False, True])
+def test_pool_and_reindex_edge_cases(per_request, cuda_lib):
+    """Requests with no visible entry, fewer entries than one block, exactly
+    one block, and exactly pool_blocks blocks; k larger than the candidates."""
+    wl = Wk.WORKLOADS["decode64k"].scaled(topk=64)
+    B, cap, block, pool_blocks = 4, 2048, 8, 16
+    seed = 4900
+    kidx, q_idx, w = integer_inputs(seed, wl, B, B, cap, (), block)
+    n_vis = np.array([0, 5, 8, block * pool_blocks], np.int32)
+    q_req = None if per_request else np.arange(B, dtype=np.int32)
+    gp, gi = gpu_pool(wl, q_idx, w, kidx, B, cap, q_req, n_vis, block, pool_blocks)
+    qd = O.decode_stored(q_idx)
+    pools = []
+    for i in range(B):
+        keys = keys_of(kidx, i, n_vis[i])
+        s = O.index_scores(qd[i], w[i], keys) if n_vis[i] else np.zeros(0)
+        ref_pool = O.candidate_pool(s, block, pool_blocks) if n_vis[i] else np.full(pool_blocks, -1)
+        assert np.array_equal(gp[i], ref_pool), f"request {i}: pool"
+        assert np.array_equal(np.sort(gi[i]), np.sort(O.topk(s, wl.topk))), f"request {i}: top-k"
+        pools.append(ref_pool)
+    pool = np.stack(pools).astype(np.int32)
+    _, q2, w2 = integer_inputs(seed + 1, wl, B, B, cap, (), block)
+    ri, rs = gpu_reindex(wl, q2, w2, kidx, B, cap, q_req, n_vis, pool, block)
+    q2d = O.decode_stored(q2)
+    for i in range(B):
+        keys = keys_of(kidx, i, n_vis[i])
+        ent = O.pool_entries(pool[i], block, int(n_vis[i]))
+        if ent.shape[0] == 0:
+            assert np.all(ri[i] == -1) and np.all(np.isneginf(rs[i])), f"request {i}: empty pool"
+            continue
+        check_reindex_row(ri[i], rs[i], pool[i], block, keys, q2d[i], w2[i], wl.topk, exact=True)
