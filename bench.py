@@ -111,13 +111,12 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-def load_traffic(name):
-    """DRAM bytes per launch from the committed ncu summary of a kernel
-    (profiles/<kernel>_<workload>.md), if the kernel's source is unchanged
-    since the capture (else None)."""
-    import glob
-    import re
-    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{name}_*.md"))):
+def load_traffic(name, workload):
+    """DRAM bytes per launch from the committed ncu summary of a kernel on a
+    workload (profiles/<kernel>_<workload>.md), if the kernel's source is
+    unchanged since the capture (else None)."""
+    for path in [os.path.join(ROOT, "profiles", f"{name}_{workload}.md")]:
+        import re
         try:
             text = open(path).read()
             nbytes = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", text).group(1))
@@ -336,7 +335,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_peak": sbytes / (ms_per_step * 1e-3) / 1e9 / peak,
                      "frac_of_8tbs": sbytes / (ms_per_step * 1e-3) / 1e9 / 8000.0},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak if achieved else None, "traffic": load_traffic(dom),
+                     "frac": achieved / peak if achieved else None, "traffic": load_traffic(dom, wl.name),
                      "algorithmic_bytes": dom_bytes, "avg_ms": dom_ms, "peak_source": f"{peak_src} hbm_gbs"},
         "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
                     for n, (c, t) in per.items()},
@@ -434,10 +433,11 @@ def run_hier(args, rank, world, local_rank):
     dom = max(per, key=lambda n: per[n][1])
     dom_ms = per[dom][1] / per[dom][0]
     P = block * pool_blocks
-    # the dominant launch: the pool scores on the CUDA cores (fp32 FMA issue bound)
-    flops = 2.0 * B * P * wl.h_idx * wl.d_idx
-    alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
-    achieved = flops / (dom_ms * 1e-3) / 1e12
+    # the dominant launch reads the pool's keys (code bytes + row scale), the
+    # pool itself, the queries and the weights
+    peak, peak_src = load_peaks()
+    dom_bytes = B * (P * key_row_bytes(wl) + pool_blocks * 4 + wl.h_idx * (wl.d_idx * _eb(wl.act_dtype) + 4))
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     res = {
         "metric": "Reindex-layer selections/s (top-512 over a 16,384-candidate pool, 1M tokens)",
         "value": B / (ms * 1e-3),
@@ -458,9 +458,9 @@ def run_hier(args, rank, world, local_rank):
         "full_layer_ms": float(sum(full_ms)) / K,
         "full_scan_ms": float(sum(scan_ms)) / K,
         "reindex_vs_full_scan": (float(sum(scan_ms)) / K) / ms,
-        "roofline": {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
-                     "frac": achieved / alu_peak, "traffic": None, "algorithmic_flops": flops, "avg_ms": dom_ms,
-                     "peak_source": "fp32 FMA issue: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": load_traffic(dom, "hier1m_reindex"),
+                     "algorithmic_bytes": dom_bytes, "avg_ms": dom_ms, "peak_source": f"{peak_src} hbm_gbs"},
         "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
                     for n, (c, t) in per.items()},
         "gpu_launches": sum(c for c, _ in per.values()),
