@@ -115,12 +115,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   }
 
   if (tid == 0) {
+    prefetch_tensormap(&qmap);
     mbar_init(qbar, 1);
     mbar_init(sbar, 1);
     mbar_init(obar, 1);
     s_flags[0] = 0;
     s_flags[1] = 0;
     fence_barrier_init();
+    // the query first: its load overlaps the gather of the keys
+    mbar_arrive_expect_tx(qbar, kH * kD * 2);
+    for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + oQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
   }
   if (tid < kTK) {
     int32_t e = -1;
@@ -146,10 +150,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + oLut));
   __syncthreads();
-  if (tid == 0) {
-    mbar_arrive_expect_tx(qbar, kH * kD * 2);
-    for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + oQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
-  }
+
   if (tid < kTK && ent[tid] <= -2) s_flags[0] = 1;
   const int nsr = s1 - s0, nwr = w1 - w0;
   const uint32_t tmem = *tmem_slot;
@@ -239,30 +240,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
       }
     }
     __syncthreads();
-    // two consecutive dims per thread, R peers each
-    for (int w = 0; w < nh; ++w) {
-      const int h = split + w * R;
-      const int dim = tid * 2;
-      float2 v[16];
+    // two consecutive dims per thread, R peers each, two heads per round:
+    // every peer's loads of both heads in flight before the sums
+    const int dim = tid * 2;
+    for (int w0 = 0; w0 < nh; w0 += 2) {
+      float2 v[2][16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j)  // every peer's load in flight before the sums
-        if (j < R) v[j] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(Osm, j) + h * kD + dim);
-      float o0 = 0.f, o1 = 0.f;
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j < R) {
-          const float wj = wgt[w * 16 + j];
-          o0 = fmaf(wj, v[j].x, o0);
-          o1 = fmaf(wj, v[j].y, o1);
+        for (int j = 0; j < 16; ++j)
+          if (j < R && w0 + u < nh)
+            v[u][j] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(Osm, j) + (split + (w0 + u) * R) * kD +
+                                                       dim);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int w = w0 + u;
+        if (w >= nh) break;
+        const int h = split + w * R;
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < R) {
+            const float wj = wgt[w * 16 + j];
+            o0 = fmaf(wj, v[u][j].x, o0);
+            o1 = fmaf(wj, v[u][j].y, o1);
+          }
+        const float inv = wgt[kH * 16 + w * 2 + 1];
+        o0 *= inv;
+        o1 *= inv;
+        const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
+        if (a.out_dtype == kF32) {
+          *reinterpret_cast<float2*>(static_cast<float*>(a.out) + off) = make_float2(o0, o1);
+        } else {
+          *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0, o1);
         }
-      const float inv = wgt[kH * 16 + w * 2 + 1];
-      o0 *= inv;
-      o1 *= inv;
-      const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
-      if (a.out_dtype == kF32) {
-        *reinterpret_cast<float2*>(static_cast<float*>(a.out) + off) = make_float2(o0, o1);
-      } else {
-        *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0, o1);
       }
     }
     cluster.sync();  // every peer has read this CTA's partial

@@ -369,24 +369,27 @@ __device__ void attend_tile(uint8_t* smem, const Src& s, bool contiguous, int ns
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
     float sum = 0.f;
-    uint32_t pk[16];
+    // keys q4*32 .. +31 of row h into P^T (K-major blocks of 64 keys), eight
+    // at a time: a rolled loop, since this code runs once per launch and
+    // every instruction of it is fetched cold
+    const int k0 = q4 * 32;
+    const float mm = (m == -INFINITY) ? 0.f : m;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t pk[4];
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float p0 = (m == -INFINITY) ? 0.f : __expf(srow[i] - m);
-      const float p1 = (m == -INFINITY) ? 0.f : __expf(srow[i + 1] - m);
-      sum += p0 + p1;
-      pk[i >> 1] = pack_bf16(p0, p1);
+      for (int u = 0; u < 4; ++u) {
+        const float p0 = (m == -INFINITY) ? 0.f : __expf(srow[c * 8 + 2 * u] - mm);
+        const float p1 = (m == -INFINITY) ? 0.f : __expf(srow[c * 8 + 2 * u + 1] - mm);
+        sum += p0 + p1;
+        pk[u] = pack_bf16(p0, p1);
+      }
+      const int kk = k0 + c * 8;
+      *reinterpret_cast<uint4*>(Pt + (kk >> 6) * (kH * 128) + sw128_offset(h, (kk & 63) >> 3)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
     sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
     sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-    // keys q4*32 .. +31 of row h: K-major blocks of 64 keys
-    const int k0 = q4 * 32;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int kk = k0 + c * 8;
-      *reinterpret_cast<uint4*>(Pt + (kk >> 6) * (kH * 128) + sw128_offset(h, (kk & 63) >> 3)) =
-          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-    }
     if (q4 == 0) {
       ml[2 * h] = m;
       ml[2 * h + 1] = sum;
