@@ -1153,19 +1153,21 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
           // every boundary entry is taken
           for (uint32_t i = tid; i < my_e; i += kThreads) put(A_tot + preE[c] + i, __ldcg(eqg + i));
         } else if (E_tot <= static_cast<uint32_t>(kEqCache)) {
-          // the request's boundary entries, in index order, into shared memory
-          constexpr int LB = 8;
-          for (uint32_t j0 = 0; j0 < E_tot; j0 += kThreads * LB) {
-            uint2 e[LB];
+          // the request's boundary entries, in index order, into shared
+          // memory: warp w copies the lists of chunks w, w + 10, ... (each
+          // list is contiguous in its chunk's staging), four loads in flight
+          // per lane
+          for (int cc = warp; cc < nch; cc += kThreads / 32) {
+            const uint2* src = a.eq + (static_cast<int64_t>(r) * nch + cc) * (kMaxChunkTiles * kTileM);
+            const uint32_t o = preE[cc], len = preE[cc + 1] - o;
+            for (uint32_t j0 = 0; j0 < len; j0 += 128) {
+              uint2 e[4];
 #pragma unroll
-            for (int b = 0; b < LB; ++b) {
-              const uint32_t i = j0 + b * kThreads + tid;
-              if (i < E_tot) e[b] = __ldcg(eq_src(i));
-            }
+              for (int b = 0; b < 4; ++b)
+                if (j0 + b * 32 + lane < len) e[b] = __ldcg(src + j0 + b * 32 + lane);
 #pragma unroll
-            for (int b = 0; b < LB; ++b) {
-              const uint32_t i = j0 + b * kThreads + tid;
-              if (i < E_tot) ecache[i] = e[b];
+              for (int b = 0; b < 4; ++b)
+                if (j0 + b * 32 + lane < len) ecache[o + j0 + b * 32 + lane] = e[b];
             }
           }
           __syncthreads();
