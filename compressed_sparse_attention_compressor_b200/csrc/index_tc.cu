@@ -908,20 +908,6 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             break;
           }
           tc_fence_after();
-          float ks = 1.f;
-          if constexpr (FP8) {
-            const int ss = t % kSStages;
-            bool sok = true;
-            if (lane == 0) sok = mbar_wait(&sfull[ss], (t / kSStages) & 1, kWaitLimit);
-            __syncwarp();
-            if (!__shfl_sync(0xFFFFFFFFu, sok, 0)) {
-              atomicOr(&g_index_tc_error, 1u);
-              sh.fail = 1;
-              break;
-            }
-            ks = scale_ring[ss * kTileM + row] * qinv;
-            mbar_arrive(&sempty[ss]);
-          }
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
           const uint32_t acc_addr = lane_addr + acc * kAccCols;
 #pragma unroll
@@ -950,6 +936,22 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
                 s3 = fmaf(w_r[hh + h + 1], fmaxf(x1, 0.f), s3);
               }
             }
+          }
+          // the row scale after the accumulator is released: its wait is off
+          // the MMA -> epilogue -> MMA chain that paces the key stream
+          float ks = 1.f;
+          if constexpr (FP8) {
+            const int ss = t % kSStages;
+            bool sok = true;
+            if (lane == 0) sok = mbar_wait(&sfull[ss], (t / kSStages) & 1, kWaitLimit);
+            __syncwarp();
+            if (!__shfl_sync(0xFFFFFFFFu, sok, 0)) {
+              atomicOr(&g_index_tc_error, 1u);
+              sh.fail = 1;
+              break;
+            }
+            ks = scale_ring[ss * kTileM + row] * qinv;
+            mbar_arrive(&sempty[ss]);
           }
           const float sc = ((s0 + s1) + (s2 + s3)) * ks;
           tmem_st1(lane_addr + kScoreCol + t, __float_as_uint(sc));
