@@ -102,6 +102,30 @@ def kernel_bytes(name, wl, n_vis):
     return None
 
 
+def rank_workload(name, rank):
+    """Every rank runs its own requests: the workload's shapes, its own seed
+    (replicas: the requests are independent, nothing is exchanged)."""
+    base = Wk.WORKLOADS[name]
+    return base.scaled(seed=base.seed + 100 * rank)
+
+
+def max_over_ranks(x, dist, device):
+    """The largest x over the ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_s(batch_per_rank, world, ms_per_step):
+    """Whole-job decode throughput: every rank's requests over the slowest
+    rank's step time."""
+    return batch_per_rank * world / (ms_per_step * 1e-3)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -196,7 +220,7 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist_
         dist = dist_
 
-    wl = Wk.WORKLOADS[args.workload].scaled(seed=Wk.WORKLOADS[args.workload].seed + 100 * rank)
+    wl = rank_workload(args.workload, rank)
     inp = Wk.make_decode_inputs(wl)
     B = wl.batch
     up = DevTensor.from_stored
@@ -254,11 +278,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     step_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
-    total_ms = float(sum(step_ms))
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / K
 
     # ---- per-kernel times: the same K steps with events around every launch ----
@@ -303,14 +323,10 @@ def run_ours(args, rank, world, local_rank):
         f1[i].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(f0, f1)))
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = B * world / (e2e_ms / K * 1e-3)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(f0, f1)), dist, "cuda")
+    e2e_value = tokens_per_s(B, world, e2e_ms / K)
 
-    value = B * world / (ms_per_step * 1e-3)
+    value = tokens_per_s(B, world, ms_per_step)
     sbytes = step_bytes(wl, n_vis)
     res = {
         "metric": "decode tokens/s (CSA+SWA attention step)",
@@ -355,8 +371,7 @@ def run_hier(args, rank, world, local_rank):
     from compressed_sparse_attention_compressor_b200.csa import DevTensor
 
     torch.cuda.set_device(local_rank)
-    base = Wk.WORKLOADS["hier1m"]
-    wl = base.scaled(seed=base.seed + 100 * rank)
+    wl = rank_workload("hier1m", rank)
     block, pool_blocks = Wk.HIER_POOL
     B, cap, s = wl.batch, wl.context // wl.m, wl.seed
     sI = 1.0 / np.sqrt(wl.d_idx)
@@ -466,7 +481,7 @@ def run_hier(args, rank, world, local_rank):
         "gpu_launches": sum(c for c, _ in per.values()),
         "clocks": clk.summary(),
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
         # the oracle on request 0: its Full layer builds the pool (not timed),
         # its Reindex layer is the sample
         from oracle import csa_oracle as O
@@ -563,11 +578,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     if args.path == "hier":
-        if rank == 0:
-            print(json.dumps(run_hier(args, rank, world, local_rank)), flush=True)
-        return 0
-    res = run_ours(args, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # one GPU's study of the hierarchical indexer: every rank runs it on
+        # its own inputs, rank 0 prints its own line
+        res = run_hier(args, rank, world, local_rank)
+    else:
+        res = run_ours(args, rank, world, local_rank)
+    if args.path == "step" and rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, t = oracle_sample(args.workload)
         res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
                                "sample": f"{n} single-request decode steps of {args.workload} ({t:.1f} s)"}
