@@ -40,6 +40,12 @@ csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int3
                          int32_t* out_idx, float* out_score, cudaStream_t stream, int nv_div = 1, int ordered = 0);
 csa_status_t launch_block_max(const float* scores, int nq, int64_t ld, const int32_t* n_visible, int64_t cap,
                               int block, float* out, int64_t ld_out, cudaStream_t stream);
+int topk_multi_ctas(int n_rows, int64_t max_n);
+size_t topk_multi_ctl_bytes(int n_rows);
+csa_status_t launch_topk_multi(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int nv_div,
+                               int64_t max_n, int k, int32_t* out_idx, float* out_score, int ordered, int G,
+                               void* ctl, cudaStream_t stream);
+uint32_t topk_multi_take_error();
 csa_status_t launch_pool_map(const int32_t* pos, const float* pos_score, int nq, int k, const int32_t* pool, int block,
                              int pool_blocks, int32_t* out_idx, cudaStream_t stream);
 csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
@@ -124,6 +130,7 @@ size_t index_ws_bytes(int nq, int64_t cap) {
 size_t pool_ws_bytes(const csa_params_t* p, int nq, int64_t cap, int block) {
   Carver c(nullptr);
   c.take<float>(static_cast<size_t>(nq) * round_up((cap + block - 1) / block, 4));
+  c.take<char>(topk_multi_ctl_bytes(nq));
   const size_t head = c.off;
   c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
   size_t need = c.off;
@@ -346,6 +353,16 @@ csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const
   const int64_t ld = round_up(cap, 4);
   const int64_t nb = (cap + block - 1) / block, ldb = round_up(nb, 4);
   float* bmax = c.take<float>(static_cast<size_t>(n_queries) * ldb);
+  void* mctl = c.take<char>(topk_multi_ctl_bytes(n_queries));
+  // the pool: the best blocks in ascending order, several CTAs per query when
+  // the rows are long (one SM would take ~100 us over 131,072 maxima)
+  auto select_pool = [&]() -> csa_status_t {
+    const int G = topk_multi_ctas(n_queries, nb);
+    if (G > 0)
+      return launch_topk_multi(bmax, n_queries, ldb, n_visible, block, nb, pool_blocks, out_pool, nullptr, 1, G, mctl,
+                               s);
+    return launch_topk(bmax, n_queries, ldb, n_visible, nb, pool_blocks, out_pool, nullptr, s, block, 1);
+  };
   if (q_req == nullptr && n_queries == batch && p->topk >= 1 &&
       index_tc_supported(p, batch, cap, q_idx->dtype, k_idx->dtype)) {
     // the fused tensor-core indexer writes its top-k and the block maxima
@@ -356,7 +373,7 @@ csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const
     if ((st = launch_index_topk_tc(p, batch, q_idx, w, k_idx, cap, n_visible, out_idx ? out_idx : idx, out_score,
                                    tws, s, nullptr, bmax, ldb, block)) != CSA_OK)
       return st;
-    return launch_topk(bmax, n_queries, ldb, n_visible, nb, pool_blocks, out_pool, nullptr, s, block, 1);
+    return select_pool();
   }
   float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
   if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s)) !=
@@ -366,7 +383,7 @@ csa_status_t csa_index_topk_pool(const csa_params_t* p, int32_t n_queries, const
       (st = launch_topk(scores, n_queries, ld, n_visible, cap, p->topk, out_idx, out_score, s)) != CSA_OK)
     return st;
   if ((st = launch_block_max(scores, n_queries, ld, n_visible, cap, block, bmax, ldb, s)) != CSA_OK) return st;
-  return launch_topk(bmax, n_queries, ldb, n_visible, nb, pool_blocks, out_pool, nullptr, s, block, 1);
+  return select_pool();
 }
 
 csa_status_t csa_index_topk_reindex(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx,
@@ -619,6 +636,8 @@ csa_status_t csa_sync_status(csa_stream_t stream) {
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the indexer gave up");
   if (attn_tc_take_error() != 0)
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the attention gave up");
+  if (topk_multi_take_error() != 0)
+    return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the multi-CTA top-k gave up");
   return CSA_OK;
 }
 
