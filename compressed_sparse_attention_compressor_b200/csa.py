@@ -26,7 +26,8 @@ STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "C
 EXPORTS = ["csa_workspace_size", "csa_compress", "csa_index_topk", "csa_index_score", "csa_topk",
            "csa_sparse_swa_attention", "csa_decode_step", "csa_last_error", "csa_sync_status", "csa_profile_start",
            "csa_profile_stop", "csa_profile_count", "csa_profile_get", "csa_sparse_swa_attention_noalloc",
-           "csa_index_topk_pool", "csa_index_topk_reindex", "csa_index_pool_workspace_size"]
+           "csa_index_topk_pool", "csa_index_topk_reindex", "csa_index_pool_workspace_size",
+           "csa_topk_workspace_size"]
 
 
 class CsaError(RuntimeError):
@@ -79,6 +80,7 @@ def load() -> ctypes.CDLL:
         "csa_index_topk_pool": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, I32, I32, V, V, V, V, SZ, V]),
         "csa_index_topk_reindex": (I32, [P(Params), I32, T, V, T, I32, I64, V, V, V, I32, I32, V, V, V, SZ, V]),
         "csa_index_pool_workspace_size": (SZ, [P(Params), I32, I64, I32, I32]),
+        "csa_topk_workspace_size": (SZ, [I32]),
         "csa_sparse_swa_attention": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V, SZ, V]),
         "csa_sparse_swa_attention_noalloc": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V]),
         "csa_decode_step": (I32, [P(Params), I32, P(DecodeCaches), P(DecodeToken), V, T, V, V, SZ, V]),
@@ -207,6 +209,10 @@ def csa_index_score(p: Params, n_queries: int, q_idx: DevTensor, w: torch.Tensor
     _check(load().csa_index_score(ctypes.byref(p), n_queries, ctypes.byref(q_idx.c()), _ptr(w),
                                   ctypes.byref(k_idx.c()), batch, cap, _ptr(q_req), _ptr(n_visible), _ptr(scores), ld,
                                   _stream(stream)), "csa_index_score")
+
+
+def csa_topk_workspace_size(n_rows: int) -> int:
+    return load().csa_topk_workspace_size(n_rows)
 
 
 def csa_topk(scores: torch.Tensor, n_rows: int, ld: int, n_valid: torch.Tensor, k: int, out_idx: torch.Tensor,

@@ -257,16 +257,21 @@ csa_status_t csa_compress(const csa_tensor_t* C, const csa_tensor_t* Z, int32_t 
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t csa_topk_workspace_size(int32_t n_rows) { return n_rows > 0 ? topk_multi_ctl_bytes(n_rows) : 0; }
+
 csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int32_t* n_valid, int32_t k,
                       int32_t* out_idx, float* out_score, void* workspace, size_t workspace_bytes,
                       csa_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   g_msg[0] = 0;
   if (n_rows < 0 || k < 1 || ld < 0) return set_error(CSA_ERR_INVALID_ARG, "bad shape n_rows=%d k=%d", n_rows, k);
-  if (n_rows > 0 && (scores == nullptr || n_valid == nullptr || out_idx == nullptr))
+  if (n_rows == 0) return CSA_OK;
+  if (scores == nullptr || n_valid == nullptr || out_idx == nullptr)
     return set_error(CSA_ERR_INVALID_ARG, "null pointer");
-  return launch_topk(scores, n_rows, ld, n_valid, ld, k, out_idx, out_score, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int G = topk_multi_ctas(n_rows, ld);
+  if (G > 0 && workspace != nullptr && workspace_bytes >= topk_multi_ctl_bytes(n_rows))
+    return launch_topk_multi(scores, n_rows, ld, n_valid, 1, ld, k, out_idx, out_score, 0, G, workspace, s);
+  return launch_topk(scores, n_rows, ld, n_valid, ld, k, out_idx, out_score, s);
 }
 
 csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,

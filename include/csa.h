@@ -185,10 +185,16 @@ csa_status_t csa_index_score(const csa_params_t* p, int32_t n_queries, const csa
 
 /* a3 alone -- top-k of given fp32 score rows, same order rule as above.
  *   scores   [n_rows][ld] fp32; row i has n_valid[i] (<= ld) valid columns.
- *   out_idx  [n_rows][k] int32 (-1 padded), out_score optional.           */
+ *   out_idx  [n_rows][k] int32 (-1 padded), out_score optional.
+ *   workspace  optional: with at least csa_topk_workspace_size(n_rows)
+ *            bytes, rows of 32,768 or more columns are each split over
+ *            several CTAs (same result); without it one CTA takes a row.   */
 csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int32_t* n_valid,
                       int32_t k, int32_t* out_idx, float* out_score, void* workspace,
                       size_t workspace_bytes, csa_stream_t stream);
+
+/* Workspace bytes that let csa_topk split long rows over several CTAs. */
+size_t csa_topk_workspace_size(int32_t n_rows);
 
 /* Hierarchical sparse indexer, first (Full) layer.  [TOUR] chapter
  * "Compressed Sparse Attention 2", section "The Hierarchical Sparse Indexer"

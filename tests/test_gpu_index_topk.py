@@ -11,9 +11,10 @@ from tests._harness import check_selection, gpu_index_topk, i32
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("multi", [False, True])
 @pytest.mark.parametrize("k,n_cols,pad", [(1, 10, 5), (64, 1000, 5), (512, 20000, 5), (1024, 100000, 5), (7, 5, 5),
                                          (1024, 100000, 4), (2048, 131072, 0), (33, 5003, 1)])
-def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, cuda_lib):
+def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, multi, cuda_lib):
     """Same fp32 scores on both sides: selection must match exactly,
     including planted exact ties, -0 vs +0, and rows with n_valid <= k.
     pad: row stride - n_cols (a multiple of 4 gives 16-byte aligned rows)."""
@@ -26,7 +27,9 @@ def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, cuda_lib):
     scores = torch.from_numpy(buf).cuda()
     out_idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
     out_score = torch.empty((rows, k), dtype=torch.float32, device="cuda")
-    csa.csa_topk(scores, rows, ld, i32(n_valid), k, out_idx, out_score)
+    # with a workspace, rows of 32,768+ columns are split over several CTAs
+    ws = csa.workspace(csa.csa_topk_workspace_size(rows)) if multi else None
+    csa.csa_topk(scores, rows, ld, i32(n_valid), k, out_idx, out_score, ws)
     torch.cuda.synchronize()
     gi, gs = out_idx.cpu().numpy(), out_score.cpu().numpy()
     for r in range(rows):
@@ -38,12 +41,14 @@ def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, cuda_lib):
         assert np.all(np.isneginf(gs[r][~sel]))
 
 
-def test_topk_all_equal_scores_takes_lowest_indices(cuda_lib):
-    n, k = 5000, 300
+@pytest.mark.parametrize("n", [5000, 40000])
+def test_topk_all_equal_scores_takes_lowest_indices(n, cuda_lib):
+    """40,000 columns with a workspace: the rows are split over CTAs."""
+    k = 300
     scores = torch.zeros((2, n), dtype=torch.float32, device="cuda")
     scores[1, ::2] = -0.0
     out_idx = torch.empty((2, k), dtype=torch.int32, device="cuda")
-    csa.csa_topk(scores, 2, n, i32([n, n]), k, out_idx)
+    csa.csa_topk(scores, 2, n, i32([n, n]), k, out_idx, None, csa.workspace(csa.csa_topk_workspace_size(2)))
     torch.cuda.synchronize()
     for r in range(2):
         assert np.array_equal(np.sort(out_idx[r].cpu().numpy()), np.arange(k))
