@@ -32,7 +32,7 @@ Sources (web pages; cited by page title and section):
   chapter "SWA Bounded Replay", section "Replay only the window" (keys in
   [max(s, i-W+1), i]).
 
-Readings where the pages are silent or garbled (each listed in the design doc):
+Readings taken where the pages are silent or garbled:
 
 * Equation (1)'s body is not extracted.  Reading: within each block of m
   consecutive tokens the pooling weights are a softmax over the block's m
