@@ -377,6 +377,64 @@ def test_decode_step_ratio1_appends_the_token_row():
         assert np.allclose(res["new_keys"][b], c_t[b] @ O.decode_stored(inp.w_ik), atol=1e-13)
 
 
+def _small_prefill(**kw):
+    from compressed_sparse_attention_compressor_b200 import workloads as Wk
+
+    base = dict(batch=1, context=16, chunk=8, d=16, h_q=3, h_idx=2, d_idx=8, act_dtype="f32",
+                kv_dtype="f32", idx_dtype="f32")
+    base.update(kw)
+    return Wk.make_prefill_inputs(Wk.WORKLOADS["prefill"].scaled(**base))
+
+
+def test_pipeline_ratio1_dense_no_window_is_causal_attention_over_the_tokens():
+    # ratio 1 keeps every token as an entry; with no top-k, no window and a
+    # zero sink, query i (position 16 + i) attends causally over the 16 cached
+    # rows and the chunk's first i + 1 rows, the sink an extra key of logit 0
+    # and value 0
+    inp = _small_prefill(m=1, topk=0, window=0, sink="zero")
+    res = O.pipeline(inp)
+    cached = O.decode_stored(inp.kv_cached)[0][:16]
+    C = O.decode_stored(inp.C)[0]
+    rows = np.concatenate([cached, C])
+    q = O.decode_stored(inp.q)
+    for i in range(8):
+        ent = rows[:17 + i]
+        K = np.concatenate([np.concatenate([ent, np.zeros((len(ent), 1))], 1), [[0.0] * 16 + [1.0]]])
+        V = np.concatenate([ent, np.zeros((1, 16))])
+        qa = np.concatenate([q[i], np.zeros((3, 1))], 1)
+        assert np.allclose(res["out"][i], _sdpa(qa, K, V), rtol=0, atol=1e-12)
+
+
+def test_pipeline_topk_covering_every_entry_equals_dense():
+    # a top-k at least the visible entry count selects them all: the CSA path
+    # equals the dense (HCA) path over the same compressed cache, window and sink
+    sparse = O.pipeline(_small_prefill(m=2, topk=64, window=3, sink="normal"))
+    dense = O.pipeline(_small_prefill(m=2, topk=0, window=3, sink="normal"))
+    assert np.allclose(sparse["out"], dense["out"], rtol=0, atol=1e-12)
+    assert np.allclose(sparse["lse"], dense["lse"], rtol=0, atol=1e-12)
+    for i, t in enumerate(range(16, 24)):
+        sel = sparse["idx"][i]
+        assert sorted(sel[sel >= 0].tolist()) == list(range((t + 1) // 2))
+
+
+def test_pipeline_window_reads_the_ring_slots_of_the_last_w_positions():
+    # with m above every position no compressed entry is visible, so the
+    # output is attention over the window alone: keys and values of ring slots
+    # p % swa_cap for p in [t - W + 1, t]; positions 40..47 wrap the 16-slot ring
+    inp = _small_prefill(context=40, m=128, topk=0, window=4, sink="zero")
+    assert inp.swa_cap == 16
+    res = O.pipeline(inp)
+    K = O.decode_stored(inp.swa_k)[0]
+    V = O.decode_stored(inp.swa_v)[0]
+    q = O.decode_stored(inp.q)
+    for i, t in enumerate(range(40, 48)):
+        slots = [p % 16 for p in range(t - 3, t + 1)]
+        Kw = np.concatenate([np.concatenate([K[slots], np.zeros((4, 1))], 1), [[0.0] * 16 + [1.0]]])
+        Vw = np.concatenate([V[slots], np.zeros((1, 16))])
+        qa = np.concatenate([q[i], np.zeros((3, 1))], 1)
+        assert np.allclose(res["out"][i], _sdpa(qa, Kw, Vw), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # hierarchical sparse indexer: candidate pool and re-indexing
 # ---------------------------------------------------------------------------
