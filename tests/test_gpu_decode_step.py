@@ -72,6 +72,45 @@ def test_decode_step_matches_oracle(name, cuda_lib):
     assert np.array_equal(oc[:, t % wl.m], O.decode_stored(inp.c_t))
 
 
+# Requests of one batch at different positions: the first token (no entry
+# visible, the window holds the token alone), the token that closes the first
+# block (one entry), an open block, and a closing block past top-k.  Rows of
+# the caches beyond a request's visible entries hold stale values that must
+# not be read.
+RAGGED = {
+    "decode1m": (Wk.WORKLOADS["decode1m"].scaled(batch=4, context=8192), [0, 3, 4097, 8191]),
+    "decode1m_fp4": (Wk.WORKLOADS["decode1m_fp4"].scaled(batch=4, context=8192), [8191, 1, 3, 5002]),
+    "decode64k": (Wk.WORKLOADS["decode64k"].scaled(batch=3, context=4096), [4095, 0, 2050]),
+    "hybrid_hca": (Wk.WORKLOADS["hybrid_hca"].scaled(batch=3, context=128 * 40), [127, 5, 128 * 40 - 1]),
+    "tiny": (Wk.WORKLOADS["tiny"].scaled(batch=2, context=1024), [3, 1023]),
+}
+
+
+@pytest.mark.parametrize("name", list(RAGGED))
+def test_decode_step_ragged_positions(name, cuda_lib):
+    wl, positions = RAGGED[name]
+    inp = Wk.make_decode_inputs(wl)
+    inp.pos = np.array(positions, np.int64)
+    g = GpuDecode(inp)
+    g.step()
+    torch.cuda.synchronize()
+    ref = O.decode_step(inp)
+    check_attention(to_f64(g.out), g.lse.double().cpu().numpy(), ref["out"], ref["lse"], _dtype_tol(wl))
+    kv = to_f64(g.kv)
+    quant = wl.kv_dtype in ("fp8", "mxfp4")
+    closed = 0
+    for b, t in enumerate(positions):
+        if (t + 1) % wl.m == 0:
+            j = (t + 1) // wl.m - 1
+            sc = g.kv.scale[b, j:j + 1].cpu().numpy() if quant else None
+            codes = g.kv.data[b, j:j + 1].cpu().numpy() if quant else None
+            check_rows(kv[b, j:j + 1], ref["new_rows"][closed][None], wl.kv_dtype, 64, sc, codes)
+            closed += 1
+        assert np.array_equal(to_f64(g.swa_k)[b, t % inp.swa_cap], O.decode_stored(inp.k_t)[b])
+        assert np.array_equal(to_f64(g.open_c)[b, t % wl.m], O.decode_stored(inp.c_t)[b])
+    assert closed == len(ref["new_rows"])
+
+
 def test_decode_step_is_repeatable(cuda_lib):
     """Same position twice: identical outputs (the step only overwrites the
     slots it owns)."""
