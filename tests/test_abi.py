@@ -129,3 +129,85 @@ def test_pool_entry_points_reject_bad_arguments(lib):
     st = lib.csa_index_topk_reindex(ctypes.byref(p), 4, ctypes.byref(q), 16, ctypes.byref(k), 1, 1000, None, 16,
                                     16, 8, 64, 16, None, 16, 1 << 30, None)
     assert st == 1 and b"topk" in lib.csa_last_error()
+
+
+def _decode_args(kv_dtype=csa.CSA_FP8_E4M3, kv_scale=32, kv_group=64):
+    """A decode step's arguments that pass host validation (fake aligned
+    device addresses: every case below changes one field so that the call
+    returns before any launch)."""
+    p = csa.params(4, 512, 128, 64, 64, 64, 128, 128)
+    bf = lambda: _t()  # noqa: E731
+    caches = csa.DecodeCaches(_t(dtype=kv_dtype, scale=kv_scale, group=kv_group),
+                              _t(dtype=csa.CSA_FP8_E4M3, scale=32, group=128), bf(), bf(), bf(), bf(), 1024)
+    tok = csa.DecodeToken(bf(), bf(), bf(), bf(), bf(), bf(), 16, None, bf())
+    return p, caches, tok
+
+
+def _decode(lib, p, caches, tok, batch=4, pos=16, out=None, ws=16, ws_bytes=64):
+    out = out if out is not None else _t()
+    return lib.csa_decode_step(ctypes.byref(p), batch, ctypes.byref(caches), ctypes.byref(tok), pos,
+                               ctypes.byref(out), None, ws, ws_bytes, None)
+
+
+def test_decode_step_rejects_bad_arguments(lib):
+    p, caches, tok = _decode_args()
+    # the valid arguments reach the workspace check, which a 64-byte workspace fails
+    assert _decode(lib, p, caches, tok) == 3 and b"workspace" in lib.csa_last_error()
+    assert _decode(lib, p, caches, tok, batch=0) == 0  # nothing to do, nothing launched
+    assert _decode(lib, p, caches, tok, pos=None) == 1 and b"null" in lib.csa_last_error()
+    p.window = 0
+    assert _decode(lib, p, caches, tok) == 1 and b"window" in lib.csa_last_error()
+    p, caches, tok = _decode_args()
+    tok.w_ik = csa.Tensor(None, None, 0, 0)
+    assert _decode(lib, p, caches, tok) == 1 and b"w_ik" in lib.csa_last_error()
+    p, caches, tok = _decode_args()
+    p.d_idx = 48  # the projection needs a multiple of 32
+    st = _decode(lib, p, caches, tok)
+    assert st in (1, 2) and b"d_idx" in lib.csa_last_error()
+    p, caches, tok = _decode_args()
+    tok.z = _t(dtype=csa.CSA_F32)
+    assert _decode(lib, p, caches, tok) == 1 and b"one dtype" in lib.csa_last_error()
+    p, caches, tok = _decode_args()
+    caches.open_c = _t(dtype=csa.CSA_F32)
+    assert _decode(lib, p, caches, tok) == 1 and b"open-block" in lib.csa_last_error()
+    p, caches, tok = _decode_args()
+    caches.kv = _t(dtype=csa.CSA_FP8_E4M3, scale=32, group=128)  # main-KV FP8 groups are 64 channels
+    assert _decode(lib, p, caches, tok) == 1 and b"scale_group" in lib.csa_last_error()
+
+
+def test_decode_step_mxfp4_layout_rules(lib):
+    # MXFP4 main KV: one E4M3 scale byte per 16 elements, 16-byte aligned scales
+    p, caches, tok = _decode_args(kv_dtype=csa.CSA_MXFP4_E2M1, kv_scale=32, kv_group=16)
+    assert _decode(lib, p, caches, tok) == 3 and b"workspace" in lib.csa_last_error()
+    p, caches, tok = _decode_args(kv_dtype=csa.CSA_MXFP4_E2M1, kv_scale=32, kv_group=32)
+    assert _decode(lib, p, caches, tok) == 1 and b"scale_group must be 16" in lib.csa_last_error()
+    p, caches, tok = _decode_args(kv_dtype=csa.CSA_MXFP4_E2M1, kv_scale=None, kv_group=16)
+    assert _decode(lib, p, caches, tok) == 1 and b"scales" in lib.csa_last_error()
+    p, caches, tok = _decode_args(kv_dtype=csa.CSA_MXFP4_E2M1, kv_scale=40, kv_group=16)
+    assert _decode(lib, p, caches, tok) == 1 and b"aligned" in lib.csa_last_error()
+    # rows must hold whole 32-element pairs of scale groups (16 bytes of codes)
+    p, caches, tok = _decode_args(kv_dtype=csa.CSA_MXFP4_E2M1, kv_scale=32, kv_group=16)
+    p.d = 48
+    assert _decode(lib, p, caches, tok) == 1 and b"multiple of 16 bytes" in lib.csa_last_error()
+
+
+def test_compress_mxfp4_output_rules(lib):
+    C, Z = _t(), _t()
+    bad_group = _t(dtype=csa.CSA_MXFP4_E2M1, scale=32, group=32)
+    st = lib.csa_compress(ctypes.byref(C), ctypes.byref(Z), 1, 64, 128, 4, ctypes.byref(bad_group), 16, None, 0,
+                          None, None)
+    assert st == 1 and b"scale_group must be 16" in lib.csa_last_error()
+    no_scale = _t(dtype=csa.CSA_MXFP4_E2M1, scale=None, group=16)
+    st = lib.csa_compress(ctypes.byref(C), ctypes.byref(Z), 1, 64, 128, 4, ctypes.byref(no_scale), 16, None, 0,
+                          None, None)
+    assert st == 1 and b"scales" in lib.csa_last_error()
+
+
+def test_topk_rejects_bad_arguments(lib):
+    assert lib.csa_topk(16, 2, 64, 16, 0, 16, None, None, 0, None) == 1 and b"bad shape" in lib.csa_last_error()
+    assert lib.csa_topk(16, -1, 64, 16, 4, 16, None, None, 0, None) == 1
+    assert lib.csa_topk(16, 0, 64, 16, 4, 16, None, None, 0, None) == 0  # no rows: nothing launched
+    assert lib.csa_topk(None, 2, 64, 16, 4, 16, None, None, 0, None) == 1 and b"null" in lib.csa_last_error()
+    assert lib.csa_topk(16, 2, 64, None, 4, 16, None, None, 0, None) == 1
+    # the multi-CTA control words grow with the rows
+    assert csa.csa_topk_workspace_size(8) >= csa.csa_topk_workspace_size(1) > 0
