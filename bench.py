@@ -21,6 +21,7 @@ collective on the data path): weak scaling, max-over-ranks device time.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle as the reference arm
   python bench.py --path hier ...        # the hierarchical sparse indexer (hier1m)
+  python bench.py --path prefill ...     # chunked prefill (query-tokens/s)
 
 ``--path hier`` times one Reindex layer of a decoder group at 1M tokens
 (ratio 1, FP8 indexer keys, top 512): the lightning indexer over the
@@ -28,6 +29,11 @@ collective on the data path): weak scaling, max-over-ranks device time.
 blocks of 8), its top-512, and the pool-position -> entry mapping.  The Full
 layer (full scan + block maxima + pool) and a full scan with the Reindex
 layer's query are timed beside it.
+
+``--path prefill`` times one 4,096-token chunk after 131,072 cached tokens:
+the chunk's compressor (1,024 new entries and their indexer keys), then the
+indexer, top-512 and attention (selection + window + sink) of its 4,096
+queries, each over the entries causally visible to it.
 """
 from __future__ import annotations
 
@@ -58,7 +64,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode1m", choices=[k for k, v in Wk.WORKLOADS.items() if not v.is_prefill])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="step", choices=["step", "hier"])
+    ap.add_argument("--path", default="step", choices=["step", "hier", "prefill"])
     return ap.parse_args()
 
 
@@ -515,6 +521,179 @@ def run_hier(args, rank, world, local_rank):
     return res
 
 
+def prefill_kernel_work(name, wl, sum_vis, sum_keys):
+    """Algorithmic work of one launch of a chunked-prefill kernel: (amount,
+    kind) with kind 'alu' (fp32 flops on CUDA cores), 'tensor' (bf16 flops)
+    or 'hbm' (bytes).  sum_vis: visible entries summed over the queries;
+    sum_keys: attended keys (selected entries + window) summed over them."""
+    if name.startswith("index_score"):
+        return 2.0 * wl.h_idx * wl.d_idx * sum_vis, "alu"
+    if name.startswith("attn_tc"):
+        return 4.0 * wl.h_q * wl.d * sum_keys, "tensor"
+    if name.startswith("attn"):
+        return 4.0 * wl.h_q * wl.d * sum_keys, "alu"
+    if name.startswith("topk"):
+        return 4.0 * sum_vis, "hbm"
+    if name.startswith("compress"):
+        n_tok = wl.chunk
+        return (2.0 * n_tok * wl.d * _eb(wl.act_dtype) + n_tok // wl.m * (kv_row_bytes(wl) + key_row_bytes(wl))), "hbm"
+    return None, None
+
+
+def alu_peak_tflops(sms):
+    """fp32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 flops x the
+    measured maximum SM clock."""
+    mhz = 1965.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    except Exception:
+        pass
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_prefill(args, rank, world, local_rank):
+    """Chunked prefill: the chunk's compressor (4,096 tokens into 1,024
+    entries appended to the cache), then the indexer, top-k and attention for
+    its 4,096 queries, each over its causally visible entries."""
+    import torch
+
+    from compressed_sparse_attention_compressor_b200 import csa
+    from compressed_sparse_attention_compressor_b200.csa import DevTensor
+
+    torch.cuda.set_device(local_rank)
+    wl = rank_workload("prefill", rank)
+    inp = Wk.make_prefill_inputs(wl)
+    up = DevTensor.from_stored
+    m, d, cap, n0 = wl.m, wl.d, inp.cap, inp.n_cached
+    nq, n_tok = inp.q_pos.shape[0], inp.C.data.shape[1]
+    kv, kidx = up(inp.kv_cached), up(inp.kidx_cached)
+    C, Z, q, q_idx, w_ik = up(inp.C), up(inp.Z), up(inp.q), up(inp.q_idx), up(inp.w_ik)
+    swa_k, swa_v = up(inp.swa_k), up(inp.swa_v)
+    w = torch.from_numpy(inp.w).cuda()
+    sink = torch.from_numpy(inp.sink).cuda()
+    q_pos = torch.from_numpy(inp.q_pos).cuda()
+    q_req = torch.from_numpy(inp.q_req).cuda()
+    n_vis_np = ((inp.q_pos + 1) // m).astype(np.int32)
+    n_vis = torch.from_numpy(n_vis_np).cuda()
+    p = csa.params(m, d, wl.d_idx, wl.h_q, wl.h_idx, wl.topk, wl.window, inp.swa_cap, 1.0)
+    ws = csa.workspace(csa.csa_workspace_size(p, nq, cap))
+    out_idx = torch.empty((nq, wl.topk), dtype=torch.int32, device="cuda")
+    out = DevTensor.empty((nq, wl.h_q, d), "bf16")
+    lse = torch.empty((nq, wl.h_q), dtype=torch.float32, device="cuda")
+    kv_new, kidx_new = kv.offset_rows(n0), kidx.offset_rows(n0)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    evict = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush.zero_()
+        evict.sum()
+        torch.cuda._sleep(200_000)
+
+    def step():
+        csa.csa_compress(C, Z, 1, n_tok, d, m, kv_new, cap, w_ik, wl.d_idx, kidx_new, stream)
+        csa.csa_index_topk(p, nq, q_idx, w, kidx, 1, cap, q_req, n_vis, out_idx, None, ws, stream)
+        csa.csa_sparse_swa_attention(p, nq, q, kv, 1, cap, out_idx, n_vis, q_req, swa_k, swa_v, q_pos, None, sink,
+                                     out, lse, ws, stream)
+
+    for _ in range(args.warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush_l2()
+            e0[i].record(stream)
+            step()
+            e1[i].record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), None, "cuda") / K
+
+    csa.csa_profile_start(64 * K)
+    for _ in range(K):
+        flush_l2()
+        step()
+    torch.cuda.synchronize()
+    csa.csa_profile_stop()
+    per = {}
+    for name, t in csa.csa_profile_records():
+        c = per.setdefault(name, [0, 0.0])
+        c[0] += 1
+        c[1] += t
+    dom = max(per, key=lambda n: per[n][1])
+    dom_ms = per[dom][1] / per[dom][0]
+    sum_vis = float(n_vis_np.sum())
+    win = np.minimum(inp.q_pos + 1, wl.window)
+    sum_keys = float(np.minimum(n_vis_np, wl.topk).sum() + win.sum())
+    work, kind = prefill_kernel_work(dom, wl, sum_vis, sum_keys)
+    sms = torch.cuda.get_device_properties(local_rank).multi_processor_count
+    if kind == "hbm":
+        peak, src = load_peaks()
+        roof = {"bound": "hbm", "unit": "GB/s", "achieved": work / (dom_ms * 1e-3) / 1e9, "peak": peak,
+                "peak_source": f"{src} hbm_gbs"}
+    elif kind == "alu":
+        roof = {"bound": "alu", "unit": "TFLOP/s", "achieved": work / (dom_ms * 1e-3) / 1e12,
+                "peak": alu_peak_tflops(sms), "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 x sm_max_mhz"}
+    elif kind == "tensor":
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "achieved": work / (dom_ms * 1e-3) / 1e12,
+                "peak": 1682.4, "peak_source": "measured bf16_tflops"}
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                roof["peak"] = float(json.load(f)["bf16_tflops"])
+        except Exception:
+            roof["peak_source"] = "fallback bf16"
+    else:
+        roof = {"bound": None, "unit": None, "achieved": None, "peak": None, "peak_source": None}
+    roof.update({"kernel": dom, "frac": roof["achieved"] / roof["peak"] if roof["achieved"] else None,
+                 "traffic": None, "algorithmic_work": work, "avg_ms": dom_ms})
+    res = {
+        "metric": "prefill query-tokens/s (a 4,096-token chunk after 131,072 cached tokens)",
+        "value": nq / (ms * 1e-3),
+        "unit": "query-tokens/s",
+        "n_gpus": 1,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian cache, chunk and queries)",
+        "config": {"workload": wl.name, "context": wl.context, "chunk": n_tok, "m": m, "cached_entries": n0,
+                   "new_entries": n_tok // m, "topk": wl.topk, "window": wl.window, "h_q": wl.h_q, "d": d,
+                   "indexer": f"{wl.h_idx}x{wl.d_idx}",
+                   "l2": "flushed between timed steps (256 MB write, then 256 MB read)"},
+        "roofline": roof,
+        "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
+                    for n, (c, t) in per.items()},
+        "gpu_launches": sum(c for c, _ in per.values()) // K,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        # the oracle on 256 of the chunk's queries (every 16th); the chunk's
+        # compressor is timed once and charged to the sample pro rata
+        from oracle import csa_oracle as O
+
+        qs = list(range(0, nq, max(nq // 256, 1)))[:256]
+        t0 = time.perf_counter()
+        rows = O.compress(O.decode_stored(inp.C)[0], O.decode_stored(inp.Z)[0], m)
+        O.project_index_keys(rows, O.decode_stored(inp.w_ik))
+        t_c = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        O.pipeline(inp, qs)
+        t_p = time.perf_counter() - t0
+        t_q = max(t_p - t_c, 1e-9) + t_c * len(qs) / nq
+        res["cpu_baseline"] = {"value": len(qs) / t_q, "unit": "query-tokens/s", "cores": _threads(),
+                               "kind": "oracle",
+                               "sample": f"{len(qs)} of the chunk's {nq} queries ({t_p:.1f} s with the chunk's "
+                                         f"compressor, {t_c:.1f} s, charged {len(qs)}/{nq} of it)"}
+    return res
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
@@ -596,6 +775,8 @@ def main():
         # one GPU's study of the hierarchical indexer: every rank runs it on
         # its own inputs, rank 0 prints its own line
         res = run_hier(args, rank, world, local_rank)
+    elif args.path == "prefill":
+        res = run_prefill(args, rank, world, local_rank)
     else:
         res = run_ours(args, rank, world, local_rank)
     if args.path == "step" and rank == 0 and world == 1 and not args.no_cpu_baseline:
