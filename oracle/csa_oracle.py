@@ -123,7 +123,8 @@ MXFP4_GROUP = 16
 
 def e2m1_round(y: np.ndarray) -> np.ndarray:
     """Round fp64 values to the nearest E2M1 value, ties to the even code,
-    saturating at +-6.  Returns codes 0..15 (sign in bit 3; a negative value
+    saturating at +-6 (tech-report tour, "FP4 main KV cache": E2M1
+    elements; the rounding rule is a reading, the page names none).  Returns codes 0..15 (sign in bit 3; a negative value
     that rounds to zero keeps its sign bit)."""
     y = np.asarray(y, np.float64)
     mags = E2M1_VALUES[:8]                       # codes 0..7, ascending
@@ -182,7 +183,9 @@ def decode_stored(t) -> np.ndarray:
 
 def e4m3_round(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to the nearest E4M3 value, ties to even code,
-    saturating at +-448 (the largest finite value).  Returns codes (uint8)."""
+    saturating at +-448 (the largest finite value).  The FP8 storage of the
+    1M-token decode configuration; the rounding rule is a reading (the pages
+    name E4M3, not how values are rounded into it).  Returns codes (uint8)."""
     x = np.asarray(x, np.float64)
     finite = E4M3_VALUES[:127]                  # codes 0x00..0x7E, ascending
     mag = np.minimum(np.abs(x), E4M3_MAX)
@@ -200,7 +203,7 @@ def e4m3_round(x: np.ndarray) -> np.ndarray:
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to the nearest bf16 value (8 significant bits), ties
-    to even.  Normal range only, which covers every value the path stores."""
+    to even (a reading: the configurations store bf16 and name no rounding).  Normal range only, which covers every value the path stores."""
     x = np.asarray(x, np.float64)
     f, e = np.frexp(x)                      # x = f * 2^e, 0.5 <= |f| < 1
     return np.ldexp(np.rint(f * 256.0), e - 8)
@@ -277,7 +280,12 @@ def project_index_keys(C_hat: np.ndarray, w_ik: np.ndarray) -> np.ndarray:
 # a2 / a3: lightning indexer and per-query top-k
 # ===========================================================================
 def n_visible(t: int | np.ndarray, m: int):
-    """Compressed blocks whose last token is at or before position t."""
+    """Compressed blocks whose last token is at or before position t.
+
+    "DeepSeek-V4.1-Flash, illustrated", the CSA2 figure (each decoder query
+    scores its causally visible context).  Reading: block j, made of tokens
+    jm .. jm+m-1, is visible to position t once it is complete, (j+1)m-1 <= t.
+    """
     return (np.asarray(t) + 1) // m
 
 
@@ -347,7 +355,9 @@ def candidate_pool(scores: np.ndarray, block: int, pool_blocks: int) -> np.ndarr
 
 
 def pool_entries(pool: np.ndarray, block: int, n_vis: int) -> np.ndarray:
-    """Visible entry ids of a pool, ascending."""
+    """Visible entry ids of a pool, ascending: the positions a Reindex layer
+    scores.  Tech-report tour, "The Hierarchical Sparse Indexer" (later
+    indexers search only the pool's candidate positions)."""
     ids = [b * block + i for b in np.asarray(pool) if b >= 0 for i in range(block) if b * block + i < n_vis]
     return np.asarray(ids, np.int64)
 
@@ -433,6 +443,15 @@ def attend(q: np.ndarray, entries: np.ndarray, win_k: np.ndarray, win_v: np.ndar
       lse_h = M + log L.
     q [h][d], entries [n][d], win_k / win_v [p][d], sink [h] or None.
     With nothing to attend to and no sink: out = 0, lse = -inf.
+
+    Atlas, "compressed KV" entry (sparse attention over the selected
+    compressed entries, or dense over all of them) and "MLA" entry (attention
+    runs over the latent, so K = V = the entry); tech-report tour, "The
+    indexer selects, SWA covers the rest" (the query attends to the selected
+    entries together with the layer's sliding-window KV, one softmax).  The
+    sink follows the atlas's entry on attention sinks and activation outliers
+    (give the model the rescaling it improvises); its form, one logit per
+    head in the denominator only, is a reading: the pages print no formula.
     """
     q = np.asarray(q, np.float64)
     keys = np.concatenate([np.asarray(entries, np.float64).reshape(-1, q.shape[1]),
