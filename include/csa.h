@@ -117,7 +117,8 @@ typedef struct csa_params {
   float softmax_scale;    /* tau: logits are tau * q . k                           */
 } csa_params_t;
 
-/* Bytes of workspace needed by a call with these shapes.
+/* Bytes of workspace needed by a call with these shapes (scratch sizing: no
+ * counterpart on the pages).
  *   n_queries    query tokens of the call (decode: batch);
  *   max_entries  largest number of visible compressed entries of any query.
  * The result covers csa_index_topk, csa_sparse_swa_attention and
@@ -174,7 +175,8 @@ csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_
                             float* out_score, void* workspace, size_t workspace_bytes,
                             csa_stream_t stream);
 
-/* a2 alone -- the indexer scores of csa_index_topk written out:
+/* a2 alone ([ATLAS] "Trained sparse attention": the lightning indexer) --
+ * the indexer scores of csa_index_topk written out:
  * scores[i][j] = s_j for j < min(n_visible[i], cap); columns beyond are not
  * written.  scores [n_queries][ld] fp32, ld >= cap.  Same sources and
  * arguments as csa_index_topk.                                             */
@@ -183,7 +185,8 @@ csa_status_t csa_index_score(const csa_params_t* p, int32_t n_queries, const csa
                              const int32_t* q_req, const int32_t* n_visible, float* scores, int64_t ld,
                              csa_stream_t stream);
 
-/* a3 alone -- top-k of given fp32 score rows, same order rule as above.
+/* a3 alone ([TOUR] "The indexer selects, SWA covers the rest": the top-k
+ * selection) -- top-k of given fp32 score rows, same order rule as above.
  *   scores   [n_rows][ld] fp32; row i has n_valid[i] (<= ld) valid columns.
  *   out_idx  [n_rows][k] int32 (-1 padded), out_score optional.
  *   workspace  optional: with at least csa_topk_workspace_size(n_rows)
@@ -193,7 +196,8 @@ csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int
                       int32_t k, int32_t* out_idx, float* out_score, void* workspace,
                       size_t workspace_bytes, csa_stream_t stream);
 
-/* Workspace bytes that let csa_topk split long rows over several CTAs. */
+/* Workspace bytes that let csa_topk split long rows over several CTAs
+ * (scratch sizing: no counterpart on the pages). */
 size_t csa_topk_workspace_size(int32_t n_rows);
 
 /* Hierarchical sparse indexer, first (Full) layer.  [TOUR] chapter
@@ -250,7 +254,8 @@ csa_status_t csa_index_topk_reindex(const csa_params_t* p, int32_t n_queries, co
                                     float* out_score, void* workspace, size_t workspace_bytes,
                                     csa_stream_t stream);
 
-/* Workspace bytes that csa_index_topk_pool and csa_index_topk_reindex need
+/* Workspace bytes (scratch sizing: no counterpart on the pages) that
+ * csa_index_topk_pool and csa_index_topk_reindex need
  * for n_queries queries with at most max_entries visible entries (0 for
  * invalid arguments).                                                       */
 size_t csa_index_pool_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries,
@@ -356,7 +361,8 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
                              const csa_tensor_t* out, float* lse, void* workspace,
                              size_t workspace_bytes, csa_stream_t stream);
 
-/* Per-kernel timing (measurement support; not on the compute path).
+/* Per-kernel timing (measurement support; not on the compute path, no
+ * counterpart on the pages).
  * csa_profile_start(n) creates 2n CUDA events and from then on records one
  * event on the launch stream right before and right after each of the
  * library's kernel launches, for the first n launches; csa_profile_stop()
@@ -368,10 +374,12 @@ csa_status_t csa_profile_stop(void);
 int32_t csa_profile_count(void);
 csa_status_t csa_profile_get(int32_t i, const char** kernel_name, float* ms);
 
-/* Message of the last failed call on this thread ("" if none). */
+/* Message of the last failed call on this thread ("" if none; error
+ * reporting, no counterpart on the pages). */
 const char* csa_last_error(void);
 
-/* Synchronises `stream` and reports device-side errors latched by earlier
+/* (Error reporting, no counterpart on the pages.)  Synchronises `stream` and
+ * reports device-side errors latched by earlier
  * calls (e.g. CSA_ERR_TIMEOUT from a bounded wait), clearing them.        */
 csa_status_t csa_sync_status(csa_stream_t stream);
 
