@@ -1,6 +1,7 @@
 // Device-side helpers shared by the kernels of the library: storage-format
 // loads/stores (fp32, bf16, FP8 E4M3 with fp32 group scales, MXFP4: E2M1
-// with E4M3 scales per 16 elements), the ordered
+// with E4M3 scales per 16 elements: tech-report tour, "FP4 main KV cache"),
+// the ordered
 // 32-bit key of an fp32 score, and host-side error plumbing.
 #pragma once
 

@@ -6,7 +6,9 @@
 // per-CTA counts.  Same result as topk_row_kernel (score descending, lower
 // index first among exactly equal scores, -0 == +0), for rows too long for
 // one CTA to go through quickly (the candidate pool's block maxima:
-// 131,072 per query at one million tokens).
+// 131,072 per query at one million tokens).  Tech-report tour, "The
+// Hierarchical Sparse Indexer" (2,048 blocks of 8 positions form the pool)
+// and "The indexer selects, SWA covers the rest" (the top-k selection).
 #include "common.cuh"
 #include "sm100.cuh"
 
