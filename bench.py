@@ -132,6 +132,15 @@ def tokens_per_s(batch_per_rank, world, ms_per_step):
     return batch_per_rank * world / (ms_per_step * 1e-3)
 
 
+def step_stats(ms):
+    """Median and 10th / 90th percentiles of per-step times (ms), this rank's."""
+    v = np.asarray(list(ms), dtype=np.float64)
+    if v.size == 0:
+        return None
+    p10, p50, p90 = np.percentile(v, [10, 50, 90])
+    return {"p10_ms": float(p10), "median_ms": float(p50), "p90_ms": float(p90)}
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -357,6 +366,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
+        "step_ms": step_stats(step_ms),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -482,6 +492,7 @@ def run_hier(args, rank, world, local_rank):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": ms,
+        "step_ms": step_stats(re_ms),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -611,7 +622,8 @@ def run_prefill(args, rank, world, local_rank):
             step()
             e1[i].record(stream)
         torch.cuda.synchronize()
-    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), None, "cuda") / K
+    pre_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
+    ms = max_over_ranks(sum(pre_ms), None, "cuda") / K
 
     csa.csa_profile_start(64 * K)
     for _ in range(K):
@@ -658,6 +670,7 @@ def run_prefill(args, rank, world, local_rank):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": ms,
+        "step_ms": step_stats(pre_ms),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
