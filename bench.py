@@ -267,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     del inp
 
     def step():
-        csa.csa_decode_step(p, B, caches, tok, pos, out, lse, ws, stream)
+        csa.csa_decode_step(p, B, caches, tok, pos, out, lse, None, ws, stream)
 
     def barrier():
         if dist is not None:
@@ -348,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
         flush_l2()
         f0[i].record(stream)
         dev_pack.copy_(host_pack, non_blocking=True)
-        csa.csa_decode_step(p, B, caches, tok_p, pos, out, lse, ws, stream)
+        csa.csa_decode_step(p, B, caches, tok_p, pos, out, lse, None, ws, stream)
         host_out.copy_(out.data, non_blocking=True)
         f1[i].record(stream)
     torch.cuda.synchronize()

@@ -27,7 +27,7 @@ EXPORTS = ["csa_workspace_size", "csa_compress", "csa_index_topk", "csa_index_sc
            "csa_sparse_swa_attention", "csa_decode_step", "csa_last_error", "csa_sync_status", "csa_profile_start",
            "csa_profile_stop", "csa_profile_count", "csa_profile_get", "csa_sparse_swa_attention_noalloc",
            "csa_index_topk_pool", "csa_index_topk_reindex", "csa_index_pool_workspace_size",
-           "csa_topk_workspace_size"]
+           "csa_topk_workspace_size", "csa_test_expire_next_barrier"]
 
 
 class CsaError(RuntimeError):
@@ -83,9 +83,10 @@ def load() -> ctypes.CDLL:
         "csa_topk_workspace_size": (SZ, [I32]),
         "csa_sparse_swa_attention": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V, SZ, V]),
         "csa_sparse_swa_attention_noalloc": (I32, [P(Params), I32, T, T, I32, I64, V, V, V, T, T, V, V, V, T, V, V]),
-        "csa_decode_step": (I32, [P(Params), I32, P(DecodeCaches), P(DecodeToken), V, T, V, V, SZ, V]),
+        "csa_decode_step": (I32, [P(Params), I32, P(DecodeCaches), P(DecodeToken), V, T, V, V, V, SZ, V]),
         "csa_last_error": (ctypes.c_char_p, []),
         "csa_sync_status": (I32, [V]),
+        "csa_test_expire_next_barrier": (I32, [I32, ctypes.c_uint32]),
         "csa_profile_start": (I32, [I32]),
         "csa_profile_stop": (I32, []),
         "csa_profile_count": (I32, []),
@@ -294,9 +295,10 @@ def decode_token(c, z, k_swa, v_swa, q, q_idx, w, sink, w_ik) -> DecodeToken:
 
 
 def csa_decode_step(p: Params, batch: int, caches: DecodeCaches, tok: DecodeToken, pos: torch.Tensor,
-                    out: DevTensor, lse: torch.Tensor | None, workspace: torch.Tensor, stream=None):
+                    out: DevTensor, lse: torch.Tensor | None, out_idx: torch.Tensor | None, workspace: torch.Tensor,
+                    stream=None):
     _check(load().csa_decode_step(ctypes.byref(p), batch, ctypes.byref(caches), ctypes.byref(tok), _ptr(pos),
-                                  ctypes.byref(out.c()), _ptr(lse), _ptr(workspace),
+                                  ctypes.byref(out.c()), _ptr(lse), _ptr(out_idx), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)), "csa_decode_step")
 
 
@@ -306,6 +308,13 @@ def csa_last_error() -> str:
 
 def csa_sync_status(stream=None):
     _check(load().csa_sync_status(_stream(stream)), "csa_sync_status")
+
+
+def csa_test_expire_next_barrier(cta: int, polls: int):
+    """Test support: the next fused-indexer launch's CTA ``cta`` skips its
+    first grid-barrier arrival and its waits give up after ``polls`` polls
+    (see include/csa.h)."""
+    _check(load().csa_test_expire_next_barrier(cta, polls), "csa_test_expire_next_barrier")
 
 
 def csa_profile_start(max_launches: int):

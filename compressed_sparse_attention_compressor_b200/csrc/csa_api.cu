@@ -30,6 +30,7 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
 bool index_tc_pool_supported(const csa_params_t* p, int batch, int64_t cap, int block, int pool_blocks, int q_dtype,
                              int k_dtype);
 uint32_t index_tc_take_error();
+csa_status_t test_expire_next_barrier(int cta, uint32_t polls);
 uint32_t attn_tc_take_error();
 csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                                 const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
@@ -59,6 +60,9 @@ csa_status_t set_error(csa_status_t st, const char* fmt, ...);
 
 namespace {
 thread_local char g_msg[512] = "";
+}  // namespace
+
+namespace {
 
 // Workspace carve-up: consecutive 256-byte aligned regions.
 struct Carver {
@@ -106,6 +110,8 @@ csa_status_t check_tensor(const char* name, const csa_tensor_t* t, int row_elems
   return CSA_OK;
 }
 
+}  // namespace
+
 csa_status_t check_params(const csa_params_t* p, bool need_idx) {
   if (p == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null params");
   if (p->m < 1 || p->d < 8 || p->h_q < 1 || p->window < 0)
@@ -117,6 +123,22 @@ csa_status_t check_params(const csa_params_t* p, bool need_idx) {
     return set_error(CSA_ERR_INVALID_ARG, "bad indexer shape h_idx=%d d_idx=%d", p->h_idx, p->d_idx);
   return CSA_OK;
 }
+
+// Keys one query's attention covers: its selection (or, dense, the cache's
+// rows) plus the window.  Computed in 64 bits; a count beyond INT_MAX is an
+// invalid argument (the kernels index keys with 32-bit ints).
+csa_status_t attention_max_keys(const csa_params_t* p, bool sparse, int64_t cap, int* out) {
+  const int64_t mk = (sparse ? static_cast<int64_t>(p->topk) : cap) + p->window;
+  if (mk < 0 || mk > static_cast<int64_t>(INT32_MAX))
+    return set_error(CSA_ERR_INVALID_ARG, "attention over %lld keys per query (more than 2^31 - 1)",
+                     static_cast<long long>(mk));
+  *out = static_cast<int>(mk);
+  return CSA_OK;
+}
+
+void clear_error() { g_msg[0] = 0; }
+
+namespace {
 
 size_t index_ws_bytes(int nq, int64_t cap) {
   Carver c(nullptr);
@@ -213,7 +235,9 @@ const char* csa_last_error(void) { return g_msg; }
 
 size_t csa_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_entries) {
   if (p == nullptr || n_queries < 0 || max_entries < 0) return 0;
-  const int max_keys = static_cast<int>((p->topk > 0 ? p->topk : max_entries) + p->window);
+  const int64_t mk = (p->topk > 0 ? static_cast<int64_t>(p->topk) : max_entries) + p->window;
+  if (mk < 0 || mk > static_cast<int64_t>(INT32_MAX)) return 0;
+  const int max_keys = static_cast<int>(mk);
   Carver c(nullptr);
   // decode-step bookkeeping
   c.take<int32_t>(n_queries);
@@ -456,7 +480,8 @@ csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, 
   }
   if (n_visible == nullptr || q_pos == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null n_visible / q_pos");
   if (idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "idx given with topk < 1");
-  const int max_keys = static_cast<int>((idx ? p->topk : cap) + p->window);
+  int max_keys = 0;
+  if ((st = attention_max_keys(p, idx != nullptr, cap, &max_keys)) != CSA_OK) return st;
   const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
@@ -466,7 +491,7 @@ csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, 
 
 csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_decode_caches_t* cc,
                              const csa_decode_token_t* tok, const int64_t* pos, const csa_tensor_t* out, float* lse,
-                             void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+                             int32_t* out_idx, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
   g_msg[0] = 0;
   csa_status_t st;
   const bool sparse = p && p->topk > 0;
@@ -503,6 +528,8 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
     if (tok->w == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null indexer weights");
   }
   if ((st = check_tensor("out", out, p->d, true, true, false, 0)) != CSA_OK) return st;
+  int max_keys = 0;
+  if ((st = attention_max_keys(p, sparse, cc->cap, &max_keys)) != CSA_OK) return st;
   const size_t need = csa_workspace_size(p, batch, cc->cap);
   if (workspace == nullptr || workspace_bytes < need)
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
@@ -517,11 +544,11 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
   const bool tc = sparse && index_tc_supported(p, batch, cc->cap, tok->q_idx.dtype, cc->kidx.dtype);
   if (sparse) {
     idx = c.take<int32_t>(static_cast<size_t>(batch) * p->topk);
+    if (out_idx != nullptr) idx = out_idx;  // the caller keeps the selection
     size_t ib = index_ws_bytes(batch, cc->cap);
     const size_t tb = index_tc_workspace_bytes(batch, cc->cap, p->topk);
     index_ws = c.take<char>(ib > tb ? ib : tb);
   }
-  const int max_keys = static_cast<int>((sparse ? p->topk : cc->cap) + p->window);
   void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys));
 
   // CSA on the tensor-core indexer: the token is appended inside the indexer
@@ -632,6 +659,11 @@ csa_status_t csa_profile_get(int32_t i, const char** name, float* ms) {
   if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "profile record %d: %s", i, cudaGetErrorString(e));
   if (name) *name = g_prof_name[i];
   return CSA_OK;
+}
+
+csa_status_t csa_test_expire_next_barrier(int32_t cta, uint32_t polls) {
+  g_msg[0] = 0;
+  return test_expire_next_barrier(cta < 0 ? -1 : cta, polls);
 }
 
 csa_status_t csa_sync_status(csa_stream_t stream) {

@@ -14,11 +14,16 @@
 // of 128-key tiles, one CTA per range (grid = batch * chunks <= #SMs, all
 // resident: cooperative launch).  Inside a CTA:
 //   warp 0     TMA producer: key tiles (128 rows x 128 B, 128B swizzle)
-//              into a ring of shared-memory stages;
-//   warp 1     MMA issuer: D[128 keys][64 heads] (fp32, TMEM, two buffers)
-//              = keys x q^T with tcgen05.mma, M=128, N=64;
-//   warps 2-5  epilogue: TMEM -> registers, s = sum_h w_h ReLU(D_h),
-//              scores kept in shared memory.
+//              into a ring of shared-memory stages (FP8: one 256-row box =
+//              two tiles per stage);
+//   warp 1     MMA issuer: D[128 keys][N] (fp32, TMEM, two accumulators of
+//              128 columns, tiles taken in pairs) = keys x q^T with
+//              tcgen05.mma, M = 128; N = 128 for FP8 keys (both E4M3 terms
+//              of the split query, 64 heads each), N = 64 for bf16 keys;
+//   warps 2-9  epilogue, two groups of four warps on alternate tiles of a
+//              pair: TMEM -> registers, s = sum_h w_h ReLU(D_h) (FP8: the
+//              two query terms summed first), one score per key written
+//              back to a TMEM column and counted in the key histogram.
 // FP8 keys are consumed as stored (kind::f8f6f4, E4M3 x E4M3): the bf16
 // query, scaled by a power of two 2^e so that max|q| 2^e lies in [128, 256),
 // is split into two E4M3 terms q1 = e4m3(q 2^e), q2 = e4m3(q 2^e - q1) and
@@ -47,6 +52,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "pool.cuh"
@@ -138,6 +144,8 @@ struct IdxArgs {
   int pool_blocks;
   int pblock;              // 8 .. 128, a power of two
   const float* kscale;     // FP8 row scales [batch][cap] (pool mode)
+  uint32_t spin_limit;     // grid-barrier polls before a wait gives up (kSpinLimit)
+  int skip_arrive;         // CTA that does not arrive at the first barrier (-1: none; test hook)
 };
 
 struct Shared {
@@ -193,20 +201,22 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // run between the arrival and the wait.  request_arrive: the CTA's earlier
 // writes, then one arrival.  request_wait: until `target` arrivals; false on
 // a timeout.
-__device__ void request_arrive(uint32_t* ctr) {
+// `skip`: this CTA does not arrive (the test hook that makes the request's
+// waits run out; false in every normal launch).
+__device__ void request_arrive(uint32_t* ctr, bool skip) {
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && !skip) {
     __threadfence();
     atomicAdd(ctr, 1u);
   }
 }
 
-__device__ bool request_wait(uint32_t* ctr, uint32_t target, Shared& sh) {
+__device__ bool request_wait(uint32_t* ctr, uint32_t target, uint32_t limit, Shared& sh) {
   if (threadIdx.x == 0) {
     int ok = 1;
     uint32_t it = 0;
     while (ld_acquire_gpu(ctr) < target) {
-      if (++it > kSpinLimit) {
+      if (++it > limit) {
         atomicOr(&g_index_tc_error, 1u);
         ok = 0;
         break;
@@ -221,7 +231,7 @@ __device__ bool request_wait(uint32_t* ctr, uint32_t target, Shared& sh) {
 }
 
 // Bounded per-request grid barrier; returns false on timeout.
-__device__ bool request_barrier(uint32_t* ctr, uint32_t target, Shared& sh) {
+__device__ bool request_barrier(uint32_t* ctr, uint32_t target, uint32_t limit, Shared& sh) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
@@ -229,7 +239,7 @@ __device__ bool request_barrier(uint32_t* ctr, uint32_t target, Shared& sh) {
     atomicAdd(ctr, 1u);
     uint32_t it = 0;
     while (ld_acquire_gpu(ctr) < target) {
-      if (++it > kSpinLimit) {
+      if (++it > limit) {
         atomicOr(&g_index_tc_error, 1u);
         ok = 0;
         break;
@@ -1043,10 +1053,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         if (v) atomicAdd(&gh1[i], v);
       }
       // arrive, copy the scores while the request's slower CTAs finish, wait
-      request_arrive(&bar[0]);
+      request_arrive(&bar[0], static_cast<int>(blockIdx.x) == a.skip_arrive);
       copy_scores();
       if constexpr (BMAX) write_block_max();
-      bool alive = request_wait(&bar[0], a.chunks, sh);
+      bool alive = request_wait(&bar[0], a.chunks, a.spin_limit, sh);
       uint32_t shift = 20, prefix = 0;
       if (alive) {
         load_hist(hist, gh1);
@@ -1066,7 +1076,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
           for (int i = tid; i < kHistBins; i += kThreads)
             if (gh_g[i]) atomicAdd(&gh2[i], gh_g[i]);
           nbar = 2;
-          alive = request_barrier(&bar[0], 2u * a.chunks, sh);
+          alive = request_barrier(&bar[0], 2u * a.chunks, a.spin_limit, sh);
           if (alive) {
             load_hist(hist, gh2);
             __syncthreads();
@@ -1117,7 +1127,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         }
         if (tid == 0) reinterpret_cast<uint2*>(a.cnt)[slot] = make_uint2(my_a, my_e);
         ++nbar;
-        alive = request_barrier(&bar[0], nbar * a.chunks, sh);
+        alive = request_barrier(&bar[0], nbar * a.chunks, a.spin_limit, sh);
       }
       if (alive) {
         // ---- every CTA: chunk offsets, then its own share of the output ----
@@ -1262,6 +1272,12 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// A pending test request (csa_test_expire_next_barrier): consumed by the
+// next launch of this kernel.
+std::mutex g_test_mu;
+int g_test_skip_cta = -1;
+uint32_t g_test_polls = kSpinLimit;
+
 struct Launcher {
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   int sms = 0;
@@ -1403,6 +1419,17 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.pool_blocks = pool_blocks;
   a.pblock = pblock;
   a.kscale = fp8 ? static_cast<const float*>(k_idx->scale) : nullptr;
+  a.spin_limit = kSpinLimit;
+  a.skip_arrive = -1;
+  {
+    std::lock_guard<std::mutex> lk(g_test_mu);
+    if (g_test_skip_cta >= 0) {
+      a.skip_arrive = g_test_skip_cta;
+      a.spin_limit = g_test_polls;
+      g_test_skip_cta = -1;
+      g_test_polls = kSpinLimit;
+    }
+  }
   if (ap) {
     a.ap = *ap;
     a.ap.shrink = kAppendShrink;
@@ -1456,6 +1483,13 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
     return set_error(CSA_ERR_CUDA, "index_topk_tc_kernel launch: %s", cudaGetErrorString(e));
   }
   return check_launch("index_topk_tc_kernel", stream);
+}
+
+csa_status_t test_expire_next_barrier(int cta, uint32_t polls) {
+  std::lock_guard<std::mutex> lk(g_test_mu);
+  g_test_skip_cta = cta;
+  g_test_polls = polls < 1 ? 1 : polls;
+  return CSA_OK;
 }
 
 // Reads and clears the device error word of this kernel (bounded waits).

@@ -22,6 +22,9 @@ static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchByt
 namespace csa {
 
 size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys);
+csa_status_t check_params(const csa_params_t* p, bool need_idx);
+csa_status_t attention_max_keys(const csa_params_t* p, bool sparse, int64_t cap, int* out);
+void clear_error();
 
 namespace {
 
@@ -58,9 +61,15 @@ extern "C" csa_status_t csa_sparse_swa_attention_noalloc(
     int64_t cap, const int32_t* idx, const int32_t* n_visible, const int32_t* q_req, const csa_tensor_t* swa_k,
     const csa_tensor_t* swa_v, const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
     const csa_tensor_t* out, float* lse, csa_stream_t stream) {
-  if (p == nullptr) return set_error(CSA_ERR_INVALID_ARG, "null params");
-  if (n_queries < 0 || cap < 0) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / cap");
-  const int max_keys = static_cast<int>((idx ? p->topk : cap) + p->window);
+  clear_error();
+  // the same checks as csa_sparse_swa_attention before the scratch is sized,
+  // so that bad parameters give the same status from both entry points
+  csa_status_t st = check_params(p, false);
+  if (st != CSA_OK) return st;
+  if (n_queries < 0 || cap < 0 || batch < 1) return set_error(CSA_ERR_INVALID_ARG, "bad n_queries / batch / cap");
+  if (idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "idx given with topk < 1");
+  int max_keys = 0;
+  if ((st = attention_max_keys(p, idx != nullptr, cap, &max_keys)) != CSA_OK) return st;
   const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
   if (need > kNoAllocScratchBytes)
     return set_error(CSA_ERR_CAPACITY,
@@ -68,7 +77,7 @@ extern "C" csa_status_t csa_sparse_swa_attention_noalloc(
                      "library's fixed %zu; use csa_sparse_swa_attention with a caller workspace",
                      need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  csa_status_t st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != CSA_OK) return st;
   // Nothing in the scratch needs clearing: every split state the merge reads
   // is written by this call first.

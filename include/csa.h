@@ -355,11 +355,18 @@ typedef struct csa_decode_token {
  *      index + top-k as csa_index_topk.
  *   4. attention as csa_sparse_swa_attention with q_pos = t.
  * pos is read, never written: the caller advances it.  The step is
- * stream-ordered and writes only the caches' slots named above.            */
+ * stream-ordered and writes only the caches' slots named above.
+ *   out       [batch][h_q][d], CSA_F32 or CSA_BF16; lse optional [batch][h_q].
+ *   out_idx   optional [batch][p->topk] int32 (sparse steps only): the
+ *             selection of step 3, exactly as csa_index_topk writes it
+ *             (a set, -1 padded); NULL keeps it inside the workspace.
+ * Errors: CSA_ERR_INVALID_ARG for bad shapes, dtypes or alignment, or when
+ * the keys of one query (topk, or cap when dense, plus window) exceed
+ * 2^31 - 1; CSA_ERR_CAPACITY for a workspace below csa_workspace_size.     */
 csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_decode_caches_t* caches,
                              const csa_decode_token_t* tok, const int64_t* pos,
-                             const csa_tensor_t* out, float* lse, void* workspace,
-                             size_t workspace_bytes, csa_stream_t stream);
+                             const csa_tensor_t* out, float* lse, int32_t* out_idx,
+                             void* workspace, size_t workspace_bytes, csa_stream_t stream);
 
 /* Per-kernel timing (measurement support; not on the compute path, no
  * counterpart on the pages).
@@ -382,6 +389,19 @@ const char* csa_last_error(void);
  * reports device-side errors latched by earlier
  * calls (e.g. CSA_ERR_TIMEOUT from a bounded wait), clearing them.        */
 csa_status_t csa_sync_status(csa_stream_t stream);
+
+/* Test support for the bounded device-side waits (no counterpart on the
+ * pages; never needed in normal use).  The next launch of the fused
+ * tensor-core indexer (csa_index_topk, csa_index_topk_pool,
+ * csa_index_topk_reindex or csa_decode_step on its tensor-core path) takes
+ * this request: its CTA number `cta` does not arrive at the first
+ * per-request grid barrier, and every grid-barrier wait of that launch gives
+ * up after `polls` polls (about 64 ns apart; normally 2^22).  The CTAs of
+ * that request then stop waiting, latch CSA_ERR_TIMEOUT for
+ * csa_sync_status, leave their selection unwritten and exit; nothing faults
+ * and the context stays usable.  Launches after that one run normally.
+ * cta < 0 withdraws a pending request.  Process-wide, mutex-protected.     */
+csa_status_t csa_test_expire_next_barrier(int32_t cta, uint32_t polls);
 
 #ifdef __cplusplus
 }

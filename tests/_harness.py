@@ -4,15 +4,20 @@ tolerances.
 
 Tolerances (the acceptance bar of the path):
 * attention outputs and lse, max-abs error against the fp64 oracle:
-  1e-4 for fp32 workloads, 2e-2 for bf16 / FP8 / MXFP4 workloads;
-* selected index sets: fp32 workloads bit-exact (a differing set is only
-  accepted, with a warning, when the oracle's own k-th / (k+1)-th score gap
-  is below the fp32 error bound of a score); bf16 / FP8 workloads may differ
-  only by boundary swaps whose oracle scores lie within 1e-3 of the oracle's
-  k-th score;
+  1e-4 for fp32 workloads, 2e-2 for bf16 / FP8 / MXFP4 workloads; and, so
+  that the bar scales with outputs far below it (bf16 workloads whose
+  values are N(0,1)/sqrt(d) give outputs of about 0.005-0.1), the output's
+  max-abs error must also stay within the same number times max |oracle
+  output|: an all-zero or garbage-but-small output fails;
+* selected index sets: fp32 workloads bit-exact, except for swaps at a
+  near-tie -- an entry in only one of the two sets must score within the
+  fp32 error bound 1e-5 (1 + max|s|) of the oracle's k-th score (reported
+  with a warning); bf16 / FP8 workloads may differ only by boundary swaps
+  whose oracle scores lie within 1e-3 of the oracle's k-th score;
 * scores the kernel reports: |gpu - oracle| <= 1e-4 * (1 + |oracle|);
-* compressor outputs: fp32 1e-5 * (1 + |x|); bf16 half an ulp (2^-9 |x|)
-  plus 1e-6; FP8 scales to 1e-6 relative and codes within one step of the
+* compressor outputs: fp32 1e-5 * (1 + |x|); bf16 half an ulp (2^-8 |x| at
+  worst, just above a power of two) plus 1e-7; FP8 scales to 1e-5 relative
+  and codes within one step of the
   oracle's round-to-nearest-even code (a step only where the oracle value sits
   within 1e-5 relative of a rounding midpoint); MXFP4 scale bytes equal the
   oracle's E4M3 rounding of max|x| / 6 and codes the oracle's E2M1 rounding
@@ -32,6 +37,7 @@ from oracle import csa_oracle as O
 
 ATT_TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8": 2e-2, "mxfp4": 2e-2}
 BOUNDARY_GAP = 1e-3
+FP32_TIE = 1e-5  # relative fp32 error bound of an indexer score (times 1 + max|s|)
 
 
 def dev(st) -> DevTensor:
@@ -90,14 +96,27 @@ class GpuDecode:
         self.pos = i64(inp.pos)
         self.out = DevTensor.empty((wl.batch, wl.h_q, wl.d), out_dtype(wl))
         self.lse = torch.empty((wl.batch, wl.h_q), dtype=torch.float32, device="cuda")
+        # the step's selection (sparse workloads), -7 so that unwritten slots show
+        self.idx = None if wl.dense else torch.full((wl.batch, wl.topk), -7, dtype=torch.int32, device="cuda")
         self.ws = csa.workspace(csa.csa_workspace_size(self.p, wl.batch, inp.cap))
         self.caches = csa.decode_caches(self.kv, self.kidx, self.swa_k, self.swa_v, self.open_c, self.open_z, inp.cap)
         self.tok = csa.decode_token(self.c_t, self.z_t, self.k_t, self.v_t, self.q, self.q_idx, self.w, self.sink,
                                     self.w_ik)
 
     def step(self, stream=None):
-        csa.csa_decode_step(self.p, self.wl.batch, self.caches, self.tok, self.pos, self.out, self.lse, self.ws,
-                            stream)
+        csa.csa_decode_step(self.p, self.wl.batch, self.caches, self.tok, self.pos, self.out, self.lse, self.idx,
+                            self.ws, stream)
+
+    def check_selections(self, ref, requests=None) -> int:
+        """The step's selection of every request (or of ``requests``, in the
+        order of ``ref``) against the oracle decode step's scores; returns
+        the boundary swaps accepted."""
+        if self.idx is None:
+            return 0
+        reqs = list(range(self.wl.batch)) if requests is None else list(requests)
+        gi = self.idx.cpu().numpy()
+        exact = self.wl.act_dtype == "f32" and self.wl.idx_dtype == "f32"
+        return sum(check_selection(gi[b], ref["scores"][n], self.wl.topk, exact) for n, b in enumerate(reqs))
 
 
 def gpu_index_topk(wl, q_idx_st, w, kidx_st, batch, cap, q_req, n_vis, k=None):
@@ -137,15 +156,15 @@ def check_selection(gpu_row: np.ndarray, scores: np.ndarray, k: int, exact: bool
     diff = oset.symmetric_difference(valid.tolist())
     if not diff:
         return 0
-    if exact:
-        gap = O.boundary_gap(scores, k)
-        bound = 1e-5 * (1.0 + np.abs(scores).max())
-        assert gap < bound, f"fp32 selection differs from the oracle with boundary gap {gap:g}"
-        warnings.warn(f"fp32 near-tie at the top-k boundary (gap {gap:g} < {bound:g}); sets differ by {len(diff)}")
-        return len(diff)
     kth = np.sort(scores)[::-1][kk - 1]
+    # fp32: only a near-tie at fp32 resolution may swap; bf16 / FP8: 1e-3
+    tol = FP32_TIE * (1.0 + np.abs(scores).max()) if exact else BOUNDARY_GAP
     for j in diff:
-        assert abs(scores[j] - kth) < BOUNDARY_GAP, f"entry {j} differs by {abs(scores[j] - kth):g} from the k-th score"
+        assert abs(scores[j] - kth) <= tol, \
+            f"entry {j} is in one set only and scores {abs(scores[j] - kth):g} from the k-th (allowed {tol:g})"
+    if exact:
+        warnings.warn(f"fp32 near-tie at the top-k boundary (oracle gap {O.boundary_gap(scores, k):g}); "
+                      f"sets differ by {len(diff)} entries within {tol:g} of the k-th score")
     return len(diff) // 2
 
 
@@ -153,6 +172,9 @@ def check_attention(gpu_out, gpu_lse, ref_out, ref_lse, dtype: str):
     tol = ATT_TOL[dtype]
     err = np.abs(gpu_out - ref_out).max() if ref_out.size else 0.0
     assert err <= tol, f"attention max-abs error {err:g} > {tol:g}"
+    scale = np.abs(ref_out).max() if ref_out.size else 0.0
+    assert err <= tol * scale, \
+        f"attention max-abs error {err:g} > {tol:g} x max|oracle output| {scale:g} (the output-scaled bar)"
     fin = np.isfinite(ref_lse)
     assert np.array_equal(fin, np.isfinite(gpu_lse)), "lse finiteness differs"
     if fin.any():

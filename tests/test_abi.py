@@ -146,7 +146,7 @@ def _decode_args(kv_dtype=csa.CSA_FP8_E4M3, kv_scale=32, kv_group=64):
 def _decode(lib, p, caches, tok, batch=4, pos=16, out=None, ws=16, ws_bytes=64):
     out = out if out is not None else _t()
     return lib.csa_decode_step(ctypes.byref(p), batch, ctypes.byref(caches), ctypes.byref(tok), pos,
-                               ctypes.byref(out), None, ws, ws_bytes, None)
+                               ctypes.byref(out), None, None, ws, ws_bytes, None)
 
 
 def test_decode_step_rejects_bad_arguments(lib):
@@ -211,3 +211,40 @@ def test_topk_rejects_bad_arguments(lib):
     assert lib.csa_topk(16, 2, 64, None, 4, 16, None, None, 0, None) == 1
     # the multi-CTA control words grow with the rows
     assert csa.csa_topk_workspace_size(8) >= csa.csa_topk_workspace_size(1) > 0
+
+
+def test_key_counts_beyond_int32_are_rejected(lib):
+    """The keys of one query (selection or, dense, the cache's rows, plus the
+    window) are counted in 64 bits: a count past 2^31 - 1 is refused, never
+    wrapped into a small positive number that would pass the workspace or
+    scratch checks."""
+    p = csa.params(4, 512, 128, 64, 64, 0, 128, 128)  # dense (HCA)
+    huge = (1 << 31) - 64
+    assert csa.csa_workspace_size(p, 2, huge) == 0
+    q, kv, out = _t(), _t(), _t()
+    sk, sv = _t(), _t()
+    st = lib.csa_sparse_swa_attention(ctypes.byref(p), 2, ctypes.byref(q), ctypes.byref(kv), 1, huge, None, 16, None,
+                                      ctypes.byref(sk), ctypes.byref(sv), 16, None, None, ctypes.byref(out), None, 16,
+                                      1 << 40, None)
+    assert st == 1 and b"2^31" in lib.csa_last_error()
+    st = lib.csa_sparse_swa_attention_noalloc(ctypes.byref(p), 2, ctypes.byref(q), ctypes.byref(kv), 1, huge, None, 16,
+                                              None, ctypes.byref(sk), ctypes.byref(sv), 16, None, None,
+                                              ctypes.byref(out), None, None)
+    assert st == 1 and b"2^31" in lib.csa_last_error()
+    p2, caches, tok = _decode_args()
+    p2.topk = 0
+    caches.cap = huge
+    assert _decode(lib, p2, caches, tok) == 1 and b"2^31" in lib.csa_last_error()
+
+
+def test_noalloc_validates_params_before_sizing_its_scratch(lib):
+    """Bad parameters give the status csa_sparse_swa_attention gives
+    (CSA_ERR_INVALID_ARG), not a capacity error from a scratch size computed
+    out of them; the previous call's message does not linger."""
+    q, kv, out = _t(), _t(), _t()
+    for field, value in (("h_q", -64), ("d", -512), ("window", -1)):
+        p = csa.params(4, 512, 128, 64, 64, 64, 128, 128)
+        setattr(p, field, value)
+        st = lib.csa_sparse_swa_attention_noalloc(ctypes.byref(p), 2, ctypes.byref(q), ctypes.byref(kv), 1, 100, 16,
+                                                  16, None, None, None, 16, None, None, ctypes.byref(out), None, None)
+        assert st == 1 and b"params" in lib.csa_last_error(), (field, lib.csa_last_error())

@@ -50,6 +50,7 @@ def test_decode_step_matches_oracle(name, cuda_lib):
     torch.cuda.synchronize()
     ref = O.decode_step(inp)
     check_attention(to_f64(g.out), g.lse.double().cpu().numpy(), ref["out"], ref["lse"], _dtype_tol(wl))
+    g.check_selections(ref)
     t = int(inp.pos[0])
     if (t + 1) % wl.m == 0:
         j = (t + 1) // wl.m - 1
@@ -96,6 +97,7 @@ def test_decode_step_ragged_positions(name, cuda_lib):
     torch.cuda.synchronize()
     ref = O.decode_step(inp)
     check_attention(to_f64(g.out), g.lse.double().cpu().numpy(), ref["out"], ref["lse"], _dtype_tol(wl))
+    g.check_selections(ref)
     kv = to_f64(g.kv)
     quant = wl.kv_dtype in ("fp8", "mxfp4")
     closed = 0

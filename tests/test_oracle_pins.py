@@ -230,6 +230,39 @@ def test_topk_brute_force_definition():
         assert (i in chosen) == (rank < k)
 
 
+def test_boundary_gap_on_hand_written_rows():
+    """s_(k) - s_(k+1), the k-th largest score minus the (k+1)-th, by hand:
+    sorted descending, [5, 3, 3, 1] has gaps 2 (k = 1), 0 (k = 2, a tie), 2
+    (k = 3); nothing is cut off for k >= n or k <= 0.  The same row shuffled
+    gives the same gaps (the scores are ranked, not read in input order);
+    -0 and +0 are a tie."""
+    row = np.array([5.0, 3.0, 3.0, 1.0])
+    want = {1: 2.0, 2: 0.0, 3: 2.0}
+    for perm in ([0, 1, 2, 3], [3, 2, 0, 1], [1, 3, 0, 2]):
+        r = row[perm]
+        for k, gap in want.items():
+            assert O.boundary_gap(r, k) == gap, (perm, k)
+        for k in (0, 4, 5):
+            assert O.boundary_gap(r, k) == math.inf
+    assert O.boundary_gap(np.array([-0.0, 0.0, -1.0]), 1) == 0.0
+    assert O.boundary_gap(np.array([-0.0, 0.0, -1.0]), 2) == 1.0
+    # distinct gaps at every k: an index off by one anywhere changes the answer
+    r = np.array([10.0, 0.5, 7.0, 3.0, 6.0])  # sorted: 10, 7, 6, 3, 0.5
+    assert [O.boundary_gap(r, k) for k in range(1, 5)] == [3.0, 1.0, 3.0, 2.5]
+
+
+def test_boundary_gap_brute_force_definition():
+    """Against its definition: the smallest selected score minus the largest
+    score left out, with the selection the top-k."""
+    g = np.random.default_rng(16)
+    for n in (2, 7, 40):
+        s = np.round(g.standard_normal(n) * 3) / 3
+        for k in range(1, n):
+            sel = O.topk(s, k)
+            rest = np.setdiff1d(np.arange(n), sel)
+            assert O.boundary_gap(s, k) == s[sel].min() - s[rest].max()
+
+
 # ---------------------------------------------------------------- attention
 def _sdpa(q, k, v, mask=None):
     qt = torch.from_numpy(q)[None]

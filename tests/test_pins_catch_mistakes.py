@@ -108,6 +108,27 @@ def _block_scores_mean(scores, block):
     return np.array([s[b * block:(b + 1) * block].mean() for b in range(nb)])
 
 
+def _gap_off_by_one(scores, k):
+    s = np.sort(np.asarray(scores, np.float64))[::-1]
+    if k <= 0 or k + 1 >= s.shape[0]:
+        return float("inf")
+    return float(s[k] - s[k + 1])  # the (k+1)-th minus the (k+2)-th
+
+
+def _gap_unsorted(scores, k):
+    s = np.asarray(scores, np.float64)  # the row's own order, not ranked
+    if k <= 0 or k >= s.shape[0]:
+        return float("inf")
+    return float(s[k - 1] - s[k])
+
+
+def _gap_ascending(scores, k):
+    s = np.sort(np.asarray(scores, np.float64))  # ranked the wrong way round
+    if k <= 0 or k >= s.shape[0]:
+        return float("inf")
+    return float(s[k - 1] - s[k])
+
+
 _real = {"attend": O.attend}
 
 # (name, oracle attribute, wrong variant, pins aimed at it)
@@ -145,6 +166,12 @@ MISTAKES = [
      ["test_pool_matches_brute_force", "test_pool_of_single_entry_blocks_is_the_top_entries"]),
     ("block score = mean, not max", "block_scores", _block_scores_mean,
      ["test_block_scores_partial_tail_and_ties", "test_pool_matches_brute_force"]),
+    ("boundary gap one rank too deep", "boundary_gap", _gap_off_by_one,
+     ["test_boundary_gap_on_hand_written_rows", "test_boundary_gap_brute_force_definition"]),
+    ("boundary gap in input order", "boundary_gap", _gap_unsorted,
+     ["test_boundary_gap_on_hand_written_rows", "test_boundary_gap_brute_force_definition"]),
+    ("boundary gap ranked ascending", "boundary_gap", _gap_ascending,
+     ["test_boundary_gap_on_hand_written_rows", "test_boundary_gap_brute_force_definition"]),
 ]
 
 

@@ -13,7 +13,8 @@ import torch
 from compressed_sparse_attention_compressor_b200 import csa
 from compressed_sparse_attention_compressor_b200 import workloads as Wk
 from compressed_sparse_attention_compressor_b200.csa import CsaError, DevTensor
-from tests._harness import ATT_TOL, dev, f32, i32, i64, params_of, to_f64
+from oracle import csa_oracle as O
+from tests._harness import check_attention, dev, f32, i32, i64, params_of, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -43,13 +44,59 @@ def _run(fn, wl, p, nq, cap, a, with_ws):
 
 
 def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
+    """Top-1,024 + window per query: one cluster per query, merged in
+    distributed shared memory (no scratch written).  The same kernels run on
+    the same inputs, so the bytes must be equal."""
     wl, p, nq, cap, a = _problem()
     ref_out, ref_lse = _run(csa.csa_sparse_swa_attention, wl, p, nq, cap, a, True)
-    tol = ATT_TOL["fp8"]
-    for _ in range(2):  # the scratch keeps the previous call's contents
+    for _ in range(2):
         out, lse = _run(csa.csa_sparse_swa_attention_noalloc, wl, p, nq, cap, a, False)
-        assert np.abs(out - ref_out).max() <= tol
-        assert np.abs(lse - ref_lse).max() <= tol
+        assert np.array_equal(out, ref_out) and np.array_equal(lse, ref_lse)
+
+
+def _dense_problem(seed, nq=2, cap=4000):
+    """Dense (HCA) attention over up to 4,000 bf16 entries + the window:
+    33 key tiles per query, more than one cluster holds, so the kernel takes
+    its split path -- per-tile partial softmax states in the scratch, then a
+    merge kernel."""
+    wl = Wk.WORKLOADS["hybrid_hca"]
+    d = wl.d
+    sd = 1 / np.sqrt(d)
+    kv = Wk.store(Wk.normal(seed, "kv", (nq, cap, d), sd), "bf16")
+    sk = Wk.store(Wk.normal(seed, "sk", (nq, 128, d), sd), "bf16")
+    sv = Wk.store(Wk.normal(seed, "sv", (nq, 128, d), sd), "bf16")
+    q = Wk.store(Wk.normal(seed, "q", (nq, wl.h_q, d), sd), "bf16")
+    sink = Wk.normal(seed, "sink", (wl.h_q,))
+    n_vis = np.array([cap, cap - 1000][:nq], np.int32)
+    q_pos = (4 * n_vis.astype(np.int64) + 3)
+    args = dict(q=dev(q), kv=dev(kv), idx=None, n_vis=i32(n_vis), swa_k=dev(sk), swa_v=dev(sv), q_pos=i64(q_pos),
+                sink=f32(sink))
+    host = dict(q=q, kv=kv, sk=sk, sv=sv, sink=sink, n_vis=n_vis, q_pos=q_pos)
+    return wl, params_of(wl, 128), nq, cap, args, host
+
+
+def test_noalloc_split_path_uses_its_scratch_and_matches(cuda_lib):
+    """The split path writes every query's per-tile (max, sum, O) states into
+    the library's scratch array and merges them.  Two calls in a row, with a
+    different problem in between that leaves other values in the scratch:
+    each result equals the workspace entry point's bit for bit, and the
+    oracle within the tolerance."""
+    wl, p, nq, cap, a, h = _dense_problem(61)
+    need = csa.csa_workspace_size(p, nq, cap)
+    assert need > 4 * nq * 64 * 514 * 4, "the problem must need split states (scratch)"
+    ref_out, ref_lse = _run(csa.csa_sparse_swa_attention, wl, p, nq, cap, a, True)
+    wl2, p2, nq2, cap2, a2, _ = _dense_problem(62)
+    for _ in range(2):
+        out, lse = _run(csa.csa_sparse_swa_attention_noalloc, wl, p, nq, cap, a, False)
+        assert np.array_equal(out, ref_out) and np.array_equal(lse, ref_lse)
+        _run(csa.csa_sparse_swa_attention_noalloc, wl2, p2, nq2, cap2, a2, False)  # other scratch contents
+    qd = O.decode_stored(h["q"])
+    sk, sv = O.decode_stored(h["sk"]), O.decode_stored(h["sv"])
+    for i in range(nq):
+        rows = O.decode(h["kv"].data[i], "bf16")
+        o, l = O.sparse_swa_attention(qd[i], rows, None, int(h["n_vis"][i]), sk[i], sv[i], 128, int(h["q_pos"][i]),
+                                      wl.window, h["sink"], 1.0)
+        check_attention(out[i], lse[i], o, l, "bf16")
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch(cuda_lib):
