@@ -380,6 +380,7 @@ int attn_splits(int nq, int max_keys) {
 bool attn_tc_supported(const csa_params_t* p, int q_dtype, int kv_dtype, int swa_dtype, bool has_window);
 size_t attn_tc_workspace_bytes(int nq, int max_keys);
 int attn_tc_splits(int max_keys);
+int attn_cluster_min(int sel_max, int window);
 csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
                                  int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
                                  const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
@@ -389,14 +390,15 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
 
 // The tensor-core attention takes few queries, each cut into 128-key
 // splits (decode); many queries (prefill) use the CUDA-core kernel.
-static bool attn_tc_shape(int nq, int hq, int d, int max_keys) {
-  return hq == 64 && d == 512 && nq <= 64 && attn_tc_splits(max_keys) <= kMaxSplits;
+static bool attn_tc_shape(int nq, int hq, int d, int max_keys, int window) {
+  if (hq != 64 || d != 512 || attn_tc_splits(max_keys) > kMaxSplits) return false;
+  return nq <= 64 || attn_cluster_min(max_keys - window, window) > 0;
 }
 
-size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys) {
+size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys, int window) {
   const int s = attn_splits(nq, max_keys);
   size_t b = s <= 1 ? 0 : static_cast<size_t>(nq) * s * hq * (d + 2) * sizeof(float);
-  if (attn_tc_shape(nq, hq, d, max_keys)) {
+  if (attn_tc_shape(nq, hq, d, max_keys, window) && nq <= 64) {
     const size_t t = attn_tc_workspace_bytes(nq, max_keys);
     if (t > b) b = t;
   }
@@ -409,7 +411,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
                               void* workspace, int max_keys, cudaStream_t stream) {
   if (nq == 0) return CSA_OK;
-  if (attn_tc_shape(nq, p->h_q, p->d, max_keys) &&
+  if (attn_tc_shape(nq, p->h_q, p->d, max_keys, p->window) &&
       attn_tc_supported(p, q->dtype, kv->dtype, swa_k ? swa_k->dtype : kBF16, p->window > 0))
     return launch_attention_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink,
                                out, lse, workspace, max_keys, stream);

@@ -388,6 +388,7 @@ csa_status_t launch_attn_fmt(TcLauncher& L, const csa_params_t* p, int nq, int m
       return check_launch("attn_tc_cluster_kernel", stream);
     }
   }
+  if (nq > 64) return set_error(CSA_ERR_UNSUPPORTED, "attention: no cluster size fits %d queries", nq);
   prof_begin(stream);
   attn_tc_kernel<false, FMT><<<dim3(a.splits, nq), kThreads, kSmem, stream>>>(qmap, a);
   csa_status_t st = check_launch("attn_tc_kernel", stream);

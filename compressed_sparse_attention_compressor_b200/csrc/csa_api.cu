@@ -47,6 +47,13 @@ csa_status_t launch_topk_multi(const float* scores, int n_rows, int64_t ld, cons
                                int64_t max_n, int k, int32_t* out_idx, float* out_score, int ordered, int G,
                                void* ctl, cudaStream_t stream);
 uint32_t topk_multi_take_error();
+bool index_many_tc_supported(const csa_params_t* p, int q_dtype, int k_dtype);
+size_t index_many_tc_table_bytes(int nq);
+csa_status_t launch_index_many_tc(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
+                                  const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
+                                  const int32_t* n_visible, float* scores, int64_t ld, int32_t* table,
+                                  cudaStream_t stream);
+uint32_t index_many_take_error();
 csa_status_t launch_pool_map(const int32_t* pos, const float* pos_score, int nq, int k, const int32_t* pool, int block,
                              int pool_blocks, int32_t* out_idx, cudaStream_t stream);
 csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
@@ -54,7 +61,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               const csa_tensor_t* swa_k, const csa_tensor_t* swa_v, const int64_t* q_pos,
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
                               void* workspace, int max_keys, cudaStream_t stream);
-size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys);
+size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys, int window);
 
 csa_status_t set_error(csa_status_t st, const char* fmt, ...);
 
@@ -143,7 +150,19 @@ namespace {
 size_t index_ws_bytes(int nq, int64_t cap) {
   Carver c(nullptr);
   c.take<float>(static_cast<size_t>(nq) * round_up(cap, 4));
+  c.take<char>(index_many_tc_table_bytes(nq));
   return c.off;
+}
+
+// Scores of many queries per request: the tensor-core contraction where the
+// shapes allow it (64 x 128 bf16 indexer, 16-byte aligned head weights),
+// else the CUDA-core scorer.
+csa_status_t score_many(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
+                        const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
+                        const int32_t* n_visible, float* scores, int64_t ld, int32_t* table, cudaStream_t s) {
+  if (index_many_tc_supported(p, q_idx->dtype, k_idx->dtype) && aligned16(w))
+    return launch_index_many_tc(p, nq, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, table, s);
+  return launch_index_score(p, nq, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s);
 }
 
 // Full layer of the hierarchical indexer: the block maxima, then either all
@@ -252,7 +271,7 @@ size_t csa_workspace_size(const csa_params_t* p, int32_t n_queries, int64_t max_
     }
     c.take<char>(ib);
   }
-  const size_t attn = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
+  const size_t attn = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys, p->window);
   return c.off + attn + 256;
 }
 
@@ -328,8 +347,8 @@ csa_status_t csa_index_topk(const csa_params_t* p, int32_t n_queries, const csa_
   Carver c(workspace);
   const int64_t ld = round_up(cap, 4);
   float* scores = c.take<float>(static_cast<size_t>(n_queries) * ld);
-  if ((st = launch_index_score(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, cap, s)) !=
-      CSA_OK)
+  int32_t* table = reinterpret_cast<int32_t*>(c.take<char>(index_many_tc_table_bytes(n_queries)));
+  if ((st = score_many(p, n_queries, q_idx, w, k_idx, batch, cap, q_req, n_visible, scores, ld, table, s)) != CSA_OK)
     return st;
   return launch_topk(scores, n_queries, ld, n_visible, cap, p->topk, out_idx, out_score, s);
 }
@@ -482,7 +501,7 @@ csa_status_t csa_sparse_swa_attention(const csa_params_t* p, int32_t n_queries, 
   if (idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "idx given with topk < 1");
   int max_keys = 0;
   if ((st = attention_max_keys(p, idx != nullptr, cap, &max_keys)) != CSA_OK) return st;
-  const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
+  const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys, p->window);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
     return set_error(CSA_ERR_CAPACITY, "workspace of %zu bytes, need %zu", workspace_bytes, need);
   return launch_attention(p, n_queries, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink, out,
@@ -549,7 +568,7 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
     const size_t tb = index_tc_workspace_bytes(batch, cc->cap, p->topk);
     index_ws = c.take<char>(ib > tb ? ib : tb);
   }
-  void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys));
+  void* attn_ws = c.take<char>(attn_workspace_bytes(batch, p->h_q, p->d, max_keys, p->window));
 
   // CSA on the tensor-core indexer: the token is appended inside the indexer
   // (by the CTA that owns each request's last chunk); otherwise by its own kernel
@@ -675,6 +694,8 @@ csa_status_t csa_sync_status(csa_stream_t stream) {
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the attention gave up");
   if (topk_multi_take_error() != 0)
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the multi-CTA top-k gave up");
+  if (index_many_take_error() != 0)
+    return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the many-query indexer gave up");
   return CSA_OK;
 }
 

@@ -21,7 +21,7 @@ static __device__ __align__(256) unsigned char g_attn_scratch[kNoAllocScratchByt
 
 namespace csa {
 
-size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys);
+size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys, int window);
 csa_status_t check_params(const csa_params_t* p, bool need_idx);
 csa_status_t attention_max_keys(const csa_params_t* p, bool sparse, int64_t cap, int* out);
 void clear_error();
@@ -70,7 +70,7 @@ extern "C" csa_status_t csa_sparse_swa_attention_noalloc(
   if (idx != nullptr && p->topk < 1) return set_error(CSA_ERR_INVALID_ARG, "idx given with topk < 1");
   int max_keys = 0;
   if ((st = attention_max_keys(p, idx != nullptr, cap, &max_keys)) != CSA_OK) return st;
-  const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys);
+  const size_t need = attn_workspace_bytes(n_queries, p->h_q, p->d, max_keys, p->window);
   if (need > kNoAllocScratchBytes)
     return set_error(CSA_ERR_CAPACITY,
                      "csa_sparse_swa_attention_noalloc: this problem needs %zu bytes of scratch, more than the "

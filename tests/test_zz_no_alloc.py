@@ -54,11 +54,12 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
         assert np.array_equal(out, ref_out) and np.array_equal(lse, ref_lse)
 
 
-def _dense_problem(seed, nq=2, cap=4000):
-    """Dense (HCA) attention over up to 4,000 bf16 entries + the window:
-    33 key tiles per query, more than one cluster holds, so the kernel takes
-    its split path -- per-tile partial softmax states in the scratch, then a
-    merge kernel."""
+def _dense_problem(seed, nq=2, cap=3000):
+    """Dense (HCA) attention over up to 3,000 bf16 entries + the window:
+    25 key tiles per query, more than one cluster of 16 CTAs holds, so the
+    kernel takes its split path -- per-tile partial softmax states in the
+    scratch, then a merge kernel.  (The scratch the call reserves, about
+    13 MB, stays under the library's fixed 16 MiB.)"""
     wl = Wk.WORKLOADS["hybrid_hca"]
     d = wl.d
     sd = 1 / np.sqrt(d)
