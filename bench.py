@@ -582,6 +582,8 @@ def prefill_kernel_work(name, wl, sum_vis, sum_keys):
     kind) with kind 'alu' (fp32 flops on CUDA cores), 'tensor' (bf16 flops)
     or 'hbm' (bytes).  sum_vis: visible entries summed over the queries;
     sum_keys: attended keys (selected entries + window) summed over them."""
+    if name.startswith("index_many"):
+        return 2.0 * wl.h_idx * wl.d_idx * sum_vis, "tensor"
     if name.startswith("index_score"):
         return 2.0 * wl.h_idx * wl.d_idx * sum_vis, "alu"
     if name.startswith("attn_tc"):
@@ -594,6 +596,15 @@ def prefill_kernel_work(name, wl, sum_vis, sum_keys):
         n_tok = wl.chunk
         return (2.0 * n_tok * wl.d * _eb(wl.act_dtype) + n_tok // wl.m * (kv_row_bytes(wl) + key_row_bytes(wl))), "hbm"
     return None, None
+
+
+def bf16_peak():
+    """Measured dense bf16 tensor peak (TFLOP/s, burst), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def alu_peak_tflops(sms):
@@ -707,6 +718,21 @@ def run_prefill(args, rank, world, local_rank):
         roof = {"bound": None, "unit": None, "achieved": None, "peak": None, "peak_source": None}
     roof.update({"kernel": dom, "frac": roof["achieved"] / roof["peak"] if roof["achieved"] else None,
                  "traffic": None, "algorithmic_work": work, "avg_ms": dom_ms})
+
+    def kernel_roof(name, c, t):
+        """Each kernel's own work against its own roof (tensor: measured bf16
+        peak; hbm: measured copy bandwidth; alu: the CUDA cores' fp32 peak)."""
+        wk, kd = prefill_kernel_work(name, wl, sum_vis, sum_keys)
+        if wk is None:
+            return {}
+        sec = t / c * 1e-3
+        if kd == "hbm":
+            ach, pk = wk / sec / 1e9, load_peaks()[0]
+        elif kd == "tensor":
+            ach, pk = wk / sec / 1e12, roof["peak"] if roof["bound"] == "tensor" else bf16_peak()
+        else:
+            ach, pk = wk / sec / 1e12, alu_peak_tflops(sms)
+        return {"bound": kd, "achieved": ach, "peak": pk, "frac": ach / pk}
     res = {
         "metric": "prefill query-tokens/s (a 4,096-token chunk after 131,072 cached tokens)",
         "value": nq / (ms * 1e-3),
@@ -726,7 +752,8 @@ def run_prefill(args, rank, world, local_rank):
                    "indexer": f"{wl.h_idx}x{wl.d_idx}",
                    "l2": "flushed between timed steps (256 MB write, then 256 MB read)"},
         "roofline": roof,
-        "kernels": {n: {"launches": c, "total_ms": t, "share": t / sum(v[1] for v in per.values())}
+        "kernels": {n: {"launches": c, "total_ms": t, "avg_ms": t / c, "share": t / sum(v[1] for v in per.values()),
+                        **kernel_roof(n, c, t)}
                     for n, (c, t) in per.items()},
         "gpu_launches": sum(c for c, _ in per.values()),  # over the K steps, as timed
         "clocks": clk.summary(),
