@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--workload", default="decode1m", choices=[k for k, v in Wk.WORKLOADS.items() if not v.is_prefill])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="step", choices=["step", "hier", "prefill"])
+    ap.add_argument("--copies", type=int, default=0,
+                    help="cache copies the decode steps rotate over (0: enough that no step finds its inputs in "
+                         "L2; a profiler run may ask for fewer to hold less memory)")
     return ap.parse_args()
 
 
@@ -268,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
     sbytes = step_bytes(wl, n_vis)
     cache_st = (inp.kv, inp.kidx, inp.swa_k, inp.swa_v, inp.open_c, inp.open_z)
     copy_bytes = sum(t.data.nbytes + (t.scale.nbytes if t.scale is not None else 0) for t in cache_st)
-    ncp = n_copies(sbytes, copy_bytes)
+    ncp = args.copies if args.copies > 0 else n_copies(sbytes, copy_bytes)
     caches, keep = [], []
     for _ in range(ncp):
         kv, kidx, swa_k, swa_v, open_c, open_z = (up(t) for t in cache_st)

@@ -69,9 +69,8 @@ constexpr int kDI = 128;
 constexpr int kEpiWarps = 8;                     // two groups of four, alternating tiles
 constexpr int kThreads = 32 * (2 + kEpiWarps);   // producer, MMA, epilogue
 constexpr int kPrep = kThreads - 32;             // threads preparing the query (warps 1..)
-constexpr int kNAcc = 2;                         // accumulator buffers, one per epilogue group
+constexpr int kNAcc = 4;                         // accumulators: two pair slots x one per epilogue group
 constexpr int kAccCols = 128;                    // TMEM columns per accumulator
-constexpr int kScoreCol = kNAcc * kAccCols;      // first TMEM column holding scores (one per tile)
 constexpr int kMaxChunkTiles = 224;              // tiles of one CTA (TMEM columns, shared-memory scores)
 constexpr int kTmemCols = 512;
 constexpr int kHistBins = 4096;
@@ -82,7 +81,7 @@ constexpr int kSStages = 16;                     // FP8 row-scale ring (one 512-
 constexpr int kAppendShrink = 26;                // tiles the appending CTA's chunk gives up
 constexpr uint32_t kWaitLimit = 1u << 22;        // mbarrier polls
 constexpr uint32_t kSpinLimit = 1u << 22;        // grid-barrier polls (~64 ns apart)
-static_assert(kScoreCol + kMaxChunkTiles <= kTmemCols, "TMEM columns");
+static_assert(kNAcc * kAccCols <= kTmemCols, "TMEM columns");
 
 __device__ uint32_t g_index_tc_error = 0;  // bit 0: a bounded wait gave up
 
@@ -103,7 +102,7 @@ struct Cfg {
   static constexpr int kSmem = oMisc + 256 + 1024;
   // FP8: N = 128 = both E4M3 terms of the split query (rows 0..63 and 64..127 of B)
   static constexpr uint32_t kIdesc = FP8 ? idesc(0, 0, kTileM, 2 * kHeads) : idesc(1, 1, kTileM, kHeads);
-  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 5) <= 512, "mbarrier area");
+  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 7) <= 512, "mbarrier area");
   static_assert(oB % 1024 == 0, "operand alignment");
   static_assert(kSmem <= 232448, "shared memory");
   // phase-2 scratch, inside the (then idle) stage and scale rings
@@ -133,6 +132,7 @@ struct IdxArgs {
   uint32_t* cnt;           // [batch][chunks][2] entries above / at the boundary per chunk
   uint2* st;               // [batch][chunks][k] (index, score bits) above the boundary, beyond kACache
   uint2* eq;               // [batch][chunks][kMaxChunkTiles * 128] (index, score bits) at the boundary
+  float* scg;              // [batch][chunks][kMaxChunkTiles * 128] the chunk's scores, tile by tile
   int append;              // 1: n = (pos + 1) / m and the last chunk's CTA appends the token
   AppendArgs ap;
   float* bmax;             // optional [batch][ldb]: max score of each block of `block` entries
@@ -585,9 +585,9 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   uint64_t* empty = full + C::kStages;
   uint64_t* sfull = empty + C::kStages;
   uint64_t* sempty = sfull + kSStages;
-  uint64_t* tfull = sempty + kSStages;  // a pair of tiles' accumulators are ready
-  uint64_t* tempty = tfull + 1;          // ... and have been read back
-  uint64_t* qbar = tempty + 1;
+  uint64_t* tfull = sempty + kSStages;  // [2] pair slot s: its two tiles' accumulators are ready
+  uint64_t* tempty = tfull + 2;          // [2] ... and have been read back
+  uint64_t* qbar = tempty + 2;
   uint64_t* mdone = qbar + 1;
   uint64_t* abar = mdone + 1;  // W_IK of the in-kernel append
   uint8_t* Bs = smem + C::oB;
@@ -635,8 +635,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 128);  // the epilogue group that read the scales
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, kNAcc * 128);
+    for (int ps = 0; ps < 2; ++ps) {
+      mbar_init(&tfull[ps], 1);
+      mbar_init(&tempty[ps], 2 * 128);  // both epilogue groups
+    }
     mbar_init(qbar, 1);
     mbar_init(mdone, 1);
     mbar_init(abar, 1);
@@ -855,13 +857,16 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             ok = mbar_wait(&full[sa], (ta / C::kStages) & 1, kWaitLimit);
             if (ok && two) ok = mbar_wait(&full[sb], ((ta + 1) / C::kStages) & 1, kWaitLimit);
           }
-          if (ok) ok = mbar_wait(tempty, (p & 1) ^ 1, kWaitLimit);
+          // pair slot p % 2: its previous use (pair p - 2) has been read back
+          const int ps = p & 1;
+          if (ok) ok = mbar_wait(&tempty[ps], ((p >> 1) & 1) ^ 1, kWaitLimit);
           if (!ok) {
             atomicOr(&g_index_tc_error, 1u);
             sh.fail = 1;
             break;
           }
           tc_fence_after();
+          const uint32_t d0 = tmem + ps * 2 * kAccCols, d1 = d0 + kAccCols;
           const uint32_t a0 = smem_u32(smem + C::oStages + sa * C::kStageBytes);
           const uint32_t a1 = FP8 ? a0 + 16384 : smem_u32(smem + C::oStages + sb * C::kStageBytes);
           if constexpr (FP8) {
@@ -869,8 +874,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = desc_k_sw128(b_base + kk * 32);
-              mma_f8f6f4(tmem, desc_k_sw128(a0 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
-              if (two) mma_f8f6f4(tmem + kAccCols, desc_k_sw128(a1 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              mma_f8f6f4(d0, desc_k_sw128(a0 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              if (two) mma_f8f6f4(d1, desc_k_sw128(a1 + kk * 32), bd, C::kIdesc, kk > 0 ? 1u : 0u);
             }
             mma_commit(&empty[sa]);
           } else {
@@ -878,13 +883,13 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t half = kk >> 2, off = (kk & 3) * 32;
               const uint64_t bd = desc_k_sw128(b_base + half * 8192 + off);
-              mma_f16(tmem, desc_k_sw128(a0 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
-              if (two) mma_f16(tmem + kAccCols, desc_k_sw128(a1 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              mma_f16(d0, desc_k_sw128(a0 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
+              if (two) mma_f16(d1, desc_k_sw128(a1 + half * 16384 + off), bd, C::kIdesc, kk > 0 ? 1u : 0u);
             }
             mma_commit(&empty[sa]);
             if (two) mma_commit(&empty[sb]);
           }
-          mma_commit(tfull);
+          mma_commit(&tfull[ps]);
         }
         // every MMA of this CTA has completed before TMEM is read back or released
         mma_commit(mdone);
@@ -906,11 +911,15 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         float w_r[kHeads];
 #pragma unroll
         for (int h = 0; h < kHeads; ++h) w_r[h] = ws[h];
+        // this chunk's scores in the workspace, tile by tile (lane = key)
+        float* scg = a.scg + (static_cast<int64_t>(r) * a.chunks + c) * (kMaxChunkTiles * kTileM);
         for (int t = grp; t < nt; t += 2) {
-          const int acc = grp;
+          // tile t = 2p + grp sits in pair slot ps = p % 2, accumulator 2 ps + grp
+          const int ps = (t >> 1) & 1;
+          const int acc = 2 * ps + grp;
           // lane 0 polls, the warp follows its verdict (warp-wide TMEM ops below)
           bool tok = true;
-          if (lane == 0) tok = mbar_wait(tfull, (t >> 1) & 1, kWaitLimit);
+          if (lane == 0) tok = mbar_wait(&tfull[ps], (t >> 2) & 1, kWaitLimit);
           __syncwarp();  // orders the other lanes after lane 0's acquire
           if (!__shfl_sync(0xFFFFFFFFu, tok, 0)) {
             atomicOr(&g_index_tc_error, 1u);
@@ -929,7 +938,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             tmem_wait_ld();
             if (hh + 32 == kHeads) {
               tc_fence_before();
-              mbar_arrive(tempty);
+              mbar_arrive(&tempty[ps]);
             }
 #pragma unroll
             for (int h = 0; h < 32; h += 2) {
@@ -964,10 +973,9 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             mbar_arrive(&sempty[ss]);
           }
           const float sc = ((s0 + s1) + (s2 + s3)) * ks;
-          tmem_st1(lane_addr + kScoreCol + t, __float_as_uint(sc));
+          scg[t * kTileM + row] = sc;
           if (static_cast<int64_t>(t0 + t) * kTileM + row < n) atomicAdd(&hist[score_key(sc) >> 20], 1u);
         }
-        tmem_wait_st();
       }
     }
   }
@@ -998,18 +1006,22 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     };
 
     // scores TMEM -> shared memory in index order: warps 2..9, two per lane quarter
+    // the chunk's scores, workspace -> shared memory in index order (the
+    // block's own writes of phase 1, ordered by the barrier after it)
     auto copy_scores = [&]() {
-      if (warp >= 2) {
-        const int q = warp & 3, half = (warp - 2) >> 2;
-        const uint32_t qaddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kScoreCol;
-        for (int tb = half * 32; tb < nt; tb += 64) {
-          uint32_t v[32];
-          tmem_ld32(qaddr + tb, v);
-          tmem_wait_ld();
+      const float4* src =
+          reinterpret_cast<const float4*>(a.scg + (static_cast<int64_t>(r) * a.chunks + c) * (kMaxChunkTiles * kTileM));
+      float4* dst = reinterpret_cast<float4*>(sc);
+      const int n4 = nt * (kTileM / 4);
+      constexpr int U = 4;
+      for (int i0 = tid; i0 < n4; i0 += U * kThreads) {
+        float4 v[U];
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (tb + u < nt) sc[(tb + u) * kTileM + q * 32 + lane] = __uint_as_float(v[u]);
-        }
+        for (int u = 0; u < U; ++u)
+          if (i0 + u * kThreads < n4) v[u] = __ldcg(src + i0 + u * kThreads);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (i0 + u * kThreads < n4) dst[i0 + u * kThreads] = v[u];
       }
     };
     // block maxima of the chunk (the chunk starts on a tile, so on a block)
@@ -1357,7 +1369,8 @@ size_t index_tc_workspace_bytes(int batch, int64_t cap, int k) {
   b += static_cast<size_t>(batch) * ch * 2 * 4;                       // cnt
   b += static_cast<size_t>(batch) * ch * k * 8;                       // staging above
   b += static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 8;  // staging boundary
-  return b + 4 * 256;
+  b += static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 4;  // scores
+  return b + 5 * 256;
 }
 
 // `ws` must hold index_tc_workspace_bytes; its first index_tc_control_bytes
@@ -1449,6 +1462,7 @@ csa_status_t launch_index_topk_tc(const csa_params_t* p, int batch, const csa_te
   a.cnt = reinterpret_cast<uint32_t*>(take(static_cast<size_t>(batch) * ch * 2 * 4));
   a.st = reinterpret_cast<uint2*>(take(static_cast<size_t>(batch) * ch * p->topk * 8));
   a.eq = reinterpret_cast<uint2*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 8));
+  a.scg = reinterpret_cast<float*>(take(static_cast<size_t>(batch) * ch * kMaxChunkTiles * kTileM * 4));
 
   const int smem = fp8 ? Cfg<true>::kSmem : Cfg<false>::kSmem;
   const int mode = pool ? kModePool : bmax ? kModeBmax
