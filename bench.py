@@ -589,7 +589,7 @@ def prefill_kernel_work(name, wl, sum_vis, sum_keys):
         return 2.0 * wl.h_idx * wl.d_idx * sum_vis, "tensor"
     if name.startswith("index_score"):
         return 2.0 * wl.h_idx * wl.d_idx * sum_vis, "alu"
-    if name.startswith("attn_tc"):
+    if name.startswith("attn_tc") or name.startswith("attn_many"):
         return 4.0 * wl.h_q * wl.d * sum_keys, "tensor"
     if name.startswith("attn"):
         return 4.0 * wl.h_q * wl.d * sum_keys, "alu"
@@ -720,7 +720,7 @@ def run_prefill(args, rank, world, local_rank):
     else:
         roof = {"bound": None, "unit": None, "achieved": None, "peak": None, "peak_source": None}
     roof.update({"kernel": dom, "frac": roof["achieved"] / roof["peak"] if roof["achieved"] else None,
-                 "traffic": None, "algorithmic_work": work, "avg_ms": dom_ms})
+                 "traffic": load_traffic(dom, "prefill"), "algorithmic_work": work, "avg_ms": dom_ms})
 
     def kernel_roof(name, c, t):
         """Each kernel's own work against its own roof (tensor: measured bf16

@@ -388,17 +388,27 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
                                  const csa_tensor_t* out, float* lse, void* workspace, int max_keys,
                                  cudaStream_t stream);
 
-// The tensor-core attention takes few queries, each cut into 128-key
-// splits (decode); many queries (prefill) use the CUDA-core kernel.
+csa_status_t launch_attention_many_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
+                                      int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
+                                      const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
+                                      const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
+                                      const csa_tensor_t* out, float* lse, cudaStream_t stream);
+
+// Tensor-core attention (64 heads of 512): few queries (decode) are each
+// cut over the CTAs of a cluster, or into 128-key splits merged by a second
+// kernel; many queries (prefill) take one CTA each that loops over the
+// query's keys (no workspace).
+constexpr int kManyQueries = 64;
 static bool attn_tc_shape(int nq, int hq, int d, int max_keys, int window) {
-  if (hq != 64 || d != 512 || attn_tc_splits(max_keys) > kMaxSplits) return false;
-  return nq <= 64 || attn_cluster_min(max_keys - window, window) > 0;
+  (void)window;
+  if (hq != 64 || d != 512) return false;
+  return nq > kManyQueries || attn_tc_splits(max_keys) <= kMaxSplits;
 }
 
 size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys, int window) {
   const int s = attn_splits(nq, max_keys);
   size_t b = s <= 1 ? 0 : static_cast<size_t>(nq) * s * hq * (d + 2) * sizeof(float);
-  if (attn_tc_shape(nq, hq, d, max_keys, window) && nq <= 64) {
+  if (attn_tc_shape(nq, hq, d, max_keys, window) && nq <= kManyQueries) {
     const size_t t = attn_tc_workspace_bytes(nq, max_keys);
     if (t > b) b = t;
   }
@@ -412,9 +422,13 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               void* workspace, int max_keys, cudaStream_t stream) {
   if (nq == 0) return CSA_OK;
   if (attn_tc_shape(nq, p->h_q, p->d, max_keys, p->window) &&
-      attn_tc_supported(p, q->dtype, kv->dtype, swa_k ? swa_k->dtype : kBF16, p->window > 0))
+      attn_tc_supported(p, q->dtype, kv->dtype, swa_k ? swa_k->dtype : kBF16, p->window > 0)) {
+    if (nq > kManyQueries)
+      return launch_attention_many_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo,
+                                      sink, out, lse, stream);
     return launch_attention_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink,
                                out, lse, workspace, max_keys, stream);
+  }
   AttnArgs a;
   a.q = q->data; a.q_dtype = q->dtype;
   a.kv = kv->data; a.kv_scale = kv->scale; a.kv_dtype = kv->dtype;

@@ -1,0 +1,480 @@
+// K4 + K5 on the tensor cores for many query tokens (chunked prefill): one
+// CTA per query, 64 heads of d = 512, looping over the query's key list --
+// its selected compressed entries (CSA) or every visible entry (HCA), then
+// its window positions -- in tiles of 128 keys, with one online softmax
+// whose running sums stay on chip for the whole list.
+//
+// Atlas "Model architectures", "compressed KV" (CSA top-k entries plus a
+// sliding window; HCA dense) and "MLA" (the latent is key and value);
+// tech-report tour, "The indexer selects, SWA covers the rest" (the query
+// attends to the selected entries together with the sliding-window KV).
+//
+// Per tile (attn_tile.cuh's layouts):
+//   1. gather: key rows -> bf16, K-major 128-byte swizzled tile (all warps);
+//   2. S^T[128 keys][64 heads] = K Q^T (tcgen05, M = 128, N = 64, K = 512);
+//      the query (64 KB) was loaded once by TMA;
+//   3. warps 4-7 read S^T from TMEM (a key per thread, 64 heads in
+//      registers), reduce the tile's per-head maximum across the keys with
+//      a transposing butterfly, and write P^T = exp(S - m) as bf16; warps
+//      0-3 meanwhile replace the window rows' keys with their values;
+//   4. O^T[512][64] += V^T P^T (tcgen05, the tile as an MN-major A operand),
+//      accumulated in TMEM over all tiles.
+// The running maximum m is updated lazily: a head's m moves only when a
+// tile's maximum exceeds it by more than kLazy (P <= e^kLazy meanwhile,
+// exact in bf16's range), and only then is its column of O rescaled in
+// TMEM.  The sink enters the denominator once at the end; out = O / L and
+// lse = M + log L exactly as in the single-tile kernels.
+#include <cudaTypedefs.h>
+
+#include "attn_tile.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+namespace {
+
+using namespace sm100;
+using namespace attn;
+
+constexpr uint32_t kTmemColsM = 512;  // S^T 64 columns + O^T 256 columns
+constexpr float kLazy = 8.f;          // nats a tile maximum may exceed m before m moves
+
+// shared memory, from a 1024-byte aligned base
+constexpr int mK = 0;                       // 8 x 16 KB key / value tile
+constexpr int mQ = mK + 8 * kTK * 128;      // 8 x 8 KB query
+constexpr int mP = mQ + 8 * kH * 128;       // 2 x 8 KB P^T (bf16, K-major over keys)
+constexpr int mRed = mP + 2 * kH * 128;     // [4][64] per-warp partial maxima / sums
+constexpr int mStat = mRed + 4 * kH * 4;    // m[64], l[64], rescale factor[64], final scale[64]
+constexpr int mEnt = mStat + 4 * kH * 4;    // [128] entry codes of the tile
+constexpr int mBars = mEnt + kTK * 4;
+constexpr int mMisc = mBars + 64;
+constexpr int mLut = mMisc + 64;            // MXFP4 code-byte table, 256 x bf16x2
+constexpr int kSmemM = mLut + 1024 + 1024;  // + alignment slack
+static_assert(kSmemM <= 232448, "shared memory");
+static_assert(mP % 1024 == 0, "operand alignment");
+
+__device__ uint32_t g_attn_many_error = 0;
+
+struct AttnManyArgs {
+  const void* kv; const void* kv_scale; int batch; int64_t cap;
+  const int32_t* idx; int topk;   // idx == nullptr: dense over n_visible
+  const int32_t* n_visible; const int32_t* q_req;
+  const uint16_t* swa_k; const uint16_t* swa_v; int swa_cap; int window;
+  const int64_t* q_pos; const int64_t* swa_lo;
+  float tau;
+  const float* sink; void* out; int out_dtype; float* lse;
+};
+
+__device__ __forceinline__ uint8_t* align1024m(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// Butterfly over the warp's 32 lanes that reduces 32 per-lane values (one
+// per head of a half) with `op` while transposing them: afterwards lane l
+// holds the warp's result for head l of the half in v[0].  31 shuffles.
+template <class Op>
+__device__ __forceinline__ void warp_reduce32(float (&v)[32], Op op) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < 5; ++r) {
+    const int o = 16 >> r;   // partner distance
+    const int n = 32 >> r;   // values still held
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? v[i] : v[i + n / 2];
+      const float keep = upper ? v[i + n / 2] : v[i];
+      v[i] = op(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+    }
+  }
+}
+
+struct MaxOp {
+  __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct SumOp {
+  __device__ float operator()(float a, float b) const { return a + b; }
+};
+
+// All 128 threads of warps 0-3: the tile's window rows (entry codes <= -2)
+// take their value rows (compressed entries are their own values).
+__device__ void gather_window_values(uint8_t* tile, const int32_t* ent, const Src& a) {
+  constexpr int B = 8;
+  const int t = static_cast<int>(threadIdx.x);  // 0..127
+  for (int t0 = t; t0 < kTK * 64; t0 += 128 * B) {
+    uint4 v[B];
+    bool put[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int task = t0 + b * 128;
+      const int32_t e = task < kTK * 64 ? ent[task >> 6] : -1;
+      put[b] = e <= -2;
+      v[b] = put[b] ? __ldg(reinterpret_cast<const uint4*>(a.swa_v + (a.sw_row0 + (-2 - e)) * kD) + (task & 63))
+                    : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int task = t0 + b * 128;
+      if (put[b]) put_chunk(tile, task >> 6, (task & 63) * 8, v[b]);
+    }
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kNT, 1)
+attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024m(smem_raw);
+  uint8_t* Kt = smem + mK;
+  uint8_t* Pt = smem + mP;
+  float* red = reinterpret_cast<float*>(smem + mRed);
+  float* m_run = reinterpret_cast<float*>(smem + mStat);
+  float* l_run = m_run + kH;
+  float* fac = l_run + kH;
+  float* fin = fac + kH;
+  int32_t* ent = reinterpret_cast<int32_t*>(smem + mEnt);
+  uint64_t* qbar = reinterpret_cast<uint64_t*>(smem + mBars);
+  uint64_t* sbar = qbar + 1;
+  uint64_t* obar = qbar + 2;
+  uint64_t* mdone = qbar + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + mMisc);
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + mMisc + 16);  // [0] rescale, [1] failed
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qi = blockIdx.x;
+  const int r = a.q_req ? a.q_req[qi] : qi;
+  const bool live = r >= 0 && r < a.batch;
+  const int nv = static_cast<int>(min(max(static_cast<int64_t>(a.n_visible[qi]), int64_t(0)), a.cap));
+  const int n_sel = a.idx ? a.topk : nv;
+  const int64_t t = a.q_pos[qi];
+  int64_t p_lo = t - a.window + 1;
+  if (a.swa_lo && a.swa_lo[qi] > p_lo) p_lo = a.swa_lo[qi];
+  if (p_lo < 0) p_lo = 0;
+  const int n_win = (a.window > 0 && t >= p_lo) ? static_cast<int>(t - p_lo + 1) : 0;
+  const int total = live ? n_sel + n_win : 0;
+  const int ntiles = (total + kTK - 1) / kTK;
+
+  if (tid == 0) {
+    prefetch_tensormap(&qmap);
+    mbar_init(qbar, 1);
+    mbar_init(sbar, 1);
+    mbar_init(obar, 1);
+    mbar_init(mdone, 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_barrier_init();
+    if (ntiles > 0) {  // the query, once; its load overlaps the first gather
+      mbar_arrive_expect_tx(qbar, kH * kD * 2);
+      for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + mQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
+    }
+  }
+  if (tid < kH) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.f;
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemColsM);
+  if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + mLut));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t dS = tmem, dO = tmem + kH;
+  Src src;
+  src.kv = a.kv;
+  src.kv_scale = a.kv_scale;
+  src.lut = reinterpret_cast<const uint32_t*>(smem + mLut);
+  src.swa_k = a.swa_k;
+  src.swa_v = a.swa_v;
+  src.kv_row0 = live ? static_cast<int64_t>(r) * a.cap : 0;
+  src.sw_row0 = live ? static_cast<int64_t>(r) * a.swa_cap : 0;
+  src.tau = a.tau;
+  const int sub = warp & 3;
+
+  for (int j = 0; j < ntiles; ++j) {
+    // entry codes of tile j: selected entry (>= 0), window slot (-2 - slot), nothing (-1)
+    if (tid < kTK) {
+      const int x = j * kTK + tid;
+      int32_t e = -1;
+      if (x < total) {
+        if (x < n_sel) {
+          const int32_t jj = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
+          e = (jj >= 0 && jj < nv) ? jj : -1;
+        } else {
+          e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
+        }
+      }
+      ent[tid] = e;
+    }
+    if (tid == 128) flags[0] = 0;
+    __syncthreads();
+    gather_rows<FMT>(Kt, ent, src, 0);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (flags[1]) break;
+    // ---- S^T = K Q^T ----
+    if (tid == 32) {
+      bool ok = true;
+      if (j == 0) ok = mbar_wait(qbar, 0, kWaitLimit);
+      if (!ok) {
+        atomicOr(&g_attn_many_error, 1u);
+        flags[1] = 1;
+      } else {
+        tc_fence_after();
+        const uint32_t kb = smem_u32(Kt), qb = smem_u32(smem + mQ);
+#pragma unroll
+        for (int blk = 0; blk < 8; ++blk)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(dS, desc_k_sw128(kb + blk * kTK * 128 + kk * 32), desc_k_sw128(qb + blk * kH * 128 + kk * 32),
+                    kIdescS, (blk | kk) ? 1u : 0u);
+        mma_commit(sbar);
+      }
+    }
+    if (tid == 0 && !mbar_wait(sbar, j & 1, kWaitLimit)) {
+      atomicOr(&g_attn_many_error, 1u);
+      flags[1] = 1;
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (flags[1]) break;
+    const int x0 = j * kTK;
+    const bool any_window = n_win > 0 && x0 + kTK > n_sel && x0 < total;
+    if (warp < 4) {
+      if (any_window) gather_window_values(Kt, ent, src);
+    } else {
+      const int row = sub * 32 + lane;  // key of the tile this thread reads
+      const bool row_ok = ent[row] != -1;
+      const uint32_t taS = dS + (static_cast<uint32_t>(sub * 32) << 16);
+      // this thread's logits of heads hh .. hh + 31 (its key), from TMEM
+      auto load_logits = [&](int hh, float (&s)[32]) {
+        uint32_t v[32];
+        tmem_ld32(taS + hh, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) s[h] = row_ok ? __uint_as_float(v[h]) * a.tau : -INFINITY;
+      };
+      // the tile's maximum of every head: per warp (lane l: head hh + l),
+      // then over the 4 warps
+#pragma unroll 1
+      for (int hh = 0; hh < kH; hh += 32) {
+        float s[32];
+        load_logits(hh, s);
+        warp_reduce32(s, MaxOp());
+        red[sub * kH + hh + lane] = s[0];
+      }
+      named_barrier(1, 128);
+      if (tid < 128 + kH) {
+        const int h = tid - 128;
+        const float mt = fmaxf(fmaxf(red[h], red[kH + h]), fmaxf(red[2 * kH + h], red[3 * kH + h]));
+        const float mo = m_run[h];
+        float f = 1.f, mu = mo;
+        if (mt != -INFINITY) {
+          if (mo == -INFINITY) {
+            mu = mt;  // no mass yet: this head's O and l are zero
+          } else if (mt > mo + kLazy) {
+            f = __expf(mo - mt);
+            mu = mt;
+            flags[0] = 1;
+          }
+        }
+        m_run[h] = mu;
+        fac[h] = f;
+      }
+      named_barrier(1, 128);
+      // P = exp(S - m) as bf16 into P^T [head][key]; the sums in fp32
+#pragma unroll 1
+      for (int hh = 0; hh < kH; hh += 32) {
+        float s[32];
+        load_logits(hh, s);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          const float mu = m_run[hh + h];
+          const float p = (s[h] == -INFINITY || mu == -INFINITY) ? 0.f : __expf(s[h] - mu);
+          s[h] = p;
+          *reinterpret_cast<uint16_t*>(Pt + (row >> 6) * (kH * 128) + sw128_offset(hh + h, (row & 63) >> 3) +
+                                       (row & 7) * 2) = f32_to_bf16_bits(p);
+        }
+        warp_reduce32(s, SumOp());
+        red[sub * kH + hh + lane] = s[0];
+      }
+      named_barrier(1, 128);
+      if (tid < 128 + kH) {
+        const int h = tid - 128;
+        l_run[h] = l_run[h] * fac[h] + ((red[h] + red[kH + h]) + (red[2 * kH + h] + red[3 * kH + h]));
+      }
+      // a head whose m moved: its column of O (all 512 dims) by the factor
+      if (j > 0 && flags[0]) {
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
+          uint32_t v0[32], v1[32];
+          tmem_ld32(ta, v0);
+          tmem_ld32(ta + 32, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            v0[h] = __float_as_uint(__uint_as_float(v0[h]) * fac[h]);
+            v1[h] = __float_as_uint(__uint_as_float(v1[h]) * fac[32 + h]);
+          }
+          tmem_st32(ta, v0);
+          tmem_st32(ta + 32, v1);
+        }
+        tmem_wait_st();
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- O^T += V^T P^T ----
+    if (tid == 32) {
+      const uint32_t kb = smem_u32(Kt), pb = smem_u32(Pt);
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int kk = 0; kk < kTK / 16; ++kk)
+          mma_f16(dO + mt * kH, desc_mn_sw128(kb + (2 * mt) * kTK * 128 + kk * 16 * 128, kTK * 128),
+                  desc_k_sw128(pb + (kk >> 2) * kH * 128 + (kk & 3) * 32), kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(obar);
+    }
+    if (tid == 0 && !mbar_wait(obar, j & 1, kWaitLimit)) {
+      atomicOr(&g_attn_many_error, 1u);
+      flags[1] = 1;
+    }
+    __syncthreads();  // the next tile may overwrite the key tile and P^T
+    tc_fence_after();
+    if (flags[1]) break;
+  }
+
+  // ---- out = O / L with the sink in L; lse = M + log L ----
+  const bool done = !flags[1];
+  if (tid < kH) {
+    const int h = tid;
+    const float m = m_run[h], l = l_run[h];
+    const float sk = a.sink ? a.sink[h] : -INFINITY;
+    const float M = fmaxf(m, sk);
+    float scale = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+      const float am = (m == -INFINITY) ? 0.f : __expf(m - M);
+      L = l * am + ((sk == -INFINITY) ? 0.f : __expf(sk - M));
+      scale = am / L;
+    }
+    fin[h] = (ntiles > 0 && done) ? scale : 0.f;
+    if (a.lse) a.lse[static_cast<int64_t>(qi) * kH + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
+  }
+  __syncthreads();
+  if (warp >= 4) {
+    const int oeb = a.out_dtype == kF32 ? 4 : 2;
+    char* obase = static_cast<char*>(a.out) + static_cast<int64_t>(qi) * kH * kD * oeb;
+#pragma unroll 1
+    for (int mt = 0; mt < 4; ++mt) {
+      const int dim = mt * 128 + sub * 32 + lane;
+      uint32_t v0[32], v1[32];
+      if (ntiles > 0) {
+        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int h = 0; h < 64; ++h) {
+        const float o = ntiles > 0 ? __uint_as_float(h < 32 ? v0[h] : v1[h - 32]) * fin[h] : 0.f;
+        if (a.out_dtype == kF32) reinterpret_cast<float*>(obase)[h * kD + dim] = o;
+        else reinterpret_cast<uint16_t*>(obase)[h * kD + dim] = f32_to_bf16_bits(o);
+      }
+    }
+  }
+  // every MMA of this CTA and the query's copy have completed before TMEM
+  // is released and the CTA exits
+  if (tid == 32) {
+    mma_commit(mdone);
+    mbar_wait(mdone, 0, kWaitLimit);
+    if (ntiles > 0) mbar_wait(qbar, 0, kWaitLimit);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemColsM);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 many_attn_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+template <int FMT>
+csa_status_t launch_many_fmt(const CUtensorMap& qmap, const AttnManyArgs& a, int nq, cudaStream_t stream) {
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_many_tc_kernel<FMT>),
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemM);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  prof_begin(stream);
+  attn_many_tc_kernel<FMT><<<nq, kNT, kSmemM, stream>>>(qmap, a);
+  return check_launch("attn_many_tc_kernel", stream);
+}
+
+}  // namespace
+
+// Many queries (no workspace): h_q = 64, d = 512, bf16 queries, bf16 window,
+// main KV in bf16, FP8 (scale per 64) or MXFP4; the caller checked them.
+csa_status_t launch_attention_many_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
+                                      int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
+                                      const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
+                                      const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
+                                      const csa_tensor_t* out, float* lse, cudaStream_t stream) {
+  if (nq == 0) return CSA_OK;
+  if (!many_attn_encoder()) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  CUtensorMap qmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(nq) * kH};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kH)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult cr = many_attn_encoder()(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q->data, dims, strides, box, estr,
+                                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled (query) failed (%d)", (int)cr);
+  AttnManyArgs a;
+  a.kv = kv->data;
+  a.kv_scale = kv->scale;
+  a.batch = batch;
+  a.cap = cap;
+  a.idx = idx;
+  a.topk = p->topk;
+  a.n_visible = n_visible;
+  a.q_req = q_req;
+  a.swa_k = swa_k ? static_cast<const uint16_t*>(swa_k->data) : nullptr;
+  a.swa_v = swa_v ? static_cast<const uint16_t*>(swa_v->data) : nullptr;
+  a.swa_cap = p->swa_cap > 0 ? p->swa_cap : 1;
+  a.window = p->window;
+  a.q_pos = q_pos;
+  a.swa_lo = swa_lo;
+  a.tau = p->softmax_scale;
+  a.sink = sink;
+  a.out = out->data;
+  a.out_dtype = out->dtype;
+  a.lse = lse;
+  if (kv->dtype == kMXFP4) return launch_many_fmt<kKvMX4>(qmap, a, nq, stream);
+  if (kv->dtype == kFP8) return launch_many_fmt<kKvFP8>(qmap, a, nq, stream);
+  return launch_many_fmt<kKvBF16>(qmap, a, nq, stream);
+}
+
+uint32_t attn_many_take_error() {
+  uint32_t v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_many_error, sizeof(v)) != cudaSuccess) return 0;
+  if (v) cudaMemcpyToSymbol(g_attn_many_error, &z, sizeof(z));
+  return v;
+}
+
+}  // namespace csa

@@ -54,6 +54,7 @@ csa_status_t launch_index_many_tc(const csa_params_t* p, int nq, const csa_tenso
                                   const int32_t* n_visible, float* scores, int64_t ld, int32_t* table,
                                   cudaStream_t stream);
 uint32_t index_many_take_error();
+uint32_t attn_many_take_error();
 csa_status_t launch_pool_map(const int32_t* pos, const float* pos_score, int nq, int k, const int32_t* pool, int block,
                              int pool_blocks, int32_t* out_idx, cudaStream_t stream);
 csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
@@ -696,6 +697,8 @@ csa_status_t csa_sync_status(csa_stream_t stream) {
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the multi-CTA top-k gave up");
   if (index_many_take_error() != 0)
     return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the many-query indexer gave up");
+  if (attn_many_take_error() != 0)
+    return set_error(CSA_ERR_TIMEOUT, "a bounded device-side wait of the many-query attention gave up");
   return CSA_OK;
 }
 

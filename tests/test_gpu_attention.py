@@ -32,6 +32,18 @@ CASES = {
     "mxfp4_many_queries": (Wk.WORKLOADS["decode1m_fp4"], 40, 4, 1200, 128, False, True, False, 1.0),
     "tiny_mxfp4": (Wk.WORKLOADS["tiny"].scaled(kv_dtype="mxfp4", kv_group=16), 3, 2, 1024, 128, False, True, False,
                    1.0),
+    # more than 64 queries: one CTA per query looping over 128-key tiles
+    # (the chunked-prefill path), every main-KV format, dense and sparse
+    "many_bf16_csa": (Wk.WORKLOADS["decode64k"], 96, 3, 3000, 128, False, True, False, 1.0),
+    "many_fp8_csa": (Wk.WORKLOADS["decode1m"], 80, 2, 4000, 128, False, True, False, 1.0),
+    "many_mxfp4_csa": (Wk.WORKLOADS["decode1m_fp4"], 72, 2, 4000, 128, False, True, False, 1.0),
+    "many_bf16_hca": (Wk.WORKLOADS["hybrid_hca"], 70, 2, 700, 128, True, True, False, 1.0),
+    "many_nosink_replay": (Wk.WORKLOADS["decode64k"], 66, 2, 2000, 256, False, False, True, 1.0),
+    "many_no_window": (Wk.WORKLOADS["decode64k"].scaled(window=0), 65, 3, 800, 128, False, True, False, 1.0),
+    # logits spread over tens of nats: a head's running maximum moves by more
+    # than the lazy threshold between tiles, so O is rescaled in TMEM
+    "many_very_sharp": (Wk.WORKLOADS["decode64k"], 68, 2, 1500, 128, False, True, False, 512.0),
+    "many_top300": (Wk.WORKLOADS["decode64k"].scaled(topk=300), 90, 2, 2000, 128, False, True, False, 1.0),
 }
 
 
