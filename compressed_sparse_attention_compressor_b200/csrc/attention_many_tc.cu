@@ -96,27 +96,46 @@ struct SumOp {
   __device__ float operator()(float a, float b) const { return a + b; }
 };
 
+// Shared-memory address of 16-byte chunk c8 (elements 8 c8 .. 8 c8 + 7) of
+// tile row r (put_chunk's layout).
+__device__ __forceinline__ uint8_t* chunk_addr(uint8_t* tile, int r, int c8) {
+  return tile + (c8 >> 3) * (kTK * 128) + sw128_offset(r, c8 & 7);
+}
+
 // All 128 threads of warps 0-3: the tile's window rows (entry codes <= -2)
-// take their value rows (compressed entries are their own values).
+// take their value rows (compressed entries are their own values), by
+// asynchronous 16-byte copies, all in flight at once.
 __device__ void gather_window_values(uint8_t* tile, const int32_t* ent, const Src& a) {
-  constexpr int B = 8;
   const int t = static_cast<int>(threadIdx.x);  // 0..127
-  for (int t0 = t; t0 < kTK * 64; t0 += 128 * B) {
-    uint4 v[B];
-    bool put[B];
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const int task = t0 + b * 128;
-      const int32_t e = task < kTK * 64 ? ent[task >> 6] : -1;
-      put[b] = e <= -2;
-      v[b] = put[b] ? __ldg(reinterpret_cast<const uint4*>(a.swa_v + (a.sw_row0 + (-2 - e)) * kD) + (task & 63))
-                    : make_uint4(0, 0, 0, 0);
+  for (int task = t; task < kTK * 64; task += 128) {
+    const int32_t e = ent[task >> 6];
+    if (e <= -2)
+      cp_async16(chunk_addr(tile, task >> 6, task & 63),
+                 reinterpret_cast<const uint4*>(a.swa_v + (a.sw_row0 + (-2 - e)) * kD) + (task & 63));
+  }
+  cp_async_wait_all();
+}
+
+// All threads: the tile's key rows.  bf16 rows (compressed bf16 entries,
+// window keys) by asynchronous 16-byte copies, all issued before any wait;
+// FP8 / MXFP4 compressed rows through registers (dequantised to bf16);
+// rows without a key (-1) zeroed.
+template <int FMT>
+__device__ void gather_keys(uint8_t* tile, const int32_t* ent, const Src& a) {
+  if constexpr (FMT != kKvBF16) gather_rows<FMT>(tile, ent, a, 0);  // quantised rows (and the rest)
+  else {
+    for (int task = static_cast<int>(threadIdx.x); task < kTK * 64; task += kNT) {
+      const int r = task >> 6, c8 = task & 63;
+      const int32_t e = ent[r];
+      uint8_t* dst = chunk_addr(tile, r, c8);
+      if (e >= 0)
+        cp_async16(dst, reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + (a.kv_row0 + e) * kD) + c8);
+      else if (e <= -2)
+        cp_async16(dst, reinterpret_cast<const uint4*>(a.swa_k + (a.sw_row0 + (-2 - e)) * kD) + c8);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
     }
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      const int task = t0 + b * 128;
-      if (put[b]) put_chunk(tile, task >> 6, (task & 63) * 8, v[b]);
-    }
+    cp_async_wait_all();
   }
 }
 
@@ -207,7 +226,7 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     }
     if (tid == 128) flags[0] = 0;
     __syncthreads();
-    gather_rows<FMT>(Kt, ent, src, 0);
+    gather_keys<FMT>(Kt, ent, src);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();

@@ -266,8 +266,12 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t d = score_key(v[u][c]) - lo;
-          if (j0 + 4 * (u * kTopkThreads + tid) + c < n && static_cast<uint64_t>(d) < span)
-            atomicAdd(&sh.hist[d >> shift], 1u);
+          const bool in = j0 + 4 * (u * kTopkThreads + tid) + c < n && static_cast<uint64_t>(d) < span;
+          // lanes that hit the same bin add together: one atomic per
+          // distinct bin and warp (scores crowd into few bins)
+          const uint32_t bin = in ? (d >> shift) : 0xFFFFFFFFu;
+          const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+          if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], static_cast<uint32_t>(__popc(peers)));
         }
     }
     __syncthreads();
