@@ -386,7 +386,7 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
                                  const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
                                  const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
                                  const csa_tensor_t* out, float* lse, void* workspace, int max_keys,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool pdl);
 
 csa_status_t launch_attention_many_tc(const csa_params_t* p, int nq, const csa_tensor_t* q, const csa_tensor_t* kv,
                                       int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible,
@@ -419,7 +419,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible, const int32_t* q_req,
                               const csa_tensor_t* swa_k, const csa_tensor_t* swa_v, const int64_t* q_pos,
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
-                              void* workspace, int max_keys, cudaStream_t stream) {
+                              void* workspace, int max_keys, cudaStream_t stream, bool pdl) {
   if (nq == 0) return CSA_OK;
   if (attn_tc_shape(nq, p->h_q, p->d, max_keys, p->window) &&
       attn_tc_supported(p, q->dtype, kv->dtype, swa_k ? swa_k->dtype : kBF16, p->window > 0)) {
@@ -427,7 +427,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
       return launch_attention_many_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo,
                                       sink, out, lse, stream);
     return launch_attention_tc(p, nq, q, kv, batch, cap, idx, n_visible, q_req, swa_k, swa_v, q_pos, swa_lo, sink,
-                               out, lse, workspace, max_keys, stream);
+                               out, lse, workspace, max_keys, stream, pdl);
   }
   AttnArgs a;
   a.q = q->data; a.q_dtype = q->dtype;

@@ -85,6 +85,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qi = blockIdx.y, split = blockIdx.x;
+  // barriers, the query's TMA, TMEM: nothing an earlier kernel of the
+  // decode step writes (the query is the caller's input)
+  auto prologue = [&]() {
+    if (tid == 0) {
+      prefetch_tensormap(&qmap);
+      mbar_init(qbar, 1);
+      mbar_init(sbar, 1);
+      mbar_init(obar, 1);
+      s_flags[0] = 0;
+      s_flags[1] = 0;
+      fence_barrier_init();
+      // the query first: its load overlaps the gather of the keys
+      mbar_arrive_expect_tx(qbar, kH * kD * 2);
+      for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + oQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+    if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + oLut));
+  };
+  // cluster path: the prologue runs before the wait for the previous
+  // kernel (a programmatic launch overlaps it with that kernel's tail);
+  // everything below reads the selection, positions and window it wrote
+  if constexpr (CLUSTER) prologue();
+  grid_dependency_wait();
   const int r = a.q_req ? a.q_req[qi] : qi;
   const bool live = r >= 0 && r < a.batch;
   const int nv = static_cast<int>(min(max(static_cast<int64_t>(a.n_visible[qi]), int64_t(0)), a.cap));
@@ -114,18 +137,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     return;
   }
 
-  if (tid == 0) {
-    prefetch_tensormap(&qmap);
-    mbar_init(qbar, 1);
-    mbar_init(sbar, 1);
-    mbar_init(obar, 1);
-    s_flags[0] = 0;
-    s_flags[1] = 0;
-    fence_barrier_init();
-    // the query first: its load overlaps the gather of the keys
-    mbar_arrive_expect_tx(qbar, kH * kD * 2);
-    for (int blk = 0; blk < 8; ++blk) tma_load_2d(smem + oQ + blk * kH * 128, &qmap, qbar, blk * 64, qi * kH);
-  }
+  if constexpr (!CLUSTER) prologue();
   if (tid < kTK) {
     int32_t e = -1;
     int xs = -1, xw = -1;  // selected-list position / window offset of this row
@@ -147,8 +159,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     }
     ent[tid] = e;
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-  if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + oLut));
   __syncthreads();
 
   if (tid < kTK && ent[tid] <= -2) s_flags[0] = 1;
@@ -331,7 +341,7 @@ csa_status_t launch_attn_merge(const float* part, int nq, int n_splits, int hq, 
 template <int FMT>
 csa_status_t launch_attn_fmt(TcLauncher& L, const csa_params_t* p, int nq, int max_keys, const CUtensorMap& qmap,
                              const AttnTcArgs& a, const float* sink, const csa_tensor_t* out, float* lse,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool pdl) {
   for (int c = 0; c < 2; ++c)
     if (!L.attr[FMT][c]) {
       void* fn = c ? reinterpret_cast<void*>(attn_tc_kernel<true, FMT>) : reinterpret_cast<void*>(attn_tc_kernel<false, FMT>);
@@ -378,6 +388,14 @@ csa_status_t launch_attn_fmt(TcLauncher& L, const csa_params_t* p, int nq, int m
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cudaLaunchAttribute attr2[2] = {attr[0], {}};
+    if (pdl) {
+      // a programmatic launch: the prologue overlaps the previous kernel's tail
+      attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr2[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr2;
+      cfg.numAttrs = 2;
+    }
     {
       prof_begin(stream);
       const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true, FMT>, qmap, a);
@@ -402,7 +420,7 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
                                  const int32_t* q_req, const csa_tensor_t* swa_k, const csa_tensor_t* swa_v,
                                  const int64_t* q_pos, const int64_t* swa_lo, const float* sink,
                                  const csa_tensor_t* out, float* lse, void* workspace, int max_keys,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool pdl) {
   TcLauncher& L = tc_launcher();
   if (!L.encode) return set_error(CSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   CUtensorMap qmap;
@@ -437,9 +455,9 @@ csa_status_t launch_attention_tc(const csa_params_t* p, int nq, const csa_tensor
   a.out = out->data;
   a.out_dtype = out->dtype;
   a.lse = lse;
-  if (a.kv_fmt == kKvMX4) return launch_attn_fmt<kKvMX4>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
-  if (a.kv_fmt == kKvFP8) return launch_attn_fmt<kKvFP8>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
-  return launch_attn_fmt<kKvBF16>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream);
+  if (a.kv_fmt == kKvMX4) return launch_attn_fmt<kKvMX4>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream, pdl);
+  if (a.kv_fmt == kKvFP8) return launch_attn_fmt<kKvFP8>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream, pdl);
+  return launch_attn_fmt<kKvBF16>(L, p, nq, max_keys, qmap, a, sink, out, lse, stream, pdl);
 }
 
 uint32_t attn_tc_take_error() {

@@ -61,7 +61,7 @@ csa_status_t launch_attention(const csa_params_t* p, int nq, const csa_tensor_t*
                               int batch, int64_t cap, const int32_t* idx, const int32_t* n_visible, const int32_t* q_req,
                               const csa_tensor_t* swa_k, const csa_tensor_t* swa_v, const int64_t* q_pos,
                               const int64_t* swa_lo, const float* sink, const csa_tensor_t* out, float* lse,
-                              void* workspace, int max_keys, cudaStream_t stream);
+                              void* workspace, int max_keys, cudaStream_t stream, bool pdl = false);
 size_t attn_workspace_bytes(int nq, int hq, int d, int max_keys, int window);
 
 csa_status_t set_error(csa_status_t st, const char* fmt, ...);
@@ -619,8 +619,11 @@ csa_status_t csa_decode_step(const csa_params_t* p, int32_t batch, const csa_dec
       return st;
     if ((st = launch_topk(scores, batch, ld, n_vis, cc->cap, p->topk, idx, nullptr, s)) != CSA_OK) return st;
   }
+  // a programmatic launch: the attention's prologue overlaps the tail of the
+  // kernel before it (this step's indexer or append), whose outputs it
+  // reads only after a grid-dependency wait
   return launch_attention(p, batch, &tok->q, &cc->kv, batch, cc->cap, idx, n_vis, q_req, &cc->swa_k, &cc->swa_v, q_pos,
-                          nullptr, tok->sink, out, lse, attn_ws, max_keys, s);
+                          nullptr, tok->sink, out, lse, attn_ws, max_keys, s, /*pdl=*/true);
 }
 
 csa_status_t csa_index_score(const csa_params_t* p, int32_t n_queries, const csa_tensor_t* q_idx, const float* w,

@@ -983,6 +983,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // a kernel launched programmatically after this one (the decode step's
+  // attention) may start its prologue on the SMs this grid frees; it reads
+  // this grid's outputs only after waiting for its completion
+  grid_launch_dependents();
 
   if (!sh.fail) {
     // ================= phase 2: exact top-k over the request =================

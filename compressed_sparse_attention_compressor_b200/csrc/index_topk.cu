@@ -144,20 +144,11 @@ __device__ void find_bin(TopkShared& sh, int nb, uint32_t need) {
 
 // Four consecutive scores of a row (zero past n), as one 16-byte load when
 // the row start allows it: each thread keeps several loads in flight.
-// STAGED: the row has been copied into shared memory, and is read there.
-template <bool STAGED>
 struct Row4 {
   const float* s;
   int64_t n;
   bool vec;
   __device__ __forceinline__ void load(int64_t j, float (&v)[4]) const {  // j % 4 == 0
-    if constexpr (STAGED) {
-      // the staged copy holds round_up(n, 4) floats (zero-padded): j < n
-      // keeps the 16-byte read inside it
-      const float4 f = j < n ? *reinterpret_cast<const float4*>(s + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      v[0] = f.x; v[1] = j + 1 < n ? f.y : 0.f; v[2] = j + 2 < n ? f.z : 0.f; v[3] = j + 3 < n ? f.w : 0.f;
-      return;
-    }
     if (vec && j + 3 < n) {
       const float4 f = __ldg(reinterpret_cast<const float4*>(s + j));
       v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
@@ -168,15 +159,10 @@ struct Row4 {
   }
 };
 
-// STAGED: the row is first copied into dynamic shared memory (one pass over
-// global memory; every later pass reads shared memory); the launch gives at
-// least round_up(max_n, 4) floats of it.
-template <bool STAGED>
 __global__ void __launch_bounds__(kTopkThreads)
 topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
                 int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int nv_div, int ordered) {
   __shared__ TopkShared sh;
-  extern __shared__ __align__(16) float srow[];
   const int row = blockIdx.x;
   // valid columns: ceil(n_valid / nv_div), or max_n without n_valid
   const int64_t nv = n_valid ? (static_cast<int64_t>(n_valid[row]) + nv_div - 1) / nv_div : max_n;
@@ -194,37 +180,7 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
     return;
   }
 
-  const float* src = s;
-  if constexpr (STAGED) {
-    // the row into shared memory, zero-padded to a multiple of 4; 16-byte
-    // loads when the row is aligned (four in flight per thread)
-    const int64_t n4 = (n + 3) / 4;
-    const bool al = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
-    for (int64_t i0 = tid; i0 < n4; i0 += 4 * kTopkThreads) {
-      float4 f[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t i = i0 + u * kTopkThreads;
-        f[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < n4) {
-          if (al && 4 * i + 3 < n) {
-            f[u] = __ldg(reinterpret_cast<const float4*>(s) + i);
-          } else {
-            float t4[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) t4[c] = 4 * i + c < n ? __ldg(s + 4 * i + c) : 0.f;
-            f[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (i0 + u * kTopkThreads < n4) reinterpret_cast<float4*>(srow)[i0 + u * kTopkThreads] = f[u];
-    }
-    __syncthreads();
-    src = srow;
-  }
-  const Row4<STAGED> rs4{src, n, (reinterpret_cast<uintptr_t>(src) & 15) == 0};
+  const Row4 rs4{s, n, (reinterpret_cast<uintptr_t>(s) & 15) == 0};
   // radix select of the k-th largest key over the keys' own range: the
   // range [lo, lo + span) is cut into <= 2048 bins of 2^shift keys and
   // narrowed to the bin holding the k-th key until a bin is one key wide.
@@ -266,12 +222,8 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t d = score_key(v[u][c]) - lo;
-          const bool in = j0 + 4 * (u * kTopkThreads + tid) + c < n && static_cast<uint64_t>(d) < span;
-          // lanes that hit the same bin add together: one atomic per
-          // distinct bin and warp (scores crowd into few bins)
-          const uint32_t bin = in ? (d >> shift) : 0xFFFFFFFFu;
-          const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-          if (in && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], static_cast<uint32_t>(__popc(peers)));
+          if (j0 + 4 * (u * kTopkThreads + tid) + c < n && static_cast<uint64_t>(d) < span)
+            atomicAdd(&sh.hist[d >> shift], 1u);
         }
     }
     __syncthreads();
@@ -400,30 +352,12 @@ csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_
   return set_error(CSA_ERR_UNSUPPORTED, "indexer shape h_idx=%d d_idx=%d is not built", p->h_idx, p->d_idx);
 }
 
-// Rows of up to kStagedMax scores are staged in shared memory.
-constexpr int64_t kStagedMax = 40960;  // 160 KB
-
 csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
                          int32_t* out_idx, float* out_score, cudaStream_t stream, int nv_div, int ordered) {
   if (n_rows == 0) return CSA_OK;
-  if (max_n > k && max_n <= kStagedMax) {
-    const int smem = static_cast<int>((max_n + 3) / 4 * 16);
-    static bool attr = false;
-    if (!attr) {
-      const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(topk_row_kernel<true>),
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kStagedMax * 4));
-      if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      attr = true;
-    }
-    prof_begin(stream);
-    topk_row_kernel<true><<<n_rows, kTopkThreads, smem, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score,
-                                                                  nv_div, ordered);
-    return check_launch("topk_row_staged_kernel", stream);
-  }
   prof_begin(stream);
-  topk_row_kernel<false><<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score,
-                                                              nv_div, ordered);
+  topk_row_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score, nv_div,
+                                                       ordered);
   return check_launch("topk_row_kernel", stream);
 }
 

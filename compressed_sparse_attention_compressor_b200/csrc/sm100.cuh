@@ -217,6 +217,18 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Waits until the grids this one depends on (a programmatic launch after
+// them on the stream) have completed and their writes are visible; returns
+// at once otherwise.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets a grid launched programmatically after this one start as soon as
+// every CTA of this grid has executed it (or exited).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
