@@ -286,7 +286,10 @@ def run_ours(args, rank, world, local_rank):
     out = DevTensor.empty((B, wl.h_q, wl.d), "bf16" if wl.act_dtype != "f32" else "f32")
     lse = torch.empty((B, wl.h_q), dtype=torch.float32, device="cuda")
     ws = csa.workspace(csa.csa_workspace_size(p, B, inp.cap))
-    tok = csa.decode_token(c_t, z_t, k_t, v_t, q, q_idx, w, sink, w_ik)
+    # a dense (HCA) layer has no indexer: no indexer query, weights or key projection
+    sparse = not wl.dense
+    tok = csa.decode_token(c_t, z_t, k_t, v_t, q, q_idx if sparse else None, w if sparse else None, sink,
+                           w_ik if sparse else None)
     stream = torch.cuda.current_stream()
     del inp
 
@@ -348,8 +351,8 @@ def run_ours(args, rank, world, local_rank):
     # The token's inputs sit back to back in one pinned host buffer and one device
     # buffer (256-byte aligned slots), so each step moves them with one copy; the
     # step reads views of the device buffer.
-    toks = (c_t, z_t, k_t, v_t, q, q_idx)
-    srcs = [t.data for t in toks] + [w] + [t.scale for t in toks if t.scale is not None]
+    toks = (c_t, z_t, k_t, v_t, q, q_idx) if sparse else (c_t, z_t, k_t, v_t, q)
+    srcs = [t.data for t in toks] + ([w] if sparse else []) + [t.scale for t in toks if t.scale is not None]
     offs, total = [], 0
     for t in srcs:
         offs.append(total)
@@ -361,10 +364,14 @@ def run_ours(args, rank, world, local_rank):
         v_.copy_(t)
         views.append(v_)
     host_pack = dev_pack.cpu().pin_memory()
-    sc_views = iter(views[7:])
-    c_p, z_p, k_p, v_p, q_p, qi_p = (DevTensor(vw, t.dtype, next(sc_views) if t.scale is not None else None, t.group)
-                                     for vw, t in zip(views[:6], toks))
-    tok_p = csa.decode_token(c_p, z_p, k_p, v_p, q_p, qi_p, views[6], sink, w_ik)
+    nt = len(toks)
+    sc_views = iter(views[nt + (1 if sparse else 0):])
+    tv = [DevTensor(vw, t.dtype, next(sc_views) if t.scale is not None else None, t.group)
+          for vw, t in zip(views[:nt], toks)]
+    if sparse:
+        tok_p = csa.decode_token(*tv, views[nt], sink, w_ik)
+    else:
+        tok_p = csa.decode_token(*tv, None, None, sink, None)
     host_out = torch.empty_like(out.data, device="cpu").pin_memory()
     h2d = host_pack.numel()
     d2h = host_out.numel() * host_out.element_size()
