@@ -205,9 +205,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
   } else {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    // this CTA's O (unnormalised) into its own shared memory as [head][dim]
-    // fp32, over the key tile (both MMAs have completed)
+    // this CTA's O (unnormalised) into its own shared memory as [head][dim],
+    // over the key tile (both MMAs have completed): fp32, or bf16 pairs when
+    // the output is bf16 (half the bytes the merge moves between the CTAs;
+    // the merge accumulates in fp32, so a partial's rounding adds at most the
+    // output's own rounding error)
+    const bool pbf = a.out_dtype != kF32;
     float* Osm = reinterpret_cast<float*>(smem + oK);
+    uint32_t* Obf = reinterpret_cast<uint32_t*>(smem + oK);  // [64][256] bf16x2
     {
       const int sub = warp & 3, mh = warp >> 2;  // two warps per TMEM lane quarter
 #pragma unroll 1
@@ -218,17 +223,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
         tmem_ld32(ta + 32, v1);
         tmem_wait_ld();
         const int dim = mt * 128 + sub * 32 + lane;
+        if (pbf) {
+          // lanes 2i and 2i + 1 hold dims 2i and 2i + 1: even lanes store the pair
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          Osm[h * kD + dim] = __uint_as_float(v0[h]);
-          Osm[(32 + h) * kD + dim] = __uint_as_float(v1[h]);
+          for (int h = 0; h < 32; ++h) {
+            const float a0 = __uint_as_float(v0[h]), b0 = __shfl_down_sync(0xFFFFFFFFu, a0, 1);
+            const float a1 = __uint_as_float(v1[h]), b1 = __shfl_down_sync(0xFFFFFFFFu, a1, 1);
+            if ((lane & 1) == 0) {
+              Obf[h * (kD / 2) + dim / 2] = pack_bf16(a0, b0);
+              Obf[(32 + h) * (kD / 2) + dim / 2] = pack_bf16(a1, b1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            Osm[h * kD + dim] = __uint_as_float(v0[h]);
+            Osm[(32 + h) * kD + dim] = __uint_as_float(v1[h]);
+          }
         }
       }
     }
     cluster.sync();
-    // heads split + r * R for r = 0, 1, ...: warp w weighs head split + w R
+    // heads split + r * R for r = 0, 1, ...: this CTA finishes nh of them
     float* wgt = reinterpret_cast<float*>(smem + oS);  // [head][16 CTAs], then [head][2] (M, 1/L); logits are dead
     const int nh = (kH - split + R - 1) / R;
+    const int dim = tid * 2;  // two consecutive dims per thread
+    // bf16 partials: the first four heads' loads from every peer go out
+    // before the weights are computed (their round trips overlap)
+    uint32_t vb[4][16];
+    auto load_bf = [&](int w0) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < R && w0 + u < nh)
+            vb[u][j] = cluster.map_shared_rank(Obf, j)[(split + (w0 + u) * R) * (kD / 2) + dim / 2];
+    };
+    if (pbf) load_bf(0);
     for (int w = warp; w < nh; w += kThreads / 32) {
       const int h = split + w * R;
       float mj = -INFINITY, lj = 0.f;
@@ -250,39 +281,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
       }
     }
     __syncthreads();
-    // two consecutive dims per thread, R peers each, two heads per round:
-    // every peer's loads of both heads in flight before the sums
-    const int dim = tid * 2;
-    for (int w0 = 0; w0 < nh; w0 += 2) {
-      float2 v[2][16];
+    if (pbf) {
+      for (int w0 = 0; w0 < nh; w0 += 4) {
+        if (w0 > 0) load_bf(w0);
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < 4; ++u) {
+          const int w = w0 + u;
+          if (w >= nh) break;
+          const int h = split + w * R;
+          float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < R && w0 + u < nh)
-            v[u][j] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(Osm, j) + (split + (w0 + u) * R) * kD +
-                                                       dim);
+          for (int j = 0; j < 16; ++j)
+            if (j < R) {
+              const float wj = wgt[w * 16 + j];
+              o0 = fmaf(wj, __uint_as_float(vb[u][j] << 16), o0);
+              o1 = fmaf(wj, __uint_as_float(vb[u][j] & 0xFFFF0000u), o1);
+            }
+          const float inv = wgt[kH * 16 + w * 2 + 1];
+          const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
+          *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0 * inv, o1 * inv);
+        }
+      }
+    } else {
+      // fp32 partials: two heads per round, every peer's loads of both in
+      // flight before the sums
+      for (int w0 = 0; w0 < nh; w0 += 2) {
+        float2 v[2][16];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int w = w0 + u;
-        if (w >= nh) break;
-        const int h = split + w * R;
-        float o0 = 0.f, o1 = 0.f;
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < R) {
-            const float wj = wgt[w * 16 + j];
-            o0 = fmaf(wj, v[u][j].x, o0);
-            o1 = fmaf(wj, v[u][j].y, o1);
-          }
-        const float inv = wgt[kH * 16 + w * 2 + 1];
-        o0 *= inv;
-        o1 *= inv;
-        const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
-        if (a.out_dtype == kF32) {
-          *reinterpret_cast<float2*>(static_cast<float*>(a.out) + off) = make_float2(o0, o1);
-        } else {
-          *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0, o1);
+          for (int j = 0; j < 16; ++j)
+            if (j < R && w0 + u < nh)
+              v[u][j] = *reinterpret_cast<const float2*>(cluster.map_shared_rank(Osm, j) + (split + (w0 + u) * R) * kD +
+                                                         dim);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int w = w0 + u;
+          if (w >= nh) break;
+          const int h = split + w * R;
+          float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < R) {
+              const float wj = wgt[w * 16 + j];
+              o0 = fmaf(wj, v[u][j].x, o0);
+              o1 = fmaf(wj, v[u][j].y, o1);
+            }
+          const float inv = wgt[kH * 16 + w * 2 + 1];
+          const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
+          *reinterpret_cast<float2*>(static_cast<float*>(a.out) + off) = make_float2(o0 * inv, o1 * inv);
         }
       }
     }
