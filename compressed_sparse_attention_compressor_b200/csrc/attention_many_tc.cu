@@ -102,41 +102,92 @@ __device__ __forceinline__ uint8_t* chunk_addr(uint8_t* tile, int r, int c8) {
   return tile + (c8 >> 3) * (kTK * 128) + sw128_offset(r, c8 & 7);
 }
 
-// All 128 threads of warps 0-3: the tile's window rows (entry codes <= -2)
-// take their value rows (compressed entries are their own values), by
-// asynchronous 16-byte copies, all in flight at once.
-__device__ void gather_window_values(uint8_t* tile, const int32_t* ent, const Src& a) {
-  const int t = static_cast<int>(threadIdx.x);  // 0..127
-  for (int task = t; task < kTK * 64; task += 128) {
+// All threads: the tile's window rows (entry codes <= -2) take their value
+// rows (compressed entries are their own values), by asynchronous 16-byte
+// copies; the caller waits for them (cp_async_wait_all) before P V.
+__device__ void issue_window_values(uint8_t* tile, const int32_t* ent, const Src& a) {
+  for (int task = static_cast<int>(threadIdx.x); task < kTK * 64; task += kNT) {
     const int32_t e = ent[task >> 6];
     if (e <= -2)
       cp_async16(chunk_addr(tile, task >> 6, task & 63),
                  reinterpret_cast<const uint4*>(a.swa_v + (a.sw_row0 + (-2 - e)) * kD) + (task & 63));
   }
-  cp_async_wait_all();
 }
 
-// All threads: the tile's key rows.  bf16 rows (compressed bf16 entries,
-// window keys) by asynchronous 16-byte copies, all issued before any wait;
-// FP8 / MXFP4 compressed rows through registers (dequantised to bf16);
-// rows without a key (-1) zeroed.
+// Named barriers 2 .. 9: column block b (dims 64 b .. 64 b + 63) of the key
+// tile is in shared memory.  Barrier 1 is free; 0 is __syncthreads.
+constexpr uint32_t kBarBlock = 2;
+
+// All threads: the tile's key rows, column block by column block.  bf16
+// rows (compressed bf16 entries, window keys) by asynchronous 16-byte
+// copies, one commit group per block: thread t copies chunks q = i kNT + t
+// (i < 4) of every block, row q / 8, chunk q % 8 of the block; FP8 / MXFP4
+// compressed rows go through registers (dequantised to bf16) before any
+// block is released; rows without a key (-1) are zeroed.  A thread releases
+// block b once its own copies of it have landed (and are fenced for the
+// tensor cores): warp 1, which issues the S MMAs, waits for the block's
+// barrier instead and issues the block's four MMAs as soon as every thread
+// has released it, so the MMAs follow the copies block by block.
 template <int FMT>
-__device__ void gather_keys(uint8_t* tile, const int32_t* ent, const Src& a) {
-  if constexpr (FMT != kKvBF16) gather_rows<FMT>(tile, ent, a, 0);  // quantised rows (and the rest)
-  else {
-    for (int task = static_cast<int>(threadIdx.x); task < kTK * 64; task += kNT) {
-      const int r = task >> 6, c8 = task & 63;
-      const int32_t e = ent[r];
-      uint8_t* dst = chunk_addr(tile, r, c8);
-      if (e >= 0)
-        cp_async16(dst, reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + (a.kv_row0 + e) * kD) + c8);
-      else if (e <= -2)
-        cp_async16(dst, reinterpret_cast<const uint4*>(a.swa_k + (a.sw_row0 + (-2 - e)) * kD) + c8);
-      else
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+__device__ bool gather_keys_issue_s(uint8_t* tile, const int32_t* ent, const Src& a, uint32_t dS, uint32_t qb,
+                                    uint64_t* qbar, bool first) {
+  const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
+  if constexpr (FMT != kKvBF16) {
+    gather_rows<FMT>(tile, ent, a, 0);  // quantised rows (and the rest), through registers
+  } else {
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = i * kNT + tid;
+        const int r = q >> 3, c8 = b * 8 + (q & 7);
+        const int32_t e = ent[r];
+        uint8_t* dst = chunk_addr(tile, r, c8);
+        if (e >= 0)
+          cp_async16(dst, reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.kv) + (a.kv_row0 + e) * kD) + c8);
+        else if (e <= -2)
+          cp_async16(dst, reinterpret_cast<const uint4*>(a.swa_k + (a.sw_row0 + (-2 - e)) * kD) + c8);
+        else
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+      cp_async_commit();
     }
-    cp_async_wait_all();
   }
+  bool ok = true;
+  const uint32_t kb = smem_u32(tile);
+  auto release = [&](int b) {
+    fence_proxy_async_smem();
+    if (warp != 1) {
+      named_barrier_arrive(kBarBlock + b, kNT);
+      return;
+    }
+    named_barrier(kBarBlock + b, kNT);
+    if (lane == 0) {
+      if (b == 0 && first) ok = mbar_wait(qbar, 0, kWaitLimit);
+      tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(dS, desc_k_sw128(kb + b * kTK * 128 + kk * 32), desc_k_sw128(qb + b * kH * 128 + kk * 32), kIdescS,
+                  (b | kk) ? 1u : 0u);
+      }
+    }
+    __syncwarp();
+  };
+  if constexpr (FMT != kKvBF16) {
+#pragma unroll
+    for (int b = 0; b < 8; ++b) release(b);
+  } else {
+    cp_async_wait_group<7>(); release(0);
+    cp_async_wait_group<6>(); release(1);
+    cp_async_wait_group<5>(); release(2);
+    cp_async_wait_group<4>(); release(3);
+    cp_async_wait_group<3>(); release(4);
+    cp_async_wait_group<2>(); release(5);
+    cp_async_wait_group<1>(); release(6);
+    cp_async_wait_group<0>(); release(7);
+  }
+  return ok;
 }
 
 template <int FMT>
@@ -172,6 +223,19 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   const int n_win = (a.window > 0 && t >= p_lo) ? static_cast<int>(t - p_lo + 1) : 0;
   const int total = live ? n_sel + n_win : 0;
   const int ntiles = (total + kTK - 1) / kTK;
+  // entry code of key-list position x: selected entry (>= 0), window slot (-2 - slot), nothing (-1)
+  auto code = [&](int x) -> int32_t {
+    int32_t e = -1;
+    if (x < total) {
+      if (x < n_sel) {
+        const int32_t jj = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
+        e = (jj >= 0 && jj < nv) ? jj : -1;
+      } else {
+        e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
+      }
+    }
+    return e;
+  };
 
   if (tid == 0) {
     prefetch_tensormap(&qmap);
@@ -191,6 +255,7 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.f;
   }
+  if (tid < kTK) ent[tid] = code(tid);
   if (warp == 1) tmem_alloc(tmem_slot, kTmemColsM);
   if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + mLut));
   tc_fence_before();
@@ -207,50 +272,21 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   src.kv_row0 = live ? static_cast<int64_t>(r) * a.cap : 0;
   src.sw_row0 = live ? static_cast<int64_t>(r) * a.swa_cap : 0;
   src.tau = a.tau;
-  const int sub = warp & 3;
+  // softmax split: warp w reads TMEM lanes (keys) 32 (w % 4) .. + 31 and
+  // takes heads hb .. hb + 31 of them
+  const int q4 = warp & 3, hb = (warp >> 2) * 32;
+  const int row = q4 * 32 + lane;  // key of the tile this thread reads
+  const uint32_t taS = dS + (static_cast<uint32_t>(q4 * 32) << 16) + hb;
 
   for (int j = 0; j < ntiles; ++j) {
-    // entry codes of tile j: selected entry (>= 0), window slot (-2 - slot), nothing (-1)
-    if (tid < kTK) {
-      const int x = j * kTK + tid;
-      int32_t e = -1;
-      if (x < total) {
-        if (x < n_sel) {
-          const int32_t jj = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
-          e = (jj >= 0 && jj < nv) ? jj : -1;
-        } else {
-          e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
-        }
-      }
-      ent[tid] = e;
+    // the next tile's entry codes: loads issued now, stored while P V runs
+    const int32_t e_next = (tid < kTK && j + 1 < ntiles) ? code((j + 1) * kTK + tid) : -1;
+    // ---- gather, and S^T = K Q^T block by block behind it ----
+    if (!gather_keys_issue_s<FMT>(Kt, ent, src, dS, smem_u32(smem + mQ), qbar, j == 0)) {
+      atomicOr(&g_attn_many_error, 1u);
+      flags[1] = 1;
     }
-    if (tid == 128) flags[0] = 0;
-    __syncthreads();
-    gather_keys<FMT>(Kt, ent, src);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (flags[1]) break;
-    // ---- S^T = K Q^T ----
-    if (tid == 32) {
-      bool ok = true;
-      if (j == 0) ok = mbar_wait(qbar, 0, kWaitLimit);
-      if (!ok) {
-        atomicOr(&g_attn_many_error, 1u);
-        flags[1] = 1;
-      } else {
-        tc_fence_after();
-        const uint32_t kb = smem_u32(Kt), qb = smem_u32(smem + mQ);
-#pragma unroll
-        for (int blk = 0; blk < 8; ++blk)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16(dS, desc_k_sw128(kb + blk * kTK * 128 + kk * 32), desc_k_sw128(qb + blk * kH * 128 + kk * 32),
-                    kIdescS, (blk | kk) ? 1u : 0u);
-        mma_commit(sbar);
-      }
-    }
+    if (tid == 32) mma_commit(sbar);
     if (tid == 0 && !mbar_wait(sbar, j & 1, kWaitLimit)) {
       atomicOr(&g_attn_many_error, 1u);
       flags[1] = 1;
@@ -259,33 +295,36 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     tc_fence_after();
     if (flags[1]) break;
     const int x0 = j * kTK;
-    const bool any_window = n_win > 0 && x0 + kTK > n_sel && x0 < total;
-    if (warp < 4) {
-      if (any_window) gather_window_values(Kt, ent, src);
-    } else {
-      const int row = sub * 32 + lane;  // key of the tile this thread reads
-      const bool row_ok = ent[row] != -1;
-      const uint32_t taS = dS + (static_cast<uint32_t>(sub * 32) << 16);
-      // this thread's logits of heads hh .. hh + 31 (its key), from TMEM
-      auto load_logits = [&](int hh, float (&s)[32]) {
-        uint32_t v[32];
-        tmem_ld32(taS + hh, v);
-        tmem_wait_ld();
+    // window rows: values replace keys in the tile (S has read it); the
+    // copies fly during the softmax
+    if (n_win > 0 && x0 + kTK > n_sel && x0 < total) issue_window_values(Kt, ent, src);
+
+    // ---- softmax over the tile: P = exp(S - m), m moving lazily ----
+    const bool row_ok = ent[row] != -1;
+    float s[32];
+    auto load_logits = [&]() {
+      uint32_t v[32];
+      tmem_ld32(taS, v);
+      tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s[h] = row_ok ? __uint_as_float(v[h]) * a.tau : -INFINITY;
-      };
-      // the tile's maximum of every head: per warp (lane l: head hh + l),
-      // then over the 4 warps
-#pragma unroll 1
-      for (int hh = 0; hh < kH; hh += 32) {
-        float s[32];
-        load_logits(hh, s);
-        warp_reduce32(s, MaxOp());
-        red[sub * kH + hh + lane] = s[0];
-      }
-      named_barrier(1, 128);
-      if (tid < 128 + kH) {
-        const int h = tid - 128;
+      for (int h = 0; h < 32; ++h) s[h] = row_ok ? __uint_as_float(v[h]) * a.tau : -INFINITY;
+    };
+    load_logits();
+    // m stays unless a logit passes m + kLazy (or a head has no mass yet)
+    bool pass = false;
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      const float mu = m_run[hb + h];
+      pass = pass || (s[h] != -INFINITY && (mu == -INFINITY || s[h] > mu + kLazy));
+    }
+    const bool moved = __syncthreads_or(pass) != 0;
+    if (moved) {
+      // the tile's maximum of every head: per warp (lane l: head hb + l), then over the 4 key quarters
+      warp_reduce32(s, MaxOp());
+      red[q4 * kH + hb + lane] = s[0];
+      __syncthreads();
+      if (tid < kH) {
+        const int h = tid;
         const float mt = fmaxf(fmaxf(red[h], red[kH + h]), fmaxf(red[2 * kH + h], red[3 * kH + h]));
         const float mo = m_run[h];
         float f = 1.f, mu = mo;
@@ -301,48 +340,47 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
         m_run[h] = mu;
         fac[h] = f;
       }
-      named_barrier(1, 128);
-      // P = exp(S - m) as bf16 into P^T [head][key]; the sums in fp32
+      __syncthreads();
+      load_logits();
+    }
+    // P^T [head][key] as bf16; the sums in fp32
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      const float mu = m_run[hb + h];
+      const float p = (s[h] == -INFINITY || mu == -INFINITY) ? 0.f : __expf(s[h] - mu);
+      s[h] = p;
+      *reinterpret_cast<uint16_t*>(Pt + (row >> 6) * (kH * 128) + sw128_offset(hb + h, (row & 63) >> 3) +
+                                   (row & 7) * 2) = f32_to_bf16_bits(p);
+    }
+    warp_reduce32(s, SumOp());
+    red[q4 * kH + hb + lane] = s[0];
+    __syncthreads();
+    if (tid < kH) {
+      const int h = tid;
+      const float f = moved ? fac[h] : 1.f;
+      l_run[h] = l_run[h] * f + ((red[h] + red[kH + h]) + (red[2 * kH + h] + red[3 * kH + h]));
+    }
+    // a head whose m moved: its column of O (all 512 dims) by the factor;
+    // warp w rescales dims 32 (w % 4) .. + 31 of the blocks 2 (w / 4), + 1
+    if (moved && j > 0 && flags[0]) {
 #pragma unroll 1
-      for (int hh = 0; hh < kH; hh += 32) {
-        float s[32];
-        load_logits(hh, s);
+      for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
+        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(q4 * 32) << 16);
+        uint32_t v0[32], v1[32];
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
-          const float mu = m_run[hh + h];
-          const float p = (s[h] == -INFINITY || mu == -INFINITY) ? 0.f : __expf(s[h] - mu);
-          s[h] = p;
-          *reinterpret_cast<uint16_t*>(Pt + (row >> 6) * (kH * 128) + sw128_offset(hh + h, (row & 63) >> 3) +
-                                       (row & 7) * 2) = f32_to_bf16_bits(p);
+          v0[h] = __float_as_uint(__uint_as_float(v0[h]) * fac[h]);
+          v1[h] = __float_as_uint(__uint_as_float(v1[h]) * fac[32 + h]);
         }
-        warp_reduce32(s, SumOp());
-        red[sub * kH + hh + lane] = s[0];
+        tmem_st32(ta, v0);
+        tmem_st32(ta + 32, v1);
       }
-      named_barrier(1, 128);
-      if (tid < 128 + kH) {
-        const int h = tid - 128;
-        l_run[h] = l_run[h] * fac[h] + ((red[h] + red[kH + h]) + (red[2 * kH + h] + red[3 * kH + h]));
-      }
-      // a head whose m moved: its column of O (all 512 dims) by the factor
-      if (j > 0 && flags[0]) {
-#pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
-          const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
-          uint32_t v0[32], v1[32];
-          tmem_ld32(ta, v0);
-          tmem_ld32(ta + 32, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            v0[h] = __float_as_uint(__uint_as_float(v0[h]) * fac[h]);
-            v1[h] = __float_as_uint(__uint_as_float(v1[h]) * fac[32 + h]);
-          }
-          tmem_st32(ta, v0);
-          tmem_st32(ta + 32, v1);
-        }
-        tmem_wait_st();
-      }
+      tmem_wait_st();
     }
+    cp_async_wait_all();  // window values
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -358,6 +396,8 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
                   desc_k_sw128(pb + (kk >> 2) * kH * 128 + (kk & 3) * 32), kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(obar);
     }
+    if (tid < kTK) ent[tid] = e_next;  // the codes of this tile were last read before the barrier
+    if (tid == 128) flags[0] = 0;
     if (tid == 0 && !mbar_wait(obar, j & 1, kWaitLimit)) {
       atomicOr(&g_attn_many_error, 1u);
       flags[1] = 1;
@@ -384,15 +424,16 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     if (a.lse) a.lse[static_cast<int64_t>(qi) * kH + h] = (M == -INFINITY) ? -INFINITY : M + __logf(L);
   }
   __syncthreads();
-  if (warp >= 4) {
+  {
+    // warp w writes dims 32 (w % 4) .. + 31 of the blocks 2 (w / 4), + 1
     const int oeb = a.out_dtype == kF32 ? 4 : 2;
     char* obase = static_cast<char*>(a.out) + static_cast<int64_t>(qi) * kH * kD * oeb;
 #pragma unroll 1
-    for (int mt = 0; mt < 4; ++mt) {
-      const int dim = mt * 128 + sub * 32 + lane;
+    for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
+      const int dim = mt * 128 + q4 * 32 + lane;
       uint32_t v0[32], v1[32];
       if (ntiles > 0) {
-        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(sub * 32) << 16);
+        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(q4 * 32) << 16);
         tmem_ld32(ta, v0);
         tmem_ld32(ta + 32, v1);
         tmem_wait_ld();

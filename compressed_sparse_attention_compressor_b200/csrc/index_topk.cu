@@ -159,27 +159,11 @@ struct Row4 {
   }
 };
 
-__global__ void __launch_bounds__(kTopkThreads)
-topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
-                int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int nv_div, int ordered) {
-  __shared__ TopkShared sh;
-  const int row = blockIdx.x;
-  // valid columns: ceil(n_valid / nv_div), or max_n without n_valid
-  const int64_t nv = n_valid ? (static_cast<int64_t>(n_valid[row]) + nv_div - 1) / nv_div : max_n;
-  const int64_t n = min(max(nv, int64_t(0)), max_n);
-  const float* s = scores + static_cast<int64_t>(row) * ld;
-  int32_t* oi = out_idx + static_cast<int64_t>(row) * k;
-  float* os = out_score ? out_score + static_cast<int64_t>(row) * k : nullptr;
+// The whole row (any distribution): a min / max pass, then the radix select
+// of the k-th key over the keys' own range, then the index-ordered pass.
+__device__ void topk_row_full(TopkShared& sh, const float* s, int64_t n, int k, int32_t* oi, float* os,
+                              int ordered) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  if (n <= k) {
-    for (int64_t j = tid; j < k; j += kTopkThreads) {
-      oi[j] = j < n ? static_cast<int32_t>(j) : -1;
-      if (os) os[j] = j < n ? s[j] : -INFINITY;
-    }
-    return;
-  }
-
   const Row4 rs4{s, n, (reinterpret_cast<uintptr_t>(s) & 15) == 0};
   // radix select of the k-th largest key over the keys' own range: the
   // range [lo, lo + span) is cut into <= 2048 bins of 2^shift keys and
@@ -318,6 +302,182 @@ topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __r
   }
 }
 
+// Candidate form of the same selection.  A strided sample of 2,048 scores
+// gives a key t that at least k entries of the row reach with high
+// probability (the sample's r-th largest, r a few standard deviations above
+// the k / n share of the sample, rounded down to a bin of 2^10 keys); one
+// pass over the row copies every entry with key >= t into shared memory, in
+// index order per warp segment.  When at least k entries reached t, the k
+// best of the row are all among them (ties at the k-th key included), and
+// the radix select and the index-ordered pass run over the candidates.
+// Returns false (uniformly over the CTA) when the candidates do not fit in
+// kCandR slots per warp or fewer than k entries reached t: the caller then
+// runs topk_row_full, so the result never depends on the sample.
+constexpr int kCandR = 256;      // candidate slots per warp
+constexpr int kSamples = 2 * kTopkThreads;
+constexpr int kTopkDynSmem = 2 * kTopkWarps * kCandR * 4;  // keys, then indices
+
+__device__ bool topk_row_candidates(TopkShared& sh, uint32_t* cand, const float* s, int64_t n, int k, int32_t* oi,
+                                    float* os, int ordered) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t below = (1u << lane) - 1u;  // lanes under this one
+  // ---- t from the sample (every entry is a candidate when the row fits) ----
+  uint32_t t = 0;
+  if (n > static_cast<int64_t>(kTopkWarps) * kCandR) {
+    const uint32_t s0 = score_key(__ldg(s + static_cast<int64_t>(tid) * n / kSamples));
+    const uint32_t s1 = score_key(__ldg(s + static_cast<int64_t>(tid + kTopkThreads) * n / kSamples));
+    const float mu = static_cast<float>(k) * kSamples / static_cast<float>(n);
+    uint32_t need = static_cast<uint32_t>(min(static_cast<float>(kSamples), ceilf(mu + 4.f * sqrtf(mu) + 4.f)));
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 21 : 10;  // bits 21..31, then 10..20
+      for (int i = tid; i < 2048; i += kTopkThreads) sh.hist[i] = 0;
+      __syncthreads();
+      if (pass == 0 || (s0 >> 21) == (t >> 21)) atomicAdd(&sh.hist[(s0 >> shift) & 2047u], 1u);
+      if (pass == 0 || (s1 >> 21) == (t >> 21)) atomicAdd(&sh.hist[(s1 >> shift) & 2047u], 1u);
+      __syncthreads();
+      if (warp == 0) find_bin(sh, 2048, need);
+      __syncthreads();
+      t |= sh.sel_bin << shift;
+      need -= sh.above;
+    }
+  }
+  // ---- candidates: key >= t, per warp segment in index order ----
+  uint32_t* ckey = cand + warp * kCandR;
+  uint32_t* cidx = cand + kTopkWarps * kCandR + warp * kCandR;
+  const Row4 rs4{s, n, (reinterpret_cast<uintptr_t>(s) & 15) == 0};
+  const int64_t segw = ((n + kTopkWarps - 1) / kTopkWarps + 127) & ~int64_t(127);
+  const int64_t a0 = min(n, warp * segw), a1 = min(n, a0 + segw);
+  uint32_t cnt = 0;  // candidates of this warp so far (warp-uniform)
+  for (int64_t j1 = a0; j1 < a1; j1 += kU * 128) {
+    float v[kU][4];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) rs4.load(j1 + u * 128 + 4 * lane, v[u]);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t j0 = j1 + u * 128 + 4 * lane;
+      if (j1 + u * 128 >= a1) break;
+      uint32_t key[4], b[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        key[c] = score_key(v[u][c]);
+        b[c] = __ballot_sync(0xFFFFFFFFu, j0 + c < a1 && key[c] >= t);
+      }
+      const uint32_t tot = __popc(b[0]) + __popc(b[1]) + __popc(b[2]) + __popc(b[3]);
+      if (tot == 0) continue;
+      uint32_t pos = cnt + __popc(b[0] & below) + __popc(b[1] & below) + __popc(b[2] & below) + __popc(b[3] & below);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if ((b[c] >> lane) & 1u) {
+          if (pos < kCandR) {
+            ckey[pos] = key[c];
+            cidx[pos] = static_cast<uint32_t>(j0 + c);
+          }
+          ++pos;
+        }
+      cnt += tot;
+    }
+  }
+  if (lane == 0) sh.warp_gt[warp] = cnt;
+  __syncthreads();
+  uint32_t total = 0;
+  bool fits = true;
+  for (int w2 = 0; w2 < kTopkWarps; ++w2) {
+    total += sh.warp_gt[w2];
+    fits = fits && sh.warp_gt[w2] <= static_cast<uint32_t>(kCandR);
+  }
+  __syncthreads();
+  if (!fits || total < static_cast<uint32_t>(k)) return false;
+
+  // ---- radix select of the k-th key among the candidates (range [t, max]) ----
+  uint32_t kmax = 0u;
+  for (uint32_t i = lane; i < cnt; i += 32) kmax = max(kmax, ckey[i]);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+  if (lane == 0) sh.warp_eq[warp] = kmax;
+  __syncthreads();
+  uint32_t hi = 0u;
+  for (int w2 = 0; w2 < kTopkWarps; ++w2) hi = max(hi, sh.warp_eq[w2]);
+  uint32_t lo = t;
+  uint64_t span = static_cast<uint64_t>(hi - lo) + 1;
+  uint32_t need = static_cast<uint32_t>(k);
+  int shift = max(0, 64 - __clzll(static_cast<long long>(span - 1)) - 11);
+  for (;;) {
+    for (int i = tid; i < 2048; i += kTopkThreads) sh.hist[i] = 0;
+    __syncthreads();
+    for (uint32_t i = lane; i < cnt; i += 32) {
+      const uint32_t d = ckey[i] - lo;
+      if (static_cast<uint64_t>(d) < span) atomicAdd(&sh.hist[d >> shift], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) find_bin(sh, 2048, need);
+    __syncthreads();
+    const uint32_t b = sh.sel_bin;
+    need -= sh.above;
+    lo += b << shift;
+    span = min(span - (static_cast<uint64_t>(b) << shift), static_cast<uint64_t>(1) << shift);
+    __syncthreads();
+    if (shift == 0) break;
+    shift = max(0, shift - 11);
+  }
+  const uint32_t T = lo;          // exact key of the k-th largest score
+  const uint32_t take_eq = need;  // entries equal to T that are kept
+  const uint32_t n_gt = static_cast<uint32_t>(k) - take_eq;
+
+  // ---- index-ordered output over the candidates ----
+  uint32_t cg = 0, ce = 0;
+  for (uint32_t i = lane; i < cnt; i += 32) {
+    const uint32_t key = ckey[i];
+    cg += key > T;
+    ce += key == T;
+  }
+  cg = __reduce_add_sync(0xFFFFFFFFu, cg);
+  ce = __reduce_add_sync(0xFFFFFFFFu, ce);
+  if (lane == 0) { sh.warp_gt[warp] = cg; sh.warp_eq[warp] = ce; }
+  __syncthreads();
+  uint32_t og = 0, oe = 0;  // entries above / at T before the current step
+  for (int w2 = 0; w2 < warp; ++w2) { og += sh.warp_gt[w2]; oe += sh.warp_eq[w2]; }
+  for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    const uint32_t key = i < cnt ? ckey[i] : 0u;
+    const bool pg = i < cnt && key > T, pe = i < cnt && key == T;
+    const uint32_t bg = __ballot_sync(0xFFFFFFFFu, pg), be = __ballot_sync(0xFFFFFFFFu, pe);
+    const uint32_t g = og + __popc(bg & below), e = oe + __popc(be & below);
+    if (pg || (pe && e < take_eq)) {
+      // ordered: the kept entries before this one are g above T and min(e, take_eq) at T
+      const uint32_t p = pg ? (ordered ? g + min(e, take_eq) : g) : (ordered ? g + e : n_gt + e);
+      const uint32_t j = cidx[i];
+      oi[p] = static_cast<int32_t>(j);
+      if (os) os[p] = __ldg(s + j);
+    }
+    og += __popc(bg);
+    oe += __popc(be);
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+topk_row_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_valid, int64_t max_n,
+                int k, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int nv_div, int ordered) {
+  __shared__ TopkShared sh;
+  extern __shared__ uint32_t cand[];
+  const int row = blockIdx.x;
+  // valid columns: ceil(n_valid / nv_div), or max_n without n_valid
+  const int64_t nv = n_valid ? (static_cast<int64_t>(n_valid[row]) + nv_div - 1) / nv_div : max_n;
+  const int64_t n = min(max(nv, int64_t(0)), max_n);
+  const float* s = scores + static_cast<int64_t>(row) * ld;
+  int32_t* oi = out_idx + static_cast<int64_t>(row) * k;
+  float* os = out_score ? out_score + static_cast<int64_t>(row) * k : nullptr;
+
+  if (n <= k) {
+    for (int64_t j = threadIdx.x; j < k; j += kTopkThreads) {
+      oi[j] = j < n ? static_cast<int32_t>(j) : -1;
+      if (os) os[j] = j < n ? s[j] : -INFINITY;
+    }
+    return;
+  }
+  if (!topk_row_candidates(sh, cand, s, n, k, oi, os, ordered)) topk_row_full(sh, s, n, k, oi, os, ordered);
+}
+
 template <int H, int DI>
 csa_status_t launch_score_t(const csa_params_t* p, int nq, const csa_tensor_t* q_idx, const float* w,
                             const csa_tensor_t* k_idx, int batch, int64_t cap, const int32_t* q_req,
@@ -355,9 +515,16 @@ csa_status_t launch_index_score(const csa_params_t* p, int nq, const csa_tensor_
 csa_status_t launch_topk(const float* scores, int n_rows, int64_t ld, const int32_t* n_valid, int64_t max_n, int k,
                          int32_t* out_idx, float* out_score, cudaStream_t stream, int nv_div, int ordered) {
   if (n_rows == 0) return CSA_OK;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(topk_row_kernel),
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kTopkDynSmem);
+    if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
   prof_begin(stream);
-  topk_row_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score, nv_div,
-                                                       ordered);
+  topk_row_kernel<<<n_rows, kTopkThreads, kTopkDynSmem, stream>>>(scores, ld, n_valid, max_n, k, out_idx, out_score,
+                                                                  nv_div, ordered);
   return check_launch("topk_row_kernel", stream);
 }
 

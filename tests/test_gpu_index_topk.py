@@ -54,6 +54,54 @@ def test_topk_all_equal_scores_takes_lowest_indices(n, cuda_lib):
         assert np.array_equal(np.sort(out_idx[r].cpu().numpy()), np.arange(k))
 
 
+
+def _shaped_rows(n):
+    """Score rows whose shape decides which form of the row top-k runs:
+    typical rows are selected among sampled candidates, while sorted rows
+    (all winners in one warp's segment), rows whose sampled positions hold
+    the largest scores (too few candidates), rows of few distinct values
+    (many ties at the k-th score) and mostly -inf rows stress the sample's
+    threshold and the fallback over the whole row."""
+    g = Wk.rng(4100 + n, "shaped")
+    rows = {
+        "normal": g.standard_normal(n, dtype=np.float32),
+        "ascending": np.arange(n, dtype=np.float32) / n,
+        "descending": (n - np.arange(n, dtype=np.float32)) / n,
+        "few_values": np.round(g.standard_normal(n)).astype(np.float32),
+        "mostly_neg_inf": np.where(g.random(n) < 0.9, -np.inf, g.standard_normal(n)).astype(np.float32),
+    }
+    planted = (g.standard_normal(n) * 0.01).astype(np.float32)
+    planted[np.arange(2048) * n // 2048] = 5 + g.random(2048, dtype=np.float32)
+    rows["sample_positions_largest"] = planted
+    return rows
+
+
+@pytest.mark.parametrize("k", [512, 2048])
+@pytest.mark.parametrize("n", [8192, 8193, 33000, 131072])
+def test_topk_row_shapes_are_bit_exact(n, k, cuda_lib):
+    """One CTA per row (no workspace): every row shape gives the oracle's
+    selection, whichever form of the selection it takes."""
+    shapes = _shaped_rows(n)
+    names = list(shapes)
+    buf = np.stack([shapes[x] for x in names])
+    rows = buf.shape[0]
+    scores = torch.from_numpy(buf).cuda()
+    out_idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
+    out_score = torch.empty((rows, k), dtype=torch.float32, device="cuda")
+    csa.csa_topk(scores, rows, n, i32([n] * rows), k, out_idx, out_score, None)
+    torch.cuda.synchronize()
+    gi, gs = out_idx.cpu().numpy(), out_score.cpu().numpy()
+    for r, name in enumerate(names):
+        ref = O.topk(buf[r].astype(np.float64), k)
+        assert np.array_equal(np.sort(gi[r]), np.sort(ref)), name
+        assert np.array_equal(gs[r], buf[r, gi[r]]), name
+        # entries above the k-th score come first, each group in index order
+        kth = np.float32(np.sort(buf[r].astype(np.float64))[::-1][k - 1])
+        above = gs[r] > kth
+        n_above = int(above.sum())
+        assert above[:n_above].all(), name
+        assert np.all(np.diff(gi[r][:n_above]) > 0) and np.all(np.diff(gi[r][n_above:]) > 0), name
+
 IDX_CASES = {
     # name: (workload, n_queries, batch, cap)
     "tiny_f32": (Wk.WORKLOADS["tiny"], 3, 3, 1024 + 37),
