@@ -38,14 +38,15 @@ using namespace attn;
 
 constexpr uint32_t kTmemColsM = 512;  // S^T 64 columns + O^T 256 columns
 constexpr float kLazy = 8.f;          // nats a tile maximum may exceed m before m moves
+constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory, from a 1024-byte aligned base
 constexpr int mK = 0;                       // 8 x 16 KB key / value tile
 constexpr int mQ = mK + 8 * kTK * 128;      // 8 x 8 KB query
 constexpr int mP = mQ + 8 * kH * 128;       // 2 x 8 KB P^T (bf16, K-major over keys)
 constexpr int mRed = mP + 2 * kH * 128;     // [4][64] per-warp partial maxima / sums
-constexpr int mStat = mRed + 4 * kH * 4;    // m[64], l[64], rescale factor[64], final scale[64]
-constexpr int mEnt = mStat + 4 * kH * 4;    // [128] entry codes of the tile
+constexpr int mStat = mRed + 4 * kH * 4;    // m, l, rescale factor, final scale, m + kLazy, m log2 e: [64] each
+constexpr int mEnt = mStat + 6 * kH * 4;    // [128] entry codes of the tile
 constexpr int mBars = mEnt + kTK * 4;
 constexpr int mMisc = mBars + 64;
 constexpr int mLut = mMisc + 64;            // MXFP4 code-byte table, 256 x bf16x2
@@ -63,6 +64,7 @@ struct AttnManyArgs {
   const int64_t* q_pos; const int64_t* swa_lo;
   float tau;
   const float* sink; void* out; int out_dtype; float* lse;
+  int out_bulk;  // out is 16-byte aligned: the block leaves by bulk stores
 };
 
 __device__ __forceinline__ uint8_t* align1024m(uint8_t* p) {
@@ -202,6 +204,8 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   float* l_run = m_run + kH;
   float* fac = l_run + kH;
   float* fin = fac + kH;
+  float* thr = fin + kH;  // m + kLazy (-inf while a head has no mass)
+  float* ml2 = thr + kH;  // m log2(e) (0 while a head has no mass)
   int32_t* ent = reinterpret_cast<int32_t*>(smem + mEnt);
   uint64_t* qbar = reinterpret_cast<uint64_t*>(smem + mBars);
   uint64_t* sbar = qbar + 1;
@@ -254,6 +258,8 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   if (tid < kH) {
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.f;
+    thr[tid] = -INFINITY;
+    ml2[tid] = 0.f;
   }
   if (tid < kTK) ent[tid] = code(tid);
   if (warp == 1) tmem_alloc(tmem_slot, kTmemColsM);
@@ -307,19 +313,23 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
       tmem_ld32(taS, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int h = 0; h < 32; ++h) s[h] = row_ok ? __uint_as_float(v[h]) * a.tau : -INFINITY;
+      for (int h = 0; h < 32; ++h) s[h] = __uint_as_float(v[h]) * a.tau;
     };
     load_logits();
     // m stays unless a logit passes m + kLazy (or a head has no mass yet)
     bool pass = false;
+    if (row_ok) {
 #pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      const float mu = m_run[hb + h];
-      pass = pass || (s[h] != -INFINITY && (mu == -INFINITY || s[h] > mu + kLazy));
+      for (int h = 0; h < 32; h += 4) {
+        const float4 t4 = *reinterpret_cast<const float4*>(thr + hb + h);
+        pass = pass || (s[h] > t4.x) || (s[h + 1] > t4.y) || (s[h + 2] > t4.z) || (s[h + 3] > t4.w);
+      }
     }
     const bool moved = __syncthreads_or(pass) != 0;
     if (moved) {
       // the tile's maximum of every head: per warp (lane l: head hb + l), then over the 4 key quarters
+#pragma unroll
+      for (int h = 0; h < 32; ++h) s[h] = row_ok ? s[h] : -INFINITY;
       warp_reduce32(s, MaxOp());
       red[q4 * kH + hb + lane] = s[0];
       __syncthreads();
@@ -339,18 +349,27 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
         }
         m_run[h] = mu;
         fac[h] = f;
+        thr[h] = mu == -INFINITY ? -INFINITY : mu + kLazy;
+        ml2[h] = mu == -INFINITY ? 0.f : mu * kLog2e;
       }
       __syncthreads();
       load_logits();
     }
-    // P^T [head][key] as bf16; the sums in fp32
+    // P^T [head][key] as bf16 (rows without a key: 0); the sums in fp32
+    {
+      uint8_t* prow = Pt + (row >> 6) * (kH * 128) + (row & 7) * 2;
+      const uint32_t ch = (row & 63) >> 3;
 #pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      const float mu = m_run[hb + h];
-      const float p = (s[h] == -INFINITY || mu == -INFINITY) ? 0.f : __expf(s[h] - mu);
-      s[h] = p;
-      *reinterpret_cast<uint16_t*>(Pt + (row >> 6) * (kH * 128) + sw128_offset(hb + h, (row & 63) >> 3) +
-                                   (row & 7) * 2) = f32_to_bf16_bits(p);
+      for (int h = 0; h < 32; h += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(ml2 + hb + h);
+        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = row_ok ? ex2_approx(fmaf(s[h + u], kLog2e, -mm[u])) : 0.f;
+          s[h + u] = p;
+          *reinterpret_cast<uint16_t*>(prow + sw128_offset(hb + h + u, ch)) = f32_to_bf16_bits(p);
+        }
+      }
     }
     warp_reduce32(s, SumOp());
     red[q4 * kH + hb + lane] = s[0];
@@ -425,9 +444,13 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   }
   __syncthreads();
   {
-    // warp w writes dims 32 (w % 4) .. + 31 of the blocks 2 (w / 4), + 1
-    const int oeb = a.out_dtype == kF32 ? 4 : 2;
-    char* obase = static_cast<char*>(a.out) + static_cast<int64_t>(qi) * kH * kD * oeb;
+    // O / L into shared memory as the output rows [head][dim] (the key tile
+    // is idle now: every MMA has completed), then one bulk store of the
+    // query's 64 x 512 block; warp w takes dims 32 (w % 4) .. + 31 of the
+    // blocks 2 (w / 4), + 1
+    const bool f32 = a.out_dtype == kF32;
+    const int oeb = f32 ? 4 : 2;
+    uint8_t* ost = Kt;  // 64 KB (bf16) or 128 KB (fp32)
 #pragma unroll 1
     for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
       const int dim = mt * 128 + q4 * 32 + lane;
@@ -441,9 +464,24 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
 #pragma unroll
       for (int h = 0; h < 64; ++h) {
         const float o = ntiles > 0 ? __uint_as_float(h < 32 ? v0[h] : v1[h - 32]) * fin[h] : 0.f;
-        if (a.out_dtype == kF32) reinterpret_cast<float*>(obase)[h * kD + dim] = o;
-        else reinterpret_cast<uint16_t*>(obase)[h * kD + dim] = f32_to_bf16_bits(o);
+        if (f32) reinterpret_cast<float*>(ost)[h * kD + dim] = o;
+        else reinterpret_cast<uint16_t*>(ost)[h * kD + dim] = f32_to_bf16_bits(o);
       }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    char* obase = static_cast<char*>(a.out) + static_cast<int64_t>(qi) * kH * kD * oeb;
+    if (a.out_bulk) {
+      if (tid == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(kH * kD * oeb);
+        for (uint32_t o = 0; o < bytes; o += 32768) bulk_store(obase + o, ost + o, 32768);
+        bulk_store_wait_read();
+      }
+    } else if (f32) {
+      for (int i = tid; i < kH * kD; i += kNT) reinterpret_cast<float*>(obase)[i] = reinterpret_cast<float*>(ost)[i];
+    } else {
+      for (int i = tid; i < kH * kD; i += kNT)
+        reinterpret_cast<uint16_t*>(obase)[i] = reinterpret_cast<uint16_t*>(ost)[i];
     }
   }
   // every MMA of this CTA and the query's copy have completed before TMEM
@@ -524,6 +562,7 @@ csa_status_t launch_attention_many_tc(const csa_params_t* p, int nq, const csa_t
   a.sink = sink;
   a.out = out->data;
   a.out_dtype = out->dtype;
+  a.out_bulk = (reinterpret_cast<uintptr_t>(out->data) & 15) == 0;
   a.lse = lse;
   if (kv->dtype == kMXFP4) return launch_many_fmt<kKvMX4>(qmap, a, nq, stream);
   if (kv->dtype == kFP8) return launch_many_fmt<kKvFP8>(qmap, a, nq, stream);

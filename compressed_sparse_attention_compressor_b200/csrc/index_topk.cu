@@ -108,37 +108,42 @@ struct TopkShared {
   uint32_t hist[2048];
   uint32_t warp_gt[kTopkWarps];
   uint32_t warp_eq[kTopkWarps];
+  uint32_t wsum[kTopkWarps];
   uint32_t sel_bin;
   uint32_t above;
 };
 
-// Within warp 0: finds the bin b of hist[0..nb) (scanned from the top) with
-// count_above(b) < need <= count_above(b) + hist[b].
-__device__ void find_bin(TopkShared& sh, int nb, uint32_t need) {
-  const int lane = threadIdx.x & 31;
-  const int per = nb / 32;
-  const int lo = lane * per;
-  uint32_t mine = 0;
-  for (int i = 0; i < per; ++i) mine += sh.hist[lo + i];
-  // suffix sum over lanes >= lane
-  uint32_t incl = mine;
+// All threads (two bins each): the bin b of hist[0..2048), scanned from the
+// top, with above(b) < need <= above(b) + hist[b], where above(b) counts the
+// entries of the bins over b; writes (b, above(b)) to sel_bin / above, read
+// after the caller's next barrier.  Needs 1 <= need <= the histogram total.
+__device__ void find_bin_all(TopkShared& sh, uint32_t need) {
+  static_assert(2 * kTopkThreads == 2048, "two bins per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint2 c = *reinterpret_cast<const uint2*>(sh.hist + 2 * tid);  // bins 2 tid, 2 tid + 1
+  const uint32_t v = c.x + c.y;
+  uint32_t incl = v;  // this lane's bins and those of the lanes above it
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
-    if (lane + o < 32) incl += v;
+    const uint32_t x = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += x;
   }
-  const uint32_t excl = incl - mine;
-  if (excl < need && need <= incl) {
-    uint32_t above = excl;
-    for (int i = per - 1; i >= 0; --i) {
-      const uint32_t c = sh.hist[lo + i];
-      if (above + c >= need) {
-        sh.sel_bin = lo + i;
-        sh.above = above;
-        break;
-      }
-      above += c;
-    }
+  if (lane == 0) sh.wsum[warp] = incl;
+  __syncthreads();
+  const uint32_t ws = sh.wsum[lane];  // lane l: the total of warp l
+  uint32_t wi = ws;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_down_sync(0xFFFFFFFFu, wi, o);
+    if (lane + o < 32) wi += x;
+  }
+  const uint32_t above = __shfl_sync(0xFFFFFFFFu, wi - ws, warp) + incl - v;  // entries over bin 2 tid + 1
+  if (above < need && need <= above + c.y) {
+    sh.sel_bin = 2 * tid + 1;
+    sh.above = above;
+  } else if (above + c.y < need && need <= above + v) {
+    sh.sel_bin = 2 * tid;
+    sh.above = above + c.y;
   }
 }
 
@@ -211,7 +216,7 @@ __device__ void topk_row_full(TopkShared& sh, const float* s, int64_t n, int k, 
         }
     }
     __syncthreads();
-    if (warp == 0) find_bin(sh, 2048, need);
+    find_bin_all(sh, need);
     __syncthreads();
     const uint32_t b = sh.sel_bin;
     need -= sh.above;
@@ -336,7 +341,7 @@ __device__ bool topk_row_candidates(TopkShared& sh, uint32_t* cand, const float*
       if (pass == 0 || (s0 >> 21) == (t >> 21)) atomicAdd(&sh.hist[(s0 >> shift) & 2047u], 1u);
       if (pass == 0 || (s1 >> 21) == (t >> 21)) atomicAdd(&sh.hist[(s1 >> shift) & 2047u], 1u);
       __syncthreads();
-      if (warp == 0) find_bin(sh, 2048, need);
+      find_bin_all(sh, need);
       __syncthreads();
       t |= sh.sel_bin << shift;
       need -= sh.above;
@@ -409,7 +414,7 @@ __device__ bool topk_row_candidates(TopkShared& sh, uint32_t* cand, const float*
       if (static_cast<uint64_t>(d) < span) atomicAdd(&sh.hist[d >> shift], 1u);
     }
     __syncthreads();
-    if (warp == 0) find_bin(sh, 2048, need);
+    find_bin_all(sh, need);
     __syncthreads();
     const uint32_t b = sh.sel_bin;
     need -= sh.above;
