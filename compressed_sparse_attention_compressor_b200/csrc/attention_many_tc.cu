@@ -227,16 +227,17 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   const int n_win = (a.window > 0 && t >= p_lo) ? static_cast<int>(t - p_lo + 1) : 0;
   const int total = live ? n_sel + n_win : 0;
   const int ntiles = (total + kTK - 1) / kTK;
-  // entry code of key-list position x: selected entry (>= 0), window slot (-2 - slot), nothing (-1)
-  auto code = [&](int x) -> int32_t {
+  // entry code of key-list position x: selected entry (>= 0), window slot
+  // (-2 - slot), nothing (-1); the selection's index is loaded apart
+  // (idx_at), so that its load can be issued well before the code is formed
+  auto idx_at = [&](int x) -> int32_t {
+    return (a.idx && x < total && x < n_sel) ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
+  };
+  auto code = [&](int x, int32_t jj) -> int32_t {
     int32_t e = -1;
     if (x < total) {
-      if (x < n_sel) {
-        const int32_t jj = a.idx ? a.idx[static_cast<int64_t>(qi) * a.topk + x] : x;
-        e = (jj >= 0 && jj < nv) ? jj : -1;
-      } else {
-        e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
-      }
+      if (x < n_sel) e = (jj >= 0 && jj < nv) ? jj : -1;
+      else e = -2 - static_cast<int32_t>((p_lo + (x - n_sel)) % a.swa_cap);
     }
     return e;
   };
@@ -261,7 +262,7 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     thr[tid] = -INFINITY;
     ml2[tid] = 0.f;
   }
-  if (tid < kTK) ent[tid] = code(tid);
+  if (tid < kTK) ent[tid] = code(tid, idx_at(tid));
   if (warp == 1) tmem_alloc(tmem_slot, kTmemColsM);
   if constexpr (FMT == kKvMX4) fill_mx4_lut(reinterpret_cast<uint32_t*>(smem + mLut));
   tc_fence_before();
@@ -285,8 +286,9 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
   const uint32_t taS = dS + (static_cast<uint32_t>(q4 * 32) << 16) + hb;
 
   for (int j = 0; j < ntiles; ++j) {
-    // the next tile's entry codes: loads issued now, stored while P V runs
-    const int32_t e_next = (tid < kTK && j + 1 < ntiles) ? code((j + 1) * kTK + tid) : -1;
+    // the next tile's entry codes: index loads issued now, codes stored while P V runs
+    const int x_next = (j + 1) * kTK + tid;
+    const int32_t jj_next = (tid < kTK && j + 1 < ntiles) ? idx_at(x_next) : 0;
     // ---- gather, and S^T = K Q^T block by block behind it ----
     if (!gather_keys_issue_s<FMT>(Kt, ent, src, dS, smem_u32(smem + mQ), qbar, j == 0)) {
       atomicOr(&g_attn_many_error, 1u);
@@ -415,7 +417,7 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
                   desc_k_sw128(pb + (kk >> 2) * kH * 128 + (kk & 3) * 32), kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(obar);
     }
-    if (tid < kTK) ent[tid] = e_next;  // the codes of this tile were last read before the barrier
+    if (tid < kTK) ent[tid] = j + 1 < ntiles ? code(x_next, jj_next) : -1;  // this tile's were last read before the barrier
     if (tid == 128) flags[0] = 0;
     if (tid == 0 && !mbar_wait(obar, j & 1, kWaitLimit)) {
       atomicOr(&g_attn_many_error, 1u);

@@ -254,59 +254,59 @@ __device__ bool request_barrier(uint32_t* ctr, uint32_t target, uint32_t limit, 
 }
 
 // Whole block: bin b of a shared-memory histogram of `nbins` bins (a power
-// of two, 128..kHistBins), scanned from the top, with
+// of two, 256..kHistBins), scanned from the top, with
 // above(b) < need <= above(b) + hist[b]; writes (b, above) to bcast[0..1].
-// Threads 0..127 own nbins / 128 consecutive bins each.
+// Threads 0..255 own nbins / 256 consecutive bins each (read at once, kept
+// in registers); a suffix scan over the lanes and the eight warps' totals
+// gives each thread the entries above its bins.
 __device__ void find_bin_block(const uint32_t* hist, int nbins, uint32_t need, Shared& sh, uint32_t* scratch) {
-  const int tid = threadIdx.x;
-  const int per = nbins / 128;
-  uint32_t mine = 0;
+  constexpr int kT = 256, kMaxPer = kHistBins / kT;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = nbins / kT;  // 1, 4 or 16
   // a histogram that holds fewer than `need` entries (never produced by the
   // kernel: the counts add up to the visible entries) selects bin 0
   if (tid == 0) {
     sh.bcast[0] = 0;
     sh.bcast[1] = 0;
   }
-  if (tid < 128)
-    for (int i = 0; i < per; i += 2) {
-      const uint2 v = *reinterpret_cast<const uint2*>(hist + tid * per + i);
-      mine += v.x + v.y;
-    }
-  if (tid < 128) scratch[tid] = mine;
-  __syncthreads();
-  if (tid < 32) {
-    uint32_t t4[4], s4 = 0;
+  uint32_t c[kMaxPer];
+  uint32_t mine = 0;
+  if (tid < kT) {
+    if (per >= 4) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      t4[q] = scratch[tid * 4 + q];
-      s4 += t4[q];
+      for (int i = 0; i < kMaxPer; i += 4)
+        if (i < per) {
+          const uint4 v = *reinterpret_cast<const uint4*>(hist + tid * per + i);
+          c[i] = v.x; c[i + 1] = v.y; c[i + 2] = v.z; c[i + 3] = v.w;
+        }
+    } else {
+      c[0] = hist[tid];
     }
-    uint32_t incl = s4;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
-      if (tid + o < 32) incl += v;
-    }
-    uint32_t above = incl - s4;
-#pragma unroll
-    for (int q = 3; q >= 0; --q) {
-      scratch[128 + tid * 4 + q] = above;
-      above += t4[q];
-    }
+    for (int i = 0; i < kMaxPer; ++i)
+      if (i < per) mine += c[i];
   }
+  uint32_t incl = mine;  // this thread's bins and those of the lanes above it
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += x;
+  }
+  if (tid < kT && lane == 0) scratch[warp] = incl;
   __syncthreads();
-  if (tid < 128) {
-    const uint32_t excl = scratch[128 + tid];
-    if (excl < need && need <= excl + mine) {
-      uint32_t above = excl;
-      for (int i = per - 1; i >= 0; --i) {
-        const uint32_t c = hist[tid * per + i];
-        if (above + c >= need) {
+  if (tid < kT) {
+    uint32_t above = incl - mine;
+    for (int w = warp + 1; w < kT / 32; ++w) above += scratch[w];
+    if (above < need && need <= above + mine) {
+#pragma unroll
+      for (int i = kMaxPer - 1; i >= 0; --i) {
+        if (i >= per) continue;
+        if (above + c[i] >= need) {
           sh.bcast[0] = tid * per + i;
           sh.bcast[1] = above;
           break;
         }
-        above += c;
+        above += c[i];
       }
     }
   }
