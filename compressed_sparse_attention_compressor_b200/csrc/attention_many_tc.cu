@@ -453,21 +453,28 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     const bool f32 = a.out_dtype == kF32;
     const int oeb = f32 ? 4 : 2;
     uint8_t* ost = Kt;  // 64 KB (bf16) or 128 KB (fp32)
+    // rolled over (block, head half) and one loop body per output type: this
+    // code runs once per CTA, and its instructions are fetched cold
 #pragma unroll 1
-    for (int mt = 2 * (warp >> 2); mt < 2 * (warp >> 2) + 2; ++mt) {
+    for (int i = 0; i < 4; ++i) {
+      const int mt = 2 * (warp >> 2) + (i >> 1), hh = (i & 1) * 32;
       const int dim = mt * 128 + q4 * 32 + lane;
-      uint32_t v0[32], v1[32];
+      uint32_t v[32];
       if (ntiles > 0) {
-        const uint32_t ta = dO + mt * kH + (static_cast<uint32_t>(q4 * 32) << 16);
-        tmem_ld32(ta, v0);
-        tmem_ld32(ta + 32, v1);
+        tmem_ld32(dO + mt * kH + hh + (static_cast<uint32_t>(q4 * 32) << 16), v);
         tmem_wait_ld();
-      }
+      } else {
 #pragma unroll
-      for (int h = 0; h < 64; ++h) {
-        const float o = ntiles > 0 ? __uint_as_float(h < 32 ? v0[h] : v1[h - 32]) * fin[h] : 0.f;
-        if (f32) reinterpret_cast<float*>(ost)[h * kD + dim] = o;
-        else reinterpret_cast<uint16_t*>(ost)[h * kD + dim] = f32_to_bf16_bits(o);
+        for (int h = 0; h < 32; ++h) v[h] = 0u;
+      }
+      if (f32) {
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          reinterpret_cast<float*>(ost)[(hh + h) * kD + dim] = __uint_as_float(v[h]) * fin[hh + h];
+      } else {
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          reinterpret_cast<uint16_t*>(ost)[(hh + h) * kD + dim] = f32_to_bf16_bits(__uint_as_float(v[h]) * fin[hh + h]);
       }
     }
     fence_proxy_async_smem();

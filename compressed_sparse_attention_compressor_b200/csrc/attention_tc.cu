@@ -248,18 +248,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     float* wgt = reinterpret_cast<float*>(smem + oS);  // [head][16 CTAs], then [head][2] (M, 1/L); logits are dead
     const int nh = (kH - split + R - 1) / R;
     const int dim = tid * 2;  // two consecutive dims per thread
-    // bf16 partials: the first four heads' loads from every peer go out
-    // before the weights are computed (their round trips overlap)
-    uint32_t vb[4][16];
-    auto load_bf = [&](int w0) {
+    // bf16 partials: thread t takes eight consecutive dims of one of the
+    // CTA's heads per round (task t + 256 i: head w = task / 64, dims
+    // 8 (task % 64) ..), one 16-byte load from every peer; the first round's
+    // loads go out before the weights are computed (their round trips overlap)
+    uint4 vb[16];
+    auto load_bf = [&](int task) {
+      const int w = task >> 6, d8 = (task & 63) * 8;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < R && w0 + u < nh)
-            vb[u][j] = cluster.map_shared_rank(Obf, j)[(split + (w0 + u) * R) * (kD / 2) + dim / 2];
+      for (int j = 0; j < 16; ++j)
+        if (j < R && w < nh)
+          vb[j] = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(Obf, j) + (split + w * R) * (kD / 2) + d8 / 2);
     };
-    if (pbf) load_bf(0);
+    if (pbf) load_bf(tid);
     for (int w = warp; w < nh; w += kThreads / 32) {
       const int h = split + w * R;
       float mj = -INFINITY, lj = 0.f;
@@ -282,24 +283,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnTcArgs a) {
     }
     __syncthreads();
     if (pbf) {
-      for (int w0 = 0; w0 < nh; w0 += 4) {
-        if (w0 > 0) load_bf(w0);
+      for (int task = tid; task < nh * 64; task += kThreads) {
+        if (task != tid) load_bf(task);
+        const int w = task >> 6, d8 = (task & 63) * 8, h = split + w * R;
+        float o[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int w = w0 + u;
-          if (w >= nh) break;
-          const int h = split + w * R;
-          float o0 = 0.f, o1 = 0.f;
+        for (int i = 0; i < 8; ++i) o[i] = 0.f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < R) {
-              const float wj = wgt[w * 16 + j];
-              o0 = fmaf(wj, __uint_as_float(vb[u][j] << 16), o0);
-              o1 = fmaf(wj, __uint_as_float(vb[u][j] & 0xFFFF0000u), o1);
+        for (int j = 0; j < 16; ++j)
+          if (j < R) {
+            const float wj = wgt[w * 16 + j];
+            const uint32_t u4[4] = {vb[j].x, vb[j].y, vb[j].z, vb[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              o[2 * i] = fmaf(wj, __uint_as_float(u4[i] << 16), o[2 * i]);
+              o[2 * i + 1] = fmaf(wj, __uint_as_float(u4[i] & 0xFFFF0000u), o[2 * i + 1]);
             }
-          const float inv = wgt[kH * 16 + w * 2 + 1];
-          const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + dim;
-          *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.out) + off) = pack_bf16(o0 * inv, o1 * inv);
+          }
+        const float inv = wgt[kH * 16 + w * 2 + 1];
+        const int64_t off = (static_cast<int64_t>(qi) * kH + h) * kD + d8;
+        const uint4 ov = make_uint4(pack_bf16(o[0] * inv, o[1] * inv), pack_bf16(o[2] * inv, o[3] * inv),
+                                    pack_bf16(o[4] * inv, o[5] * inv), pack_bf16(o[6] * inv, o[7] * inv));
+        uint16_t* dst = static_cast<uint16_t*>(a.out) + off;
+        if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+          *reinterpret_cast<uint4*>(dst) = ov;
+        } else {  // an output that is only 4-byte aligned
+          uint32_t* d4 = reinterpret_cast<uint32_t*>(dst);
+          d4[0] = ov.x; d4[1] = ov.y; d4[2] = ov.z; d4[3] = ov.w;
         }
       }
     } else {
