@@ -361,15 +361,21 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
     {
       uint8_t* prow = Pt + (row >> 6) * (kH * 128) + (row & 7) * 2;
       const uint32_t ch = (row & 63) >> 3;
+      // P for 16 heads at a time: their m log2 e into registers before the
+      // stores (a shared-memory load after a shared-memory store waits for it)
 #pragma unroll
-      for (int h = 0; h < 32; h += 4) {
-        const float4 m4 = *reinterpret_cast<const float4*>(ml2 + hb + h);
-        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+      for (int h0 = 0; h0 < 32; h0 += 16) {
+        float mm[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p = row_ok ? ex2_approx(fmaf(s[h + u], kLog2e, -mm[u])) : 0.f;
-          s[h + u] = p;
-          *reinterpret_cast<uint16_t*>(prow + sw128_offset(hb + h + u, ch)) = f32_to_bf16_bits(p);
+        for (int h = 0; h < 16; h += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(ml2 + hb + h0 + h);
+          mm[h] = m4.x; mm[h + 1] = m4.y; mm[h + 2] = m4.z; mm[h + 3] = m4.w;
+        }
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+          const float p = row_ok ? ex2_approx(fmaf(s[h0 + h], kLog2e, -mm[h])) : 0.f;
+          s[h0 + h] = p;
+          *reinterpret_cast<uint16_t*>(prow + sw128_offset(hb + h0 + h, ch)) = f32_to_bf16_bits(p);
         }
       }
     }
@@ -467,14 +473,23 @@ attn_many_tc_kernel(const __grid_constant__ CUtensorMap qmap, AttnManyArgs a) {
 #pragma unroll
         for (int h = 0; h < 32; ++h) v[h] = 0u;
       }
+      // the scales into registers before the first store (a shared-memory
+      // load after a shared-memory store waits for it)
+      float o[32];
+#pragma unroll
+      for (int h = 0; h < 32; h += 4) {
+        const float4 f4 = *reinterpret_cast<const float4*>(fin + hh + h);
+        o[h] = __uint_as_float(v[h]) * f4.x;
+        o[h + 1] = __uint_as_float(v[h + 1]) * f4.y;
+        o[h + 2] = __uint_as_float(v[h + 2]) * f4.z;
+        o[h + 3] = __uint_as_float(v[h + 3]) * f4.w;
+      }
       if (f32) {
 #pragma unroll
-        for (int h = 0; h < 32; ++h)
-          reinterpret_cast<float*>(ost)[(hh + h) * kD + dim] = __uint_as_float(v[h]) * fin[hh + h];
+        for (int h = 0; h < 32; ++h) reinterpret_cast<float*>(ost)[(hh + h) * kD + dim] = o[h];
       } else {
 #pragma unroll
-        for (int h = 0; h < 32; ++h)
-          reinterpret_cast<uint16_t*>(ost)[(hh + h) * kD + dim] = f32_to_bf16_bits(__uint_as_float(v[h]) * fin[hh + h]);
+        for (int h = 0; h < 32; ++h) reinterpret_cast<uint16_t*>(ost)[(hh + h) * kD + dim] = f32_to_bf16_bits(o[h]);
       }
     }
     fence_proxy_async_smem();
