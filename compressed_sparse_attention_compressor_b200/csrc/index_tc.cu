@@ -379,30 +379,6 @@ __device__ __forceinline__ void block_rank2(bool f0, bool f1, uint32_t& r0, uint
   __syncthreads();
 }
 
-// One warp: in-place exclusive prefix sums of v[0..n); returns the total
-// (valid in every lane).
-__device__ uint32_t warp_scan_inplace(uint32_t* v, int n) {
-  const int lane = threadIdx.x & 31;
-  const int seg = (n + 31) / 32;
-  const int lo = min(n, lane * seg), hi = min(n, lo + seg);
-  uint32_t mine = 0;
-  for (int i = lo; i < hi; ++i) mine += v[i];
-  uint32_t incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += x;
-  }
-  uint32_t run = incl - mine;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t x = v[i];
-    v[i] = run;
-    run += x;
-  }
-  __syncwarp();
-  return __shfl_sync(0xFFFFFFFFu, incl, 31);
-}
-
 // Whole block: a global histogram of kHistBins words into shared memory,
 // every load issued before the first store.
 __device__ __forceinline__ void load_hist(uint32_t* dst, const uint32_t* src) {
@@ -1064,9 +1040,13 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       uint32_t* bar = a.sync + r * 4;
       uint32_t nbar = 1;
       // level 1 (bits 31..20): the histogram built while streaming
-      for (int i = tid; i < kHistBins; i += kThreads) {
-        const uint32_t v = gh_g[i] + gh_g[kHistBins + i];
-        if (v) atomicAdd(&gh1[i], v);
+      for (int i = tid; i < kHistBins / 4; i += kThreads) {
+        const uint4 x = reinterpret_cast<const uint4*>(gh_g)[i];
+        const uint4 y = reinterpret_cast<const uint4*>(gh_g + kHistBins)[i];
+        const uint32_t v[4] = {x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (v[e]) atomicAdd(&gh1[4 * i + e], v[e]);
       }
       // arrive, copy the scores while the request's slower CTAs finish, wait
       request_arrive(&bar[0], static_cast<int>(blockIdx.x) == a.skip_arrive);
@@ -1147,19 +1127,38 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       }
       if (alive) {
         // ---- every CTA: chunk offsets, then its own share of the output ----
+        // chunk counts straight into registers (warp 0: above, warp 1: at
+        // the boundary; lane l holds chunks 5 l .. 5 l + 4), exclusive prefix
+        // sums by a lane scan, written with the total at [nch]
         const uint2* cnt = reinterpret_cast<const uint2*>(a.cnt) + static_cast<int64_t>(r) * nch;
-        for (int i = tid; i < nch; i += kThreads) {
-          const uint2 ce = __ldcg(cnt + i);
-          preA[i] = ce.x;
-          preE[i] = ce.y;
-        }
-        __syncthreads();
-        if (warp == 0) {
-          const uint32_t ta = warp_scan_inplace(preA, nch);
-          if (lane == 0) preA[nch] = ta;
-        } else if (warp == 1) {
-          const uint32_t te = warp_scan_inplace(preE, nch);
-          if (lane == 0) preE[nch] = te;
+        static_assert(kMaxChunks <= 5 * 32, "five chunks per lane");
+        if (warp < 2) {
+          uint32_t v[5], mine = 0;
+#pragma unroll
+          for (int u = 0; u < 5; ++u) {
+            const int i = lane * 5 + u;
+            v[u] = 0u;
+            if (i < nch) {
+              const uint2 ce = __ldcg(cnt + i);
+              v[u] = warp == 0 ? ce.x : ce.y;
+            }
+            mine += v[u];
+          }
+          uint32_t incl = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += x;
+          }
+          uint32_t* pre = warp == 0 ? preA : preE;
+          uint32_t run = incl - mine;
+#pragma unroll
+          for (int u = 0; u < 5; ++u) {
+            const int i = lane * 5 + u;
+            if (i < nch) pre[i] = run;
+            run += v[u];
+          }
+          if (lane == 31) pre[nch] = incl;
         }
         __syncthreads();
         const uint32_t A_tot = preA[nch], E_tot = preE[nch];
