@@ -19,9 +19,10 @@
 //     (A operand, M = 128, K = 128, 128-byte swizzle);
 //   * per tile the MMA issuer writes D_G[128 keys][256] = K_tile Q_G^T into
 //     TMEM accumulator G (G = 0, 1; 2 x 256 columns), and the epilogue group
-//     G (four warps, one TMEM lane quarter each) reduces each key's row:
-//     s = sum_h w_h ReLU(D[h]) for each of its 4 queries, and stores the
-//     score of every key the query sees (causal: j < n_visible[i]).
+//     G (eight warps: a TMEM lane quarter and two of the half's four queries
+//     each) reduces each key's row: s = sum_h w_h ReLU(D[h]) for each of its
+//     queries, and stores the score of every key the query sees (causal:
+//     j < n_visible[i]).
 //     Accumulator G is released as soon as it is read, so the MMAs of the
 //     other half run while one half is reduced;
 //   * the work -- every (group, key tile) pair, groups in query order and
@@ -49,7 +50,8 @@ constexpr int kN = kQH * kHeads;               // 256: MMA N, TMEM columns per a
 constexpr int kStages = 3;
 constexpr int kStageBytes = kTile * kDI * 2;   // 32 KB: two 16 KB K halves of 128 rows x 128 B
 constexpr int kQBytes = kQG * kHeads * kDI * 2;  // 128 KB: two 64 KB K halves of 512 rows x 128 B
-constexpr int kThreads = 320;                  // producer warp, MMA warp, 8 epilogue warps
+constexpr int kEpiPerGroup = 8;                // epilogue warps per accumulator: 4 lane quarters x 2 query pairs
+constexpr int kThreads = 32 * (2 + 2 * kEpiPerGroup);  // producer warp, MMA warp, 16 epilogue warps
 constexpr uint32_t kTmemCols = 2 * kN;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int G = 0; G < 2; ++G) {
       mbar_init(&tfull[G], 1);
-      mbar_init(&tempty[G], 4 * 32);
+      mbar_init(&tempty[G], kEpiPerGroup * 32);
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -323,8 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mdone, 0, kWaitLimit);
     }
   } else {
-    // epilogue: group G = warps 2-5 / 6-9, warp w reads TMEM lanes 32 (w % 4) ..
-    const int G = (warp - 2) >> 2, sub = warp & 3;
+    // epilogue: group G = warps 2-9 / 10-17; warp w of a group reads TMEM
+    // lanes 32 (w % 4) .. + 31 for the queries 2 (w / 4), + 1 of the half
+    const int G = (warp - 2) / kEpiPerGroup, sub = warp & 3, qp = ((warp - 2) % kEpiPerGroup) >> 2;
     const int row = sub * 32 + lane;
     const uint32_t lane_addr = tmem + G * kN + (static_cast<uint32_t>(sub * 32) << 16);
     for (int i = 0; i < n_tiles && !*fail; ++i) {
@@ -341,10 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = cur.first_query() + G * kQH;
       const int nqh = min(kQH, cur.queries() - G * kQH);  // queries of this half (may be <= 0)
       const int64_t key = static_cast<int64_t>(cur.lt) * kTile + row;
-      float sc[kQH];
+      float sc[2];
 #pragma unroll
-      for (int qq = 0; qq < kQH; ++qq) {
-        sc[qq] = 0.f;
+      for (int u = 0; u < 2; ++u) {
+        const int qq = 2 * qp + u;
+        sc[u] = 0.f;
         if (qq < nqh) {  // warp-uniform
           uint32_t v0[32], v1[32];
           tmem_ld32(lane_addr + qq * kHeads, v0);
@@ -364,18 +368,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             s2 = fmaf(wb.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), s2);
             s3 = fmaf(wb.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), s3);
           }
-          sc[qq] = (s0 + s1) + (s2 + s3);
+          sc[u] = (s0 + s1) + (s2 + s3);
         }
       }
       // every column of the accumulator this warp reads is in registers
       tc_fence_before();
       mbar_arrive(&tempty[G]);
 #pragma unroll
-      for (int qq = 0; qq < kQH; ++qq) {
+      for (int u = 0; u < 2; ++u) {
+        const int qq = 2 * qp + u;
         if (qq >= nqh) break;
         const int qi = q0 + qq;
         const int64_t nv = min(max(static_cast<int64_t>(__ldg(a.n_visible + qi)), int64_t(0)), a.cap);
-        if (key < nv) a.scores[static_cast<int64_t>(qi) * a.ld + key] = sc[qq];
+        if (key < nv) a.scores[static_cast<int64_t>(qi) * a.ld + key] = sc[u];
       }
     }
   }
