@@ -270,7 +270,8 @@ int topk_multi_ctas(int n_rows, int64_t max_n) {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 0;
-  if (n_rows < 1 || max_n < 32768) return 0;  // shorter rows: one CTA is faster
+  // rows of up to 65,536 scores: one CTA per row (its candidate form) is faster
+  if (n_rows < 1 || max_n <= 65536) return 0;
   const int64_t need = (max_n + kMSeg - 1) / kMSeg;
   int64_t G = (max_n + 4095) / 4096;
   if (G < need) G = need;

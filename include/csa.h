@@ -190,7 +190,7 @@ csa_status_t csa_index_score(const csa_params_t* p, int32_t n_queries, const csa
  *   scores   [n_rows][ld] fp32; row i has n_valid[i] (<= ld) valid columns.
  *   out_idx  [n_rows][k] int32 (-1 padded), out_score optional.
  *   workspace  optional: with at least csa_topk_workspace_size(n_rows)
- *            bytes, rows of 32,768 or more columns are each split over
+ *            bytes, rows of more than 65,536 columns are each split over
  *            several CTAs (same result); without it one CTA takes a row.   */
 csa_status_t csa_topk(const float* scores, int32_t n_rows, int64_t ld, const int32_t* n_valid,
                       int32_t k, int32_t* out_idx, float* out_score, void* workspace,

@@ -27,7 +27,7 @@ def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, multi, cuda_lib):
     scores = torch.from_numpy(buf).cuda()
     out_idx = torch.full((rows, k), -7, dtype=torch.int32, device="cuda")
     out_score = torch.empty((rows, k), dtype=torch.float32, device="cuda")
-    # with a workspace, rows of 32,768+ columns are split over several CTAs
+    # with a workspace, rows of more than 65,536 columns are split over several CTAs
     ws = csa.workspace(csa.csa_topk_workspace_size(rows)) if multi else None
     csa.csa_topk(scores, rows, ld, i32(n_valid), k, out_idx, out_score, ws)
     torch.cuda.synchronize()
@@ -41,9 +41,9 @@ def test_topk_alone_is_bit_exact_with_ties(k, n_cols, pad, multi, cuda_lib):
         assert np.all(np.isneginf(gs[r][~sel]))
 
 
-@pytest.mark.parametrize("n", [5000, 40000])
+@pytest.mark.parametrize("n", [5000, 70000])
 def test_topk_all_equal_scores_takes_lowest_indices(n, cuda_lib):
-    """40,000 columns with a workspace: the rows are split over CTAs."""
+    """70,000 columns with a workspace: the rows are split over CTAs."""
     k = 300
     scores = torch.zeros((2, n), dtype=torch.float32, device="cuda")
     scores[1, ::2] = -0.0

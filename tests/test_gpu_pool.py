@@ -98,8 +98,8 @@ EXACT = {
     "bf16_b8": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 3, 3, 6000 + 3, 8, 96),
     "bf16_b128": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 2, 2, 9000, 128, 7),
     "bf16_b32_many_chunks": (Wk.WORKLOADS["decode64k"].scaled(topk=256), 2, 2, 150000, 32, 300),
-    # 40,000 single-entry blocks per query: the pool is selected by several CTAs per query (>= 32,768)
-    "bf16_b1_long_rows": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 2, 2, 40000, 1, 3000),
+    # 70,000 single-entry blocks per query: the pool is selected by several CTAs per query (> 65,536)
+    "bf16_b1_long_rows": (Wk.WORKLOADS["decode64k"].scaled(topk=128), 2, 2, 70000, 1, 3000),
 }
 
 
