@@ -10,20 +10,25 @@
 // attends to the selected entries together with the sliding-window KV).
 //
 // Per tile (attn_tile.cuh's layouts):
-//   1. gather: key rows -> bf16, K-major 128-byte swizzled tile (all warps);
-//   2. S^T[128 keys][64 heads] = K Q^T (tcgen05, M = 128, N = 64, K = 512);
-//      the query (64 KB) was loaded once by TMA;
-//   3. warps 4-7 read S^T from TMEM (a key per thread, 64 heads in
-//      registers), reduce the tile's per-head maximum across the keys with
-//      a transposing butterfly, and write P^T = exp(S - m) as bf16; warps
-//      0-3 meanwhile replace the window rows' keys with their values;
+//   1. gather: key rows -> bf16, K-major 128-byte swizzled tile, in eight
+//      64-dim column blocks (all warps, asynchronous copies);
+//   2. S^T[128 keys][64 heads] = K Q^T (tcgen05, M = 128, N = 64, K = 512),
+//      each block's four MMAs issued as soon as every thread's copies of the
+//      block have landed; the query (64 KB) was loaded once by TMA;
+//   3. all eight warps read S^T from TMEM (warp w: keys 32 (w % 4) .. + 31,
+//      heads 32 (w / 4) .. + 31, a key per thread), and write
+//      P^T = exp(S - m) as bf16; the window rows' values replace their keys
+//      by asynchronous copies meanwhile;
 //   4. O^T[512][64] += V^T P^T (tcgen05, the tile as an MN-major A operand),
 //      accumulated in TMEM over all tiles.
 // The running maximum m is updated lazily: a head's m moves only when a
-// tile's maximum exceeds it by more than kLazy (P <= e^kLazy meanwhile,
-// exact in bf16's range), and only then is its column of O rescaled in
-// TMEM.  The sink enters the denominator once at the end; out = O / L and
-// lse = M + log L exactly as in the single-tile kernels.
+// logit exceeds it by more than kLazy (P <= e^kLazy meanwhile, exact in
+// bf16's range; the tile's per-head maxima are reduced across the keys, by
+// a transposing warp butterfly, only in tiles where some logit does), and
+// only then is its column of O rescaled in TMEM.  The sink enters the
+// denominator once at the end; out = O / L and lse = M + log L exactly as
+// in the single-tile kernels; the output block is staged in shared memory
+// and leaves by bulk stores.
 #include <cudaTypedefs.h>
 
 #include "attn_tile.cuh"

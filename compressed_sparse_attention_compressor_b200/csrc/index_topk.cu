@@ -11,10 +11,13 @@
 //
 // Top-k order: score descending; among exactly equal scores the lower index
 // wins (-0 == +0).  The selection is a radix select on the ordered 32-bit
-// key of each fp32 score (three histogram passes of 11/11/10 bits), which
-// yields the exact k-th key T and the number r of entries equal to T that
-// are kept; an index-ordered pass then takes every entry above T and the r
-// lowest-index entries equal to T.
+// key of each fp32 score (histogram levels of up to 2,048 bins over the
+// keys' own range), which yields the exact k-th key T and the number r of
+// entries equal to T that are kept; an index-ordered pass then takes every
+// entry above T and the r lowest-index entries equal to T.  The row kernel
+// first keeps, in shared memory, the candidates that reach a threshold
+// taken from a sample of the row and runs the levels over them; a row whose
+// candidates do not fit (or fall short of k) takes them over the whole row.
 #include "common.cuh"
 
 namespace csa {
