@@ -255,7 +255,8 @@ __device__ bool request_barrier(uint32_t* ctr, uint32_t target, uint32_t limit, 
 
 // Whole block: bin b of a shared-memory histogram of `nbins` bins (a power
 // of two, 256..kHistBins), scanned from the top, with
-// above(b) < need <= above(b) + hist[b]; writes (b, above) to bcast[0..1].
+// above(b) < need <= above(b) + hist[b]; writes (b, above, hist[b]) to
+// bcast[0..2].
 // Threads 0..255 own nbins / 256 consecutive bins each (read at once, kept
 // in registers); a suffix scan over the lanes and the eight warps' totals
 // gives each thread the entries above its bins.
@@ -268,6 +269,7 @@ __device__ void find_bin_block(const uint32_t* hist, int nbins, uint32_t need, S
   if (tid == 0) {
     sh.bcast[0] = 0;
     sh.bcast[1] = 0;
+    sh.bcast[2] = 0;
   }
   uint32_t c[kMaxPer];
   uint32_t mine = 0;
@@ -304,6 +306,7 @@ __device__ void find_bin_block(const uint32_t* hist, int nbins, uint32_t need, S
         if (above + c[i] >= need) {
           sh.bcast[0] = tid * per + i;
           sh.bcast[1] = above;
+          sh.bcast[2] = c[i];
           break;
         }
         above += c[i];
@@ -1198,11 +1201,15 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             }
           }
           __syncthreads();
-          // radix levels over the low `shift` key bits (10 + 10, or 8): the
-          // take-th largest key T and how many entries equal to T are taken
+          // radix levels over the low `shift` key bits (12 + 8, or 8): the
+          // take-th largest key T and how many entries equal to T are taken.
+          // A level whose chosen bin is taken whole (usual after 12 bits: a
+          // few thousand entries over 4,096 bins) ends the search: T is then
+          // the key just below that bin and no entry equal to T is taken
           uint32_t pfx = prefix, rb = shift, tk = take;
+          bool whole = false;
           while (rb > 0) {
-            const uint32_t nb = rb > 10 ? 10 : rb;
+            const uint32_t nb = rb > 12 ? 12 : rb;
             const uint32_t sft = rb - nb;
             for (int i = tid; i < (1 << nb); i += kThreads) hist[i] = 0;
             __syncthreads();
@@ -1212,11 +1219,17 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
             }
             __syncthreads();
             find_bin_block(hist, 1 << nb, tk, sh, scratch);
-            pfx = (pfx << nb) | sh.bcast[0];
+            const uint32_t bsel = sh.bcast[0];
+            pfx = (pfx << nb) | bsel;
             tk -= sh.bcast[1];
             rb = sft;
+            if (rb > 0 && sh.bcast[2] == tk && (pfx << rb) != 0u) {
+              whole = true;
+              break;
+            }
           }
-          const uint32_t T = pfx;
+          const uint32_t T = whole ? (pfx << rb) - 1u : pfx;
+          if (whole) tk = 0;
           // taken: key > T, and the first tk (lowest indices) with key == T
           const uint32_t e0 = preE[c], e1 = preE[c + 1];
           uint32_t g = 0, q = 0;
