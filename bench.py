@@ -310,23 +310,32 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: K back-to-back steps on rotating cache copies ----
+    # ---- timed region: K back-to-back steps on rotating cache copies, one
+    # event pair around all of them (the K steps' device time, gaps included) ----
     K = args.steps
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         head_start()
+        t_start.record(stream)
         for i in range(K):
-            e0[i].record(stream)
             step(i)
-            e1[i].record(stream)
+        t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
-    step_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
-    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, "cuda")
     ms_per_step = total_ms / K
+    # the spread of single steps: the same K steps with an event pair around each
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    head_start()
+    for i in range(K):
+        e0[i].record(stream)
+        step(i)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
 
     # ---- per-kernel times: the same K steps with events around every launch ----
     csa.csa_profile_start(64 * K)
