@@ -102,7 +102,7 @@ struct Cfg {
   static constexpr int kSmem = oMisc + 256 + 1024;
   // FP8: N = 128 = both E4M3 terms of the split query (rows 0..63 and 64..127 of B)
   static constexpr uint32_t kIdesc = FP8 ? idesc(0, 0, kTileM, 2 * kHeads) : idesc(1, 1, kTileM, kHeads);
-  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 7) <= 512, "mbarrier area");
+  static_assert(sizeof(uint64_t) * (2 * kStages + 2 * kSStages + 8) <= 512, "mbarrier area");
   static_assert(oB % 1024 == 0, "operand alignment");
   static_assert(kSmem <= 232448, "shared memory");
   // phase-2 scratch, inside the (then idle) stage and scale rings
@@ -569,6 +569,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   uint64_t* qbar = tempty + 2;
   uint64_t* mdone = qbar + 1;
   uint64_t* abar = mdone + 1;  // W_IK of the in-kernel append
+  uint64_t* cbar = abar + 1;   // the chunk's scores, workspace -> shared memory (phase 2)
   uint8_t* Bs = smem + C::oB;
   const float* scale_ring = reinterpret_cast<const float*>(smem + C::oScales);
 
@@ -621,6 +622,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     mbar_init(qbar, 1);
     mbar_init(mdone, 1);
     mbar_init(abar, 1);
+    mbar_init(cbar, 1);
     sh.fail = 0;
     fence_barrier_init();
   }
@@ -958,6 +960,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
       }
     }
   }
+  // the staged scores come back by a bulk copy (the async proxy) in phase 2
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -991,21 +995,16 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
     // scores TMEM -> shared memory in index order: warps 2..9, two per lane quarter
     // the chunk's scores, workspace -> shared memory in index order (the
     // block's own writes of phase 1, ordered by the barrier after it)
+    // (one bulk copy of the chunk's nt x 512 contiguous bytes, waited for by
+    // every thread)
     auto copy_scores = [&]() {
-      const float4* src =
-          reinterpret_cast<const float4*>(a.scg + (static_cast<int64_t>(r) * a.chunks + c) * (kMaxChunkTiles * kTileM));
-      float4* dst = reinterpret_cast<float4*>(sc);
-      const int n4 = nt * (kTileM / 4);
-      constexpr int U = 4;
-      for (int i0 = tid; i0 < n4; i0 += U * kThreads) {
-        float4 v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (i0 + u * kThreads < n4) v[u] = __ldcg(src + i0 + u * kThreads);
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (i0 + u * kThreads < n4) dst[i0 + u * kThreads] = v[u];
+      if (nt <= 0) return;
+      if (tid == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(nt) * kTileM * 4;
+        mbar_arrive_expect_tx(cbar, bytes);
+        bulk_load(sc, a.scg + (static_cast<int64_t>(r) * a.chunks + c) * (kMaxChunkTiles * kTileM), bytes, cbar);
       }
+      if (!mbar_wait(cbar, 0, kWaitLimit)) atomicOr(&g_index_tc_error, 1u);
     };
     // block maxima of the chunk (the chunk starts on a tile, so on a block)
     auto write_block_max = [&]() {
